@@ -1,0 +1,113 @@
+"""Pins for oracle/awq.py and oracle/nvfp4.py: round trips, exact special
+cases, error bounds of the rounding rules, and torch conversions."""
+
+import numpy as np
+import torch
+
+from oracle import awq, formats, nvfp4
+
+
+def test_awq_pack_layout_and_round_trip():
+    codes = np.arange(1, 9).reshape(1, 8)
+    w = awq.pack_nibbles(codes)
+    assert w.view(np.uint32)[0, 0] == 0x87654321
+    rng = np.random.default_rng(0)
+    c = rng.integers(0, 16, (64, 96))
+    assert np.array_equal(awq.unpack_nibbles(awq.pack_nibbles(c)), c)
+    words = rng.integers(-2 ** 31, 2 ** 31, (7, 5), dtype=np.int64).astype(np.int32)
+    assert np.array_equal(awq.pack_nibbles(awq.unpack_nibbles(words)), words)
+
+
+def _awq_case(rng, K=64, N=32, lo_scale=0.0):
+    q = rng.integers(0, 16, (K, N))
+    z = rng.integers(0, 16, (K // 32, N))
+    s = np.abs(rng.standard_normal((K // 32, N)) * 0.02).astype(np.float16)
+    if lo_scale:
+        s = np.maximum(s, np.float16(lo_scale))
+    return q, z, s
+
+
+def test_awq_dequant_zero_at_zero_point_and_vs_torch_half():
+    rng = np.random.default_rng(1)
+    q, z, s = _awq_case(rng)
+    W = awq.dequant(awq.pack_nibbles(q), awq.pack_nibbles(z), s)
+    g = np.arange(q.shape[0]) // 32
+    # (q - z) * s with q = z is exactly zero
+    qz = z[g]
+    assert np.all(awq.dequant(awq.pack_nibbles(qz), awq.pack_nibbles(z), s) == 0)
+    # exact product in float32, rounded once to half by torch
+    prod = torch.from_numpy((q - z[g]).astype(np.float32) * s[g].astype(np.float32))
+    assert np.array_equal(W, prod.to(torch.float16).double().numpy())
+
+
+def test_awq_quantize_inverts_dequant_and_error_bound():
+    rng = np.random.default_rng(2)
+    q, z, s = _awq_case(rng, K=128, N=64, lo_scale=2.0 ** -10)
+    W = awq.dequant(awq.pack_nibbles(q), awq.pack_nibbles(z), s)
+    assert np.array_equal(awq.quantize(W, s, z), q)
+    # in-range weights come back within half a step
+    g = np.arange(128) // 32
+    lo = (0 - z[g]) * s[g].astype(np.float64)
+    hi = (15 - z[g]) * s[g].astype(np.float64)
+    w = lo + rng.uniform(0, 1, lo.shape) * (hi - lo)
+    qq = awq.quantize(w, s, z)
+    back = (qq - z[g]) * s[g].astype(np.float64)
+    assert np.all(np.abs(back - w) <= 0.5 * s[g].astype(np.float64) * (1 + 1e-12))
+    # clipping outside the code range
+    assert np.all(awq.quantize(lo - 10 * s[g].astype(np.float64), s, z) == 0)
+    assert np.all(awq.quantize(hi + 10 * s[g].astype(np.float64), s, z) == 15)
+
+
+def test_nvfp4_pack_layout():
+    c = np.array([[1, 2, 3, 4]], np.uint8)
+    assert list(nvfp4.pack(c)[0]) == [0x21, 0x43]
+    rng = np.random.default_rng(3)
+    cc = rng.integers(0, 16, (5, 32)).astype(np.uint8)
+    assert np.array_equal(nvfp4.unpack(nvfp4.pack(cc)), cc)
+
+
+def test_nvfp4_zero_tensor_and_zero_block():
+    c, sb, g = nvfp4.quantize(np.zeros((3, 32), np.float32))
+    assert g == 0 and np.all(c == 0) and np.all(sb == 0)
+    v = np.random.default_rng(4).standard_normal((2, 48)).astype(np.float32)
+    v[1, 16:32] = 0
+    c, sb, g = nvfp4.quantize(v)
+    assert np.all(c[1, 16:32] == 0) and sb[1, 1] == 0
+
+
+def test_nvfp4_grid_values_round_trip_exactly():
+    # s_g a power of two, block scales E4M3 values, elements on the E2M1
+    # grid, each block holding a +-6 element: every division is exact
+    rng = np.random.default_rng(5)
+    rows, K = 8, 64
+    s_g = np.float32(2.0 ** -12)
+    sb_codes = rng.integers(0x20, 0x7F, (rows, K // 16)).astype(np.uint8)
+    sb_codes[0, 0] = 0x7E  # one block at 448, so amax = 6 * 448 * s_g
+    ecodes = rng.integers(0, 16, (rows, K)).astype(np.uint8)
+    ecodes[:, ::16] = 0x7  # +6 in every block
+    v = nvfp4.dequant(ecodes, sb_codes, s_g).astype(np.float32)
+    c, sb, g = nvfp4.quantize(v)
+    assert g == s_g
+    assert np.array_equal(sb, sb_codes)
+    # -0 and +0 decode equal; compare values
+    assert np.array_equal(formats.e2m1_to_f64(c), formats.e2m1_to_f64(ecodes))
+
+
+def test_nvfp4_error_bound_and_block_max():
+    rng = np.random.default_rng(6)
+    v = (rng.standard_normal((64, 256)) * np.exp(rng.standard_normal((64, 1)))).astype(np.float32)
+    c, sb, g = nvfp4.quantize(v)
+    back = nvfp4.dequant(c, sb, g)
+    scale = np.repeat(formats.e4m3_to_f64(sb), 16, axis=1) * np.float64(g)
+    # the largest E2M1 gap is 2 (between 4 and 6): error <= 1 step-scale
+    assert np.all(np.abs(back - v) <= 1.0 * scale * (1 + 1e-6))
+    # the tensor's largest element lands on code +-6 at block scale 448
+    i = np.unravel_index(np.argmax(np.abs(v)), v.shape)
+    assert sb[i[0], i[1] // 16] == 0x7E
+    assert (c[i] & 0x7) == 0x7
+
+
+def test_nvfp4_static_scale_saturates():
+    v = np.array([[100.0] + [0.0] * 15], np.float32)
+    c, sb, g = nvfp4.quantize(v, s_g=np.float32(1e-3))  # 6*448*1e-3 = 2.688 < 100
+    assert sb[0, 0] == 0x7E and c[0, 0] == 0x7
