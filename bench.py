@@ -1,0 +1,399 @@
+#!/usr/bin/env python3
+"""Throughput of the routed-expert MoE layer on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic tokens:
+router GEMM + softmax/top-k + renormalisation, permutation by expert, grouped
+SwiGLU experts (gate/up + SwiGLU, down), the shared expert, and the weighted
+combine (the Refill workload adds the Refill-RMS accumulation and the
+selection).  The default workload is the BF16 layer at Flash-Next shape in
+prefill: T=8192 tokens, H=2048, E=512 experts, top-10, expert width 640, one
+shared expert of width 640.
+
+`value` is whole-job tokens/s (tokens of all ranks / the slowest rank's
+time), timed with CUDA events on the launching stream over exactly K steps
+with inputs resident in HBM.  `e2e` repeats the measurement through the same
+public API with the token batch copied from pinned host memory and the layer
+output copied back inside every step.  Under torchrun every rank runs its own
+batch (weak scaling; the forward has no collective).
+
+--impl reference times the CPU oracle (oracle/, float64 NumPy) on a bounded
+sample of the same workload on this machine's host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_expert_gemm_b200 import MoELayer, abi, synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at E=512,k=10 (prefill TFLOP/s & decode HBM GB/s vs roofline)"
+L2_BYTES = 126 * 1024 * 1024
+
+# name -> (synth workload, T, kind)
+WORKLOADS = {
+    "bf16_prefill": ("bf16", 8192, "forward"),
+    "bf16_decode_t1": ("bf16", 1, "forward"),
+    "bf16_decode_t8": ("bf16", 8, "forward"),
+    "bf16_decode_t64": ("bf16", 64, "forward"),
+    "bf16_h2560_prefill": ("bf16_h2560", 8192, "forward"),
+    "refill": ("refill", 32768, "refill"),
+}
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="bf16_prefill", choices=sorted(WORKLOADS))
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-tokens", type=int, default=0, help="oracle sample size (0: automatic)")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; no collective in the data path)
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.barrier()
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks() -> dict:
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        return {}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline; also the --impl reference arm)
+# ---------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_tokens_per_s(wl, w, x: torch.Tensor, n_tokens: int, kind: str):
+    """Runs the float64 oracle on the first n_tokens tokens; returns (tokens/s, seconds)."""
+    from oracle import moe, razor
+
+    I = wl.I
+
+    def to64(t):
+        return t.detach().float().cpu().double().numpy()
+
+    cache = {}
+
+    def ew(e):
+        if e not in cache:
+            g = to64(w["w_gate_up"][e])
+            cache[e] = (g[:I], g[I:], to64(w["w_down"][e]))
+        return cache[e]
+
+    xs = to64(x[:n_tokens])
+    wr, b = to64(w["w_router"]), to64(w["bias"])
+    sh = to64(w["w_sh_gate_up"])
+    shared = (sh[: wl.I_sh], sh[wl.I_sh:], to64(w["w_sh_down"]))
+    t0 = time.perf_counter()
+    if kind == "refill":
+        out = moe.moe_layer(xs, wr, b, wl.k, ew, shared, extra=1)
+        r = out["route"]
+        d = razor.refill_deltas_closed_form(out["f"], out["perm"]["slot_row"], r["idx"], r["p"], wl.k)
+        s, c = np.zeros(wl.E), np.zeros(wl.E, np.int64)
+        razor.accumulate(s, c, d, r["idx"], wl.k)
+        razor.select(s, c, wl.keep)
+    else:
+        moe.moe_layer(xs, wr, b, wl.k, ew, shared)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt
+
+
+# ---------------------------------------------------------------------------
+def expert_flops(rows: int, H: int, I: int) -> float:
+    return 2.0 * rows * 3 * H * I
+
+
+def run_native(args, dist: Dist) -> None:
+    wname, T, kind = WORKLOADS[args.workload]
+    wl = synth.WORKLOADS[wname]
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    w = synth.make_weights(wl, seed=0, device=dev)
+    extra = 1 if kind == "refill" else 0
+    layer = MoELayer(w, wl.k, wl.fmt, T_max=T, extra=extra)
+    # token batches: distinct per rank, rotated so that the inputs of the
+    # timed steps exceed the L2 cache
+    x_bytes = T * wl.H * 2
+    n_batches = max(2, min(8, -(-2 * L2_BYTES // x_bytes)))
+    xs = [synth.make_tokens(wl, T, seed=1 + dist.rank, batch=b, device=dev) for b in range(n_batches)]
+    sum_sq = torch.zeros(wl.E, dtype=torch.float64, device=dev)
+    count = torch.zeros(wl.E, dtype=torch.int64, device=dev)
+    kept = torch.empty(max(wl.keep, 1), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    ffn_ev = []
+
+    def step(i: int, record: bool):
+        x = xs[i % n_batches]
+        if kind == "refill":
+            layer.route(x)
+        else:
+            layer.route(x)
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        f = layer.experts(x)
+        if record:
+            e1.record(stream)
+            ffn_ev.append((e0, e1))
+        sh = layer.shared_expert(x)
+        if kind == "refill":
+            abi.razor_refill_rms_accumulate(f, layer.slot_row[:T], layer.topk_idx[:T], layer.topk_logit[:T],
+                                            layer.offsets, sum_sq, count, shared_out=sh, y_out=layer.y[:T],
+                                            ws=layer.ws_refill)
+            abi.razor_select(sum_sq, count, wl.keep, kept=kept)
+        else:
+            abi.moe_combine(f, layer.slot_row[:T], layer.topk_w[:T], shared_out=sh, y=layer.y[:T])
+
+    for i in range(args.warmup):
+        step(i, False)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0, "device status after warm-up"
+
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dist.local)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, True)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    ms_local = t_start.elapsed_time(t_end) / args.steps
+    ms = dist.max(ms_local)
+    ffn_ms = statistics.mean(a.elapsed_time(b) for a, b in ffn_ev)
+    ffn_ms = dist.max(ffn_ms)
+    status = abi.moe_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    rows = T * (wl.k + extra)
+    tokens = T * dist.world
+    value = tokens / (ms / 1e3)
+    peaks = measured_peaks()
+    peak_kind = "bf16_tflops_sustained"
+    peak = peaks.get(peak_kind)
+    peak_note = "measured (MEASURED_PEAKS.json bf16_tflops_sustained: kernel timed inside a multi-second loop)"
+    if peak is None:
+        peak, peak_note = 1400.0, "fallback (no MEASURED_PEAKS.json)"
+    achieved = expert_flops(rows, wl.H, wl.I) / (ffn_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": "moe_grouped_swiglu_bf16 (row gather + GEMM1/SwiGLU + GEMM2)",
+                "work_per_launch": f"{expert_flops(rows, wl.H, wl.I) / 1e9:.1f} GFLOP = 2*rows*3*H*I, rows={rows}",
+                "peak_source": peak_note}
+
+    # end-to-end through the public API: pinned host x -> y in pinned host memory
+    e2e = None
+    if not args.no_e2e and kind == "forward":
+        xh = [xs[b].cpu().pin_memory() for b in range(n_batches)]
+        yh = torch.empty((T, wl.H), dtype=layer.y.dtype).pin_memory()
+        xd = torch.empty_like(xs[0])
+        for i in range(max(2, args.warmup)):
+            layer.forward_host(xh[i % n_batches], yh, xd)
+        dist.barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(args.steps):
+            layer.forward_host(xh[i % n_batches], yh, xd)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e2e_ms = dist.max(a.elapsed_time(b) / args.steps)
+        e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
+               "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
+               "d2h_bytes_per_step": int(yh.numel() * yh.element_size())}
+
+    launches_per_step = 2 + 4 + 3 + 2 + (2 if kind == "refill" else 1)  # route, permute, experts, shared, combine/refill+reduce
+    if kind == "refill":
+        launches_per_step += 1  # selection
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) tokens, N(0,1/sqrt(fan_in)) weights)",
+        "config": {"workload": f"{args.workload}: T={T} H={wl.H} E={wl.E} k={wl.k} I={wl.I} shared={wl.I_sh} "
+                               f"fmt={wl.fmt}" + (" +Refill-RMS accumulate/select" if kind == "refill" else ""),
+                   "tokens_per_step_per_gpu": T, "parallelism": f"dp{dist.world} (replicas, no collective)",
+                   "l2": f"{n_batches} rotating token batches ({n_batches * x_bytes / 2**20:.0f} MiB) and "
+                         f"{wl.E} experts of weights ({sum(t.numel() * t.element_size() for t in w.values()) / 2**30:.1f} GiB), "
+                         "both larger than the 126 MB L2"},
+        "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+        "expert_ffn_ms": round(ffn_ms, 4),
+    }
+    if dist.rank == 0 and not args.no_cpu_baseline:
+        n = args.cpu_sample_tokens or (8 if kind == "refill" else 16)
+        tps, dt = oracle_tokens_per_s(wl, w, xs[0], min(n, T), kind)
+        line["cpu_baseline"] = {"value": round(tps, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"first {min(n, T)} tokens of one batch of the same workload, full layer "
+                                          f"in float64 NumPy ({dt:.1f} s)"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, dist: Dist) -> None:
+    """The CPU oracle as the reference arm, rank 0 only."""
+    if dist.rank != 0:
+        return
+    wname, T, kind = WORKLOADS[args.workload]
+    wl = synth.WORKLOADS[wname]
+    dev = torch.device("cuda", dist.local) if torch.cuda.is_available() else torch.device("cpu")
+    w = synth.make_weights(wl, seed=0, device=dev)
+    x = synth.make_tokens(wl, T, seed=1, device=dev)
+    n = args.cpu_sample_tokens or (4 if kind == "refill" else 8)
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(wl, w, x, n, kind)
+    tot_t, tot_n = 0.0, 0
+    for i in range(args.steps):
+        xi = x[(i * n) % T:][:n]
+        _, dt = oracle_tokens_per_s(wl, w, xi, n, kind)
+        tot_t += dt
+        tot_n += n
+    v = tot_n / tot_t
+    line = {
+        "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{args.workload}: T={T} H={wl.H} E={wl.E} k={wl.k} I={wl.I} shared={wl.I_sh} "
+                               f"fmt={wl.fmt}", "tokens_per_step_per_gpu": n},
+        "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{n} tokens per step of the same workload, float64 NumPy"},
+        "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    dist = Dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist)
+        else:
+            run_native(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

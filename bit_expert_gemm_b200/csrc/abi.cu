@@ -1,0 +1,331 @@
+// extern "C" entry points declared in include/moe.h: host-side argument
+// checks, workspace sizing, and dispatch to the kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+
+#include "common.cuh"
+#include "gemm_sm100.cuh"
+
+namespace moe {
+
+// implemented in the other translation units
+size_t route_ws_bytes(int T, int E);
+int route_topk(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
+               int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, void* ws, size_t ws_bytes,
+               cudaStream_t stream);
+size_t permute_ws_bytes(int T, int E);
+int permute(const int32_t* topk_idx, int T, int ks, int E, int32_t* offsets, int32_t* row_token, int32_t* slot_row,
+            void* ws, size_t ws_bytes, cudaStream_t stream);
+int gather_rows(const void* x, const int32_t* row_token, int rows, int H, void* out, cudaStream_t stream);
+int combine(const void* f, int f_fp32, const int32_t* slot_row, int ks, const float* w, const void* shared,
+            const float* gate, int T, int k, int H, int dtype, void* y, cudaStream_t stream);
+size_t refill_ws_bytes(int T, int k);
+int refill(const void* f, int f_fp32, const int32_t* slot_row, const float* topk_logit, const int32_t* offsets, int T,
+           int k, int H, int E, double* sum_sq, int64_t* count, const void* shared, void* y_out, int dtype, void* ws,
+           size_t ws_bytes, cudaStream_t stream);
+int select_experts(const double* sum_sq, const int64_t* count, int E, int keep, int32_t* kept, int32_t* ranking,
+                   double* score, cudaStream_t stream);
+size_t awq_ws_bytes(int rows, int H, int I, int E);
+int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
+                       int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
+                       const int32_t* qz_d, const void* sc_d, int out_fp32, void* f, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+size_t nvfp4_quant_ws_bytes(int batch, int rows, int K);
+int nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const float* gs_in, uint8_t* codes,
+                   uint8_t* sf, float* gs_out, void* ws, size_t ws_bytes, cudaStream_t stream);
+size_t nvfp4_ws_bytes(int rows, int H, int I, int E);
+int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
+                         int I, int E, const uint8_t* w_gu, const uint8_t* sf_gu, const float* gs_gu,
+                         const uint8_t* w_d, const uint8_t* sf_d, const float* gs_d, const float* act_gs_in,
+                         float* act_gs_out, int out_fp32, void* f, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+namespace {
+thread_local char g_err[1024] = "";
+__device__ int g_status = 0;
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_sms[kMaxDevices] = {0};
+}  // namespace
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_status(cudaError_t e, const char* what) {
+  return set_error(MOE_ERR_CUDA, "%s failed: %s", what, cudaGetErrorString(e));
+}
+
+static int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return 0;
+  return d < kMaxDevices ? d : 0;
+}
+
+int* device_status_ptr() {
+  const int d = current_device();
+  if (!g_status_ptr[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) == cudaSuccess) g_status_ptr[d] = static_cast<int*>(p);
+  }
+  return g_status_ptr[d];
+}
+
+int num_sms() {
+  const int d = current_device();
+  if (!g_sms[d]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
+    g_sms[d] = n;
+  }
+  return g_sms[d];
+}
+
+unsigned long long wait_limit_ns() {
+  static unsigned long long lim = 0;
+  if (!lim) {
+    const char* s = getenv("BIT_EXPERT_GEMM_WAIT_LIMIT_MS");
+    long ms = s ? atol(s) : 0;
+    lim = (ms > 0 ? (unsigned long long)ms : 5000ull) * 1000000ull;
+  }
+  return lim;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Tile-width choice of a grouped GEMM from host-known sizes only: the widest
+// tile that still gives at least one tile per SM for an upper bound of the
+// number of row tiles.
+static int pick_bn(int rows, int groups, int n_out, bool swiglu) {
+  const long mt = (rows + 127) / 128 + (groups < rows ? groups : rows);
+  const int cands[3] = {256, 128, 64};
+  int last_ok = 0;
+  for (int bn : cands) {
+    const int bnh = swiglu ? bn / 2 : bn;
+    if (n_out % bnh) continue;
+    last_ok = bn;
+    if (mt * (n_out / bnh) >= num_sms()) return bn;
+  }
+  return last_ok;
+}
+
+static int swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
+                       int E, const void* w_gu, const void* w_d, int dtype, int out_fp32, void* f, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  WsCarver carve(ws, ws_bytes);
+  void* xp = row_token ? carve.take<uint16_t>(size_t(rows) * H) : nullptr;
+  uint16_t* h = carve.take<uint16_t>(size_t(rows) * I);
+  MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_grouped_swiglu_bf16: workspace of %zu bytes is too small", ws_bytes);
+  if (rows == 0) return MOE_OK;
+  const void* a = x;
+  if (row_token) {
+    int rc = gather_rows(x, row_token, rows, H, xp, stream);
+    if (rc) return rc;
+    a = xp;
+  }
+  GemmArgs g1{};
+  g1.group_offsets = offsets;
+  g1.G = E;
+  g1.rows = rows;
+  g1.K = H;
+  g1.n_out = I;
+  g1.b_rows_per_group = 2 * I;
+  g1.up_offset = I;
+  g1.out = h;
+  g1.ldo = I;
+  g1.out_fp32 = 0;
+  g1.bias = nullptr;
+  g1.bf16 = dtype == MOE_DTYPE_BF16;
+  g1.status = device_status_ptr();
+  g1.limit_ns = wait_limit_ns();
+  int rc = launch_grouped_gemm(a, rows, w_gu, E * 2 * I, g1, EPI_SWIGLU, pick_bn(rows, E, I, true), stream);
+  if (rc) return rc;
+  GemmArgs g2 = g1;
+  g2.K = I;
+  g2.n_out = H;
+  g2.b_rows_per_group = H;
+  g2.up_offset = 0;
+  g2.out = f;
+  g2.ldo = H;
+  g2.out_fp32 = out_fp32;
+  return launch_grouped_gemm(h, rows, w_d, E * H, g2, EPI_STORE, pick_bn(rows, E, H, false), stream);
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_abi_version(void) { return 1; }
+
+const char* moe_last_error(void) { return g_err; }
+
+int moe_device_status(int clear, void* stream) {
+  MOE_CHECK_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0;
+  MOE_CHECK_CUDA(cudaMemcpyFromSymbol(&v, g_status, sizeof(int)));
+  if (clear) {
+    const int z = 0;
+    MOE_CHECK_CUDA(cudaMemcpyToSymbol(g_status, &z, sizeof(int)));
+  }
+  return v;
+}
+
+size_t moe_workspace_size(int op, int T, int H, int E, int k_slots, int I) {
+  if (T < 0 || H < 0 || E < 0 || k_slots < 0 || I < 0) return 0;
+  const int rows = T * k_slots;
+  switch (op) {
+    case MOE_OP_ROUTE_TOPK: return route_ws_bytes(T, E);
+    case MOE_OP_PERMUTE: return permute_ws_bytes(T, E);
+    case MOE_OP_SWIGLU_BF16: {
+      WsCounter c;
+      c.take<uint16_t>(size_t(rows) * H);
+      c.take<uint16_t>(size_t(rows) * I);
+      return c.used;
+    }
+    case MOE_OP_SWIGLU_AWQ_G32: return awq_ws_bytes(rows, H, I, E);
+    case MOE_OP_SWIGLU_NVFP4: return nvfp4_ws_bytes(rows, H, I, E);
+    case MOE_OP_REFILL: return refill_ws_bytes(T, k_slots > 0 ? k_slots - 1 : 0);
+    case MOE_OP_NVFP4_QUANTIZE: return nvfp4_quant_ws_bytes(1, T, H);
+    default: return 0;
+  }
+}
+
+int moe_route_topk(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
+                   int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, void* ws, size_t ws_bytes,
+                   void* stream) {
+  MOE_REQUIRE(T >= 0 && H > 0 && E > 0, MOE_ERR_INVALID_ARG, "moe_route_topk: bad sizes T=%d H=%d E=%d", T, H, E);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_route_topk: dtype %d",
+              dtype);
+  MOE_REQUIRE(extra == 0 || extra == 1, MOE_ERR_INVALID_ARG, "moe_route_topk: extra must be 0 or 1");
+  MOE_REQUIRE(k >= 1 && k + extra <= 16 && k + extra <= E, MOE_ERR_UNSUPPORTED,
+              "moe_route_topk: need 1 <= k, k+extra <= 16 and <= E (k=%d extra=%d E=%d)", k, extra, E);
+  MOE_REQUIRE(E <= 1024, MOE_ERR_UNSUPPORTED, "moe_route_topk: E=%d > 1024", E);
+  MOE_REQUIRE(H % 64 == 0, MOE_ERR_UNSUPPORTED, "moe_route_topk: H=%d is not a multiple of 64", H);
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(x && w_router && topk_idx && topk_w, MOE_ERR_INVALID_ARG, "moe_route_topk: null pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(w_router), MOE_ERR_INVALID_ARG, "moe_route_topk: x / w_router not 16-byte aligned");
+  return route_topk(x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w, topk_logit, ws, ws_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int moe_permute(const int32_t* topk_idx, int T, int k_slots, int E, int32_t* expert_offsets, int32_t* row_token,
+                int32_t* slot_row, void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(T >= 0 && k_slots >= 1 && k_slots <= 16 && E >= 1 && E <= 1024, MOE_ERR_UNSUPPORTED,
+              "moe_permute: need T>=0, 1<=k_slots<=16, 1<=E<=1024 (T=%d k_slots=%d E=%d)", T, k_slots, E);
+  MOE_REQUIRE(expert_offsets != nullptr, MOE_ERR_INVALID_ARG, "moe_permute: expert_offsets is null");
+  MOE_REQUIRE(T == 0 || (topk_idx && row_token && slot_row), MOE_ERR_INVALID_ARG, "moe_permute: null pointer");
+  MOE_REQUIRE(long(T) * k_slots < (1l << 31), MOE_ERR_UNSUPPORTED, "moe_permute: T*k_slots overflows int32");
+  return permute(topk_idx, T, k_slots, E, expert_offsets, row_token, slot_row, ws, ws_bytes,
+                 static_cast<cudaStream_t>(stream));
+}
+
+int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows,
+                            int H, int I, int E, const void* w_gate_up, const void* w_down, int dtype, int out_fp32,
+                            void* f, void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1, MOE_ERR_INVALID_ARG, "moe_grouped_swiglu_bf16: bad sizes");
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_bf16: dtype %d", dtype);
+  MOE_REQUIRE(H > 0 && I > 0 && H % 64 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_grouped_swiglu_bf16: H=%d and I=%d must be positive multiples of 64", H, I);
+  MOE_REQUIRE(E <= kGemmMaxGroups, MOE_ERR_UNSUPPORTED, "moe_grouped_swiglu_bf16: E=%d > %d", E, kGemmMaxGroups);
+  MOE_REQUIRE(row_token || rows == T, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_bf16: without row_token, rows (%d) must equal T (%d)", rows, T);
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(x && expert_offsets && w_gate_up && w_down && f, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_bf16: null pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(w_gate_up) && aligned16(w_down) && aligned16(f), MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_bf16: operands must be 16-byte aligned");
+  return swiglu_bf16(x, row_token, expert_offsets, T, rows, H, I, E, w_gate_up, w_down, dtype, out_fp32, f, ws,
+                     ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
+                               int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
+                               const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
+                               int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_awq_g32: bad sizes");
+  MOE_REQUIRE(H > 0 && I > 0 && H % 64 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_grouped_swiglu_awq_g32: H=%d and I=%d must be positive multiples of 64", H, I);
+  MOE_REQUIRE(row_token || rows == T, MOE_ERR_INVALID_ARG, "moe_grouped_swiglu_awq_g32: without row_token rows must equal T");
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(x && expert_offsets && qw_gu && qz_gu && sc_gu && qw_d && qz_d && sc_d && f, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_awq_g32: null pointer");
+  return grouped_swiglu_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
+                            out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int moe_nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const float* global_scale_in,
+                       uint8_t* codes, uint8_t* sf, float* global_scale_out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  MOE_REQUIRE(batch >= 0 && rows >= 0 && K > 0 && K % 16 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_nvfp4_quantize: need K a positive multiple of 16 (K=%d)", K);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_nvfp4_quantize: dtype");
+  if (batch == 0 || rows == 0) return MOE_OK;
+  MOE_REQUIRE(v && codes && sf && global_scale_out, MOE_ERR_INVALID_ARG, "moe_nvfp4_quantize: null pointer");
+  return nvfp4_quantize(v, batch, rows, K, dtype, global_scale_in, codes, sf, global_scale_out, ws, ws_bytes,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int moe_grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows,
+                             int H, int I, int E, const uint8_t* w_gu, const uint8_t* sf_gu, const float* gs_gu,
+                             const uint8_t* w_d, const uint8_t* sf_d, const float* gs_d, const float* act_gs_in,
+                             float* act_gs_out, int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_nvfp4: bad sizes");
+  MOE_REQUIRE(H > 0 && I > 0 && H % 128 == 0 && I % 128 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_grouped_swiglu_nvfp4: H=%d and I=%d must be positive multiples of 128", H, I);
+  MOE_REQUIRE(row_token || rows == T, MOE_ERR_INVALID_ARG, "moe_grouped_swiglu_nvfp4: without row_token rows must equal T");
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(x && expert_offsets && w_gu && sf_gu && gs_gu && w_d && sf_d && gs_d && f, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_nvfp4: null pointer");
+  return grouped_swiglu_nvfp4(x, row_token, expert_offsets, T, rows, H, I, E, w_gu, sf_gu, gs_gu, w_d, sf_d, gs_d,
+                              act_gs_in, act_gs_out, out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int moe_combine(const void* f, int f_fp32, const int32_t* slot_row, int k_slots, const float* topk_w,
+                const void* shared_out, const float* shared_gate, int T, int k, int H, int dtype, void* y,
+                void* stream) {
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= k_slots && k_slots <= 16, MOE_ERR_INVALID_ARG,
+              "moe_combine: need 1 <= k <= k_slots <= 16");
+  MOE_REQUIRE(H > 0 && H % 8 == 0, MOE_ERR_UNSUPPORTED, "moe_combine: H=%d must be a multiple of 8", H);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_combine: dtype %d", dtype);
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(f && slot_row && topk_w && y, MOE_ERR_INVALID_ARG, "moe_combine: null pointer");
+  return combine(f, f_fp32, slot_row, k_slots, topk_w, shared_out, shared_gate, T, k, H, dtype, y,
+                 static_cast<cudaStream_t>(stream));
+}
+
+int razor_refill_rms_accumulate(const void* f, int f_fp32, const int32_t* slot_row, const int32_t* topk_idx,
+                                const float* topk_logit, const int32_t* expert_offsets, int T, int k, int H, int E,
+                                double* sum_sq, int64_t* count, const void* shared_out, void* y_out, int dtype,
+                                void* ws, size_t ws_bytes, void* stream) {
+  (void)topk_idx;  // the expert of each row is implied by expert_offsets
+  MOE_REQUIRE(T >= 0 && k >= 1 && k + 1 <= 16 && E >= 1 && E <= 1024, MOE_ERR_UNSUPPORTED,
+              "razor_refill_rms_accumulate: need 1 <= k, k+1 <= 16, 1 <= E <= 1024");
+  MOE_REQUIRE(H > 0 && H % 8 == 0, MOE_ERR_UNSUPPORTED, "razor_refill_rms_accumulate: H=%d must be a multiple of 8", H);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG,
+              "razor_refill_rms_accumulate: dtype %d", dtype);
+  MOE_REQUIRE(sum_sq && count && expert_offsets, MOE_ERR_INVALID_ARG, "razor_refill_rms_accumulate: null pointer");
+  MOE_REQUIRE(T == 0 || (f && slot_row && topk_logit), MOE_ERR_INVALID_ARG,
+              "razor_refill_rms_accumulate: null pointer");
+  return refill(f, f_fp32, slot_row, topk_logit, expert_offsets, T, k, H, E, sum_sq, count, shared_out, y_out, dtype,
+                ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int razor_select(const double* sum_sq, const int64_t* count, int E, int keep, int32_t* kept_idx, int32_t* ranking,
+                 double* score, void* stream) {
+  MOE_REQUIRE(E >= 1 && E <= 1024, MOE_ERR_UNSUPPORTED, "razor_select: E=%d outside [1, 1024]", E);
+  MOE_REQUIRE(keep >= 0 && keep <= E, MOE_ERR_INVALID_ARG, "razor_select: keep=%d outside [0, E]", keep);
+  MOE_REQUIRE(sum_sq && count && (kept_idx || keep == 0), MOE_ERR_INVALID_ARG, "razor_select: null pointer");
+  return select_experts(sum_sq, count, E, keep, kept_idx, ranking, score, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,360 @@
+// Persistent grouped tcgen05 GEMM (see gemm_sm100.cuh for the contract).
+#include <cstring>
+
+#include "gemm_sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int A_TILE_BYTES = BM * BK * 2;
+constexpr int kThreads = 192;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int B_TILE_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
+  static constexpr int STAGES = (196 * 1024) / STAGE_BYTES > 8 ? 8 : (196 * 1024) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // +1024: alignment slack
+  static constexpr uint32_t TMEM_COLS = 2 * BN;                    // two accumulators
+};
+
+struct TileMap {
+  int g, m, n;
+};
+
+// Exclusive scan of per-group m-tile counts into tile_start[0..G]; also
+// stores group row offsets in goff[0..G].  All threads participate.
+__device__ void build_tile_table(const GemmArgs& a, int* goff, int* tile_start, int* warp_sums) {
+  const int G = a.G;
+  const int tid = threadIdx.x;
+  for (int i = tid; i <= G; i += blockDim.x) goff[i] = a.group_offsets ? a.group_offsets[i] : (i == 0 ? 0 : a.rows);
+  __syncthreads();
+  // each thread owns a contiguous chunk of groups
+  const int per = (G + blockDim.x - 1) / blockDim.x;
+  const int g0 = tid * per;
+  int local = 0;
+  for (int g = g0; g < g0 + per && g < G; ++g) {
+    int n = goff[g + 1] - goff[g];
+    local += (n > 0 ? (n + BM - 1) / BM : 0);
+  }
+  // block exclusive scan of `local`
+  const int lane = tid & 31, warp = tid >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  int warp_base = 0;
+  for (int w = 0; w < warp; ++w) warp_base += warp_sums[w];
+  int run = warp_base + incl - local;
+  for (int g = g0; g < g0 + per && g < G; ++g) {
+    tile_start[g] = run;
+    int n = goff[g + 1] - goff[g];
+    run += (n > 0 ? (n + BM - 1) / BM : 0);
+  }
+  if (tid == blockDim.x - 1) tile_start[G] = run;
+  __syncthreads();
+}
+
+__device__ __forceinline__ TileMap decode_tile(int L, int nt, const int* tile_start, int G) {
+  TileMap t;
+  int mt = L / nt;
+  t.n = L - mt * nt;
+  // last g with tile_start[g] <= mt (empty groups share their start with the next one)
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= mt) lo = mid; else hi = mid - 1;
+  }
+  t.g = lo;
+  t.m = mt - tile_start[lo];
+  return t;
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmArgs args) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr int BNH = (EPI == EPI_SWIGLU) ? BN / 2 : BN;  // output columns per tile
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+  __shared__ int goff[kGemmMaxGroups + 1];
+  __shared__ int tile_start[kGemmMaxGroups + 1];
+  __shared__ int warp_sums[kThreads / 32];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  auto smA = [&](int s) { return smem + s * Cfg::STAGE_BYTES; };
+  auto smB = [&](int s) { return smem + s * Cfg::STAGE_BYTES + A_TILE_BYTES; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], 128);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  build_tile_table(args, goff, tile_start, warp_sums);  // contains __syncthreads
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+
+  const int G = args.G;
+  const int nt = args.n_out / BNH;
+  const int total = tile_start[G] * nt;
+  const int KB = args.K / BK;
+  int* status = args.status;
+  const unsigned long long lim = args.limit_ns;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        TileMap t = decode_tile(L, nt, tile_start, G);
+        const int a_row = goff[t.g] + t.m * BM;
+        const int b_row = t.g * args.b_rows_per_group + t.n * BNH;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
+          tma_load_2d(smA(stage), &tmA, &full_bar[stage], kb * BK, a_row);
+          if (EPI == EPI_SWIGLU) {
+            tma_load_2d(smB(stage), &tmB, &full_bar[stage], kb * BK, b_row);
+            tma_load_2d(smB(stage) + BNH * BK * 2, &tmB, &full_bar[stage], kb * BK, b_row + args.up_offset);
+          } else {
+            tma_load_2d(smB(stage), &tmB, &full_bar[stage], kb * BK, b_row);
+          }
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        // let the copies already in flight land before the CTA exits
+        volatile int never = 0;
+        for (long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+          mbar_wait(&full_bar[i % STAGES], uint32_t((i / STAGES) & 1), &never, nullptr, lim);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- UMMA issuer ----------------
+      const uint32_t idesc = idesc_f16(args.bf16, BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, &abort_flag, status, lim)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + uint32_t(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = sdesc_kmajor_sw128(smem_u32(smA(stage)));
+          const uint64_t bd = sdesc_kmajor_sw128(smem_u32(smB(stage)));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_f16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+          umma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull_bar[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      // every issued UMMA must be complete before TMEM is released
+      umma_commit(&drain_bar);
+      volatile int never = 0;
+      mbar_wait(&drain_bar, 0, &never, nullptr, lim);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5 ----------------
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      TileMap t = decode_tile(L, nt, tile_start, G);
+      const int n_g = goff[t.g + 1] - goff[t.g];
+      const size_t out_row = size_t(goff[t.g]) + size_t(t.m) * BM + row_in_tile;
+      // rows past the group, or (with inconsistent offsets) past the output, are not written
+      const bool valid = t.m * BM + row_in_tile < n_g && out_row < size_t(args.rows);
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag, status, lim)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+      if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BNH / 32; ++c) {
+          float gv[32], uv[32];
+          tmem_ld32x2(tb + c * 32, tb + BNH + c * 32, gv, uv);
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float h0 = silu_f(gv[2 * i]) * uv[2 * i];
+              float h1 = silu_f(gv[2 * i + 1]) * uv[2 * i + 1];
+              pk[i] = args.bf16 ? Pack2<__nv_bfloat16>::pack(h0, h1) : Pack2<__half>::pack(h0, h1);
+            }
+            uint16_t* dst = reinterpret_cast<uint16_t*>(args.out) + out_row * size_t(args.ldo) + t.n * BNH + c * 32;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) st_global_v4(dst + 8 * v, pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tb + c * 32, v);
+          if (valid) {
+            const int col0 = t.n * BN + c * 32;
+            if (args.bias) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] += __ldg(args.bias + col0 + i);
+            }
+            if (args.out_fp32) {
+              float* dst = reinterpret_cast<float*>(args.out) + out_row * size_t(args.ldo) + col0;
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                st_global_v4(dst + 4 * i, __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
+                             __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
+            } else {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = args.bf16 ? Pack2<__nv_bfloat16>::pack(v[2 * i], v[2 * i + 1])
+                                  : Pack2<__half>::pack(v[2 * i], v[2 * i + 1]);
+              uint16_t* dst = reinterpret_cast<uint16_t*>(args.out) + out_row * size_t(args.ldo) + col0;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) st_global_v4(dst + 8 * i, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// 2-D tensor map of a row-major [rows, cols] 16-bit matrix, box [box_rows, 64]
+// with the 128-byte swizzle (the K-major UMMA operand layout).
+int make_tmap_16bit_sw128(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  MOE_REQUIRE(enc != nullptr, MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  MOE_REQUIRE((reinterpret_cast<uintptr_t>(base) & 15) == 0, MOE_ERR_INVALID_ARG, "operand is not 16-byte aligned");
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MOE_REQUIRE(r == CUDA_SUCCESS, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a [%d, %d] operand", int(r),
+              rows, cols);
+  return MOE_OK;
+}
+
+template <int BN, int EPI>
+static int launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN>;
+  static bool attr_set[64] = {false};  // per device
+  auto kern = k_grouped_gemm<BN, EPI>;
+  int dev = 0;
+  MOE_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev >= 64 || !attr_set[dev]) {
+    MOE_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+    if (dev < 64) attr_set[dev] = true;
+  }
+  int grid = num_sms();
+  kern<<<grid, kThreads, Cfg::SMEM_BYTES, stream>>>(ta, tb, args);
+  MOE_CHECK_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_total, const GemmArgs& args, int epi,
+                        int bn, cudaStream_t stream) {
+  MOE_REQUIRE(args.K % BK == 0 && args.K > 0, MOE_ERR_UNSUPPORTED, "GEMM K=%d is not a positive multiple of 64",
+              args.K);
+  MOE_REQUIRE(args.G >= 1 && args.G <= kGemmMaxGroups, MOE_ERR_UNSUPPORTED, "GEMM group count %d outside [1, %d]",
+              args.G, kGemmMaxGroups);
+  MOE_REQUIRE(bn == 64 || bn == 128 || bn == 256, MOE_ERR_INVALID_ARG, "tile width %d", bn);
+  const int bnh = epi == EPI_SWIGLU ? bn / 2 : bn;
+  MOE_REQUIRE(args.n_out % bnh == 0, MOE_ERR_UNSUPPORTED, "output width %d is not a multiple of the tile (%d)",
+              args.n_out, bnh);
+  if (a_rows == 0) return MOE_OK;
+  CUtensorMap ta, tb;
+  int rc = make_tmap_16bit_sw128(&ta, A, a_rows, args.K, BM);
+  if (rc) return rc;
+  rc = make_tmap_16bit_sw128(&tb, B, b_rows_total, args.K, bnh);
+  if (rc) return rc;
+  if (epi == EPI_SWIGLU) {
+    if (bn == 256) return launch_bn<256, EPI_SWIGLU>(ta, tb, args, stream);
+    if (bn == 128) return launch_bn<128, EPI_SWIGLU>(ta, tb, args, stream);
+    return launch_bn<64, EPI_SWIGLU>(ta, tb, args, stream);
+  }
+  if (bn == 256) return launch_bn<256, EPI_STORE>(ta, tb, args, stream);
+  if (bn == 128) return launch_bn<128, EPI_STORE>(ta, tb, args, stream);
+  return launch_bn<64, EPI_STORE>(ta, tb, args, stream);
+}
+
+}  // namespace moe

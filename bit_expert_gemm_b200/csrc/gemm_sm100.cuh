@@ -1,0 +1,45 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05 /
+// TMEM), fed by TMA.  Used for the expert GEMMs of the MoE layer (gate/up
+// with a fused SwiGLU epilogue, and down), for dense experts (one group) and
+// for the router logits (one group, FP32 output plus bias).
+//
+//   for every group g (an expert) with rows R_g = [off[g], off[g+1]) of A:
+//     D[r, n] = sum_k A[r, k] * B[g * b_rows + n, k]          (FP32 in TMEM)
+//
+// Tiles are 128 rows of A by BN rows of B, K stepped by 64 (one 128-byte
+// swizzle row of 16-bit elements).  Warp roles: warp 0 = TMA producer,
+// warp 1 = UMMA issuer (and TMEM owner), warps 2..5 = epilogue, one TMEM
+// lane quadrant each.  The accumulator is double-buffered in TMEM so the
+// epilogue of one tile overlaps the main loop of the next.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
+constexpr int kGemmMaxGroups = 1024;
+
+struct GemmArgs {
+  const int* group_offsets;  // [G+1] on the device, or nullptr: one group of `rows` rows
+  int G;
+  int rows;
+  int K;                 // multiple of 64
+  int n_out;             // output columns per group (SwiGLU: I; store: N)
+  int b_rows_per_group;  // rows of B per group (SwiGLU: 2I; store: N)
+  int up_offset;         // SwiGLU: row offset of the up rows (I)
+  void* out;
+  int ldo;               // output leading dimension (elements)
+  int out_fp32;          // store: 1 -> FP32 output, 0 -> 16-bit of the input dtype
+  const float* bias;     // store: per output column, may be nullptr
+  int bf16;              // 1: BF16 operands, 0: FP16
+  int* status;
+  unsigned long long limit_ns;
+};
+
+// Host launcher (gemm_sm100.cu).  A [a_rows, K] and B [b_rows_total, K] are
+// row-major 16-bit device arrays.  bn selects the tile width (64/128/256).
+int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_total, const GemmArgs& args, int epi,
+                        int bn, cudaStream_t stream);
+
+}  // namespace moe

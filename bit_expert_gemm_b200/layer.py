@@ -1,0 +1,141 @@
+"""The routed-expert MoE layer as a sequence of C-ABI calls.
+
+MoELayer owns the device weights of one layer plus every intermediate
+buffer and workspace for a maximum token count, so that a forward pass
+launches only the library's kernels (no allocation, no host sync).  The
+weight format is one of "bf16" (16-bit weights, BF16 or FP16 activations),
+"awq_g32" and "nvfp4"; the router and the shared expert are always 16-bit.
+
+forward(x)               x [T, H] on the device -> y [T, H]
+forward_host(xh, yh)     pinned host x -> y in pinned host memory (copies in
+                         the stream, for end-to-end measurements)
+refill_pass(x, stats)    one Refill-RMS scoring pass (k+1 slots), adds to the
+                         statistics and returns y
+"""
+
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import abi
+
+
+class MoELayer:
+    def __init__(self, weights: Dict[str, torch.Tensor], k: int, fmt: str = "bf16", T_max: int = 8192,
+                 extra: int = 0, device: Optional[torch.device] = None):
+        self.w = weights
+        self.k = k
+        self.fmt = fmt
+        self.extra = extra
+        self.dev = device or weights["w_router"].device
+        self.E, self.H = weights["w_router"].shape
+        self.adt = weights["w_router"].dtype
+        self.I_sh = weights["w_sh_down"].shape[1]
+        if fmt in ("bf16",):
+            self.I = weights["w_gate_up"].shape[1] // 2
+        elif fmt == "awq_g32":
+            self.I = weights["qw_gu"].shape[2] * 8 // 2
+        elif fmt == "nvfp4":
+            self.I = weights["w_gu"].shape[1] // 2
+        else:
+            raise ValueError(fmt)
+        self._alloc(T_max)
+
+    def _alloc(self, T_max: int) -> None:
+        d, H, E = self.dev, self.H, self.E
+        ks = self.k + self.extra
+        rows = T_max * ks
+        i32 = torch.int32
+        self.T_max = T_max
+        self.topk_idx = torch.empty((T_max, ks), dtype=i32, device=d)
+        self.topk_w = torch.empty((T_max, self.k), dtype=torch.float32, device=d)
+        self.topk_logit = torch.empty((T_max, ks), dtype=torch.float32, device=d)
+        self.offsets = torch.empty((E + 1,), dtype=i32, device=d)
+        self.row_token = torch.empty((rows,), dtype=i32, device=d)
+        self.slot_row = torch.empty((T_max, ks), dtype=i32, device=d)
+        f_dt = torch.float32 if self.extra else (torch.float16 if self.fmt == "awq_g32" else torch.bfloat16)
+        if self.fmt == "bf16" and not self.extra:
+            f_dt = self.adt
+        self.f = torch.empty((rows, H), dtype=f_dt, device=d)
+        self.shared = torch.empty((T_max, H), dtype=self.adt, device=d)
+        self.y = torch.empty((T_max, H), dtype=self.adt, device=d)
+        op = {"bf16": abi.MOE_OP_SWIGLU_BF16, "awq_g32": abi.MOE_OP_SWIGLU_AWQ_G32,
+              "nvfp4": abi.MOE_OP_SWIGLU_NVFP4}[self.fmt]
+        self.ws_route = abi.workspace(abi.MOE_OP_ROUTE_TOPK, T_max, H, E, ks, 0, d)
+        self.ws_perm = abi.workspace(abi.MOE_OP_PERMUTE, T_max, H, E, ks, 0, d)
+        self.ws_ffn = abi.workspace(op, T_max, H, E, ks, self.I, d)
+        self.ws_sh = abi.workspace(abi.MOE_OP_SWIGLU_BF16, T_max, H, 1, 1, self.I_sh, d)
+        self.ws_refill = abi.workspace(abi.MOE_OP_REFILL, T_max, H, E, ks, 0, d)
+        self._sh_off = {}
+
+    def _shared_offsets(self, T: int) -> torch.Tensor:
+        t = self._sh_off.get(T)
+        if t is None:
+            t = torch.tensor([0, T], dtype=torch.int32, device=self.dev)
+            self._sh_off[T] = t
+        return t
+
+    def route(self, x: torch.Tensor):
+        T = x.shape[0]
+        ks = self.k + self.extra
+        abi.moe_route_topk(x, self.w["w_router"], self.w["bias"], self.k, self.extra, topk_idx=self.topk_idx[:T],
+                           topk_w=self.topk_w[:T], topk_logit=self.topk_logit[:T], ws=self.ws_route)
+        abi.moe_permute(self.topk_idx[:T], self.E, expert_offsets=self.offsets, row_token=self.row_token[:T * ks],
+                        slot_row=self.slot_row[:T], ws=self.ws_perm)
+
+    def experts(self, x: torch.Tensor) -> torch.Tensor:
+        T = x.shape[0]
+        rows = T * (self.k + self.extra)
+        f = self.f[:rows]
+        w = self.w
+        if self.fmt == "bf16":
+            abi.moe_grouped_swiglu_bf16(x, self.row_token[:rows], self.offsets, rows, w["w_gate_up"], w["w_down"],
+                                        out_fp32=f.dtype == torch.float32, f=f, ws=self.ws_ffn)
+        elif self.fmt == "awq_g32":
+            abi.moe_grouped_swiglu_awq_g32(x, self.row_token[:rows], self.offsets, rows, w["qw_gu"], w["qz_gu"],
+                                           w["sc_gu"], w["qw_d"], w["qz_d"], w["sc_d"],
+                                           out_fp32=f.dtype == torch.float32, f=f, ws=self.ws_ffn)
+        else:
+            abi.moe_grouped_swiglu_nvfp4(x, self.row_token[:rows], self.offsets, rows, w["w_gu"], w["sf_gu"],
+                                         w["gs_gu"], w["w_d"], w["sf_d"], w["gs_d"], act_gs_in=w.get("act_gs"),
+                                         out_fp32=f.dtype == torch.float32, f=f, ws=self.ws_ffn)
+        return f
+
+    def shared_expert(self, x: torch.Tensor) -> torch.Tensor:
+        T = x.shape[0]
+        sh = self.shared[:T]
+        abi.moe_grouped_swiglu_bf16(x, None, self._shared_offsets(T), T, self.w["w_sh_gate_up"].unsqueeze(0),
+                                    self.w["w_sh_down"].unsqueeze(0), out_fp32=False, f=sh, ws=self.ws_sh)
+        return sh
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        T = x.shape[0]
+        assert T <= self.T_max and self.extra == 0
+        self.route(x)
+        f = self.experts(x)
+        sh = self.shared_expert(x)
+        y = self.y[:T]
+        abi.moe_combine(f, self.slot_row[:T], self.topk_w[:T], shared_out=sh, y=y)
+        return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, x_dev: torch.Tensor) -> None:
+        """Pinned host x -> device -> forward -> pinned host y, all enqueued on
+        the current stream."""
+        T = x_host.shape[0]
+        x_dev[:T].copy_(x_host, non_blocking=True)
+        y = self.forward(x_dev[:T])
+        y_host.copy_(y, non_blocking=True)
+
+    def refill_pass(self, x: torch.Tensor, sum_sq: torch.Tensor, count: torch.Tensor) -> torch.Tensor:
+        """One Refill-RMS scoring pass over x; statistics are added in place."""
+        T = x.shape[0]
+        assert self.extra == 1
+        self.route(x)
+        f = self.experts(x)
+        sh = self.shared_expert(x)
+        y = self.y[:T]
+        abi.razor_refill_rms_accumulate(f, self.slot_row[:T], self.topk_idx[:T], self.topk_logit[:T], self.offsets,
+                                        sum_sq, count, shared_out=sh, y_out=y, ws=self.ws_refill)
+        return y

@@ -1,0 +1,271 @@
+/*
+ * bit_expert_gemm_b200 -- C ABI of the routed-expert MoE layer and RAZOR
+ * Refill-RMS scoring on one NVIDIA B200 (sm_100a).
+ *
+ * The operations follow these pages (cited by page title and section):
+ *   [ARCH]  Qwen3.8-Flash-Next architecture fact sheet (archdb model page):
+ *           entries "Routed experts per MoE layer" (512), "Routed experts
+ *           selected per token" (10), "Always-on experts per MoE layer" (1),
+ *           "Intermediate width of one routed expert" (640), "Gating function
+ *           over expert logits" (softmax), "Selected expert weights are
+ *           renormalized to sum to 1" (yes), "FFN activation" (SwiGLU),
+ *           "Clamping of GLU gate / up activations" (none), "FFN projections
+ *           have bias terms" (no).
+ *   [AWQ]   Qwen3.8-Flash-Next-AWQ-g32 card, sections "Checkpoint" (format:
+ *           asymmetric W4A16, group 32, integer zero point, GEMM packing, FP16
+ *           expert scales) and "Calibration" (code rule
+ *           clip(round(w/scale + zero), 0, 15)).
+ *   [NVFP4] Qwen3.8-Flash-Next-RAZOR-96B-A6B-NVFP4 card, component table
+ *           ("Routed experts: NVFP4 W4A4 (group 16, FP8 block scales, FP32
+ *           global scales)"; shared expert and router BF16).
+ *   [RAZOR] Qwen3.8-Flash-Next-RAZOR-65B-A6B-E256of512 card, section
+ *           "Selection and calibration" (Refill-RMS score, conditional RMS
+ *           aggregation, keep the top 256 / 384, additive statistics) and the
+ *           opening paragraphs (experts and router rows sliced in matching
+ *           order; keep manifest in output order).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every function returns an int status (MOE_OK or an MOE_ERR_* code).  On
+ *    error, moe_last_error() returns a message for the calling host thread.
+ *    Argument checks happen on the host before anything is launched; a call
+ *    that fails its checks launches nothing.
+ *  - Tensor arguments are DEVICE pointers owned by the caller, contiguous,
+ *    row-major, unless a comment says otherwise.  The library never allocates
+ *    or frees device memory and never synchronises the host; all work is
+ *    enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream).
+ *  - Scratch memory is passed as (ws, ws_bytes); its required size is
+ *    returned by moe_workspace_size().  The workspace must be 256-byte
+ *    aligned and must not be used by another call that may run concurrently.
+ *  - "dtype" is MOE_DTYPE_BF16 or MOE_DTYPE_F16 and describes the 16-bit
+ *    activations and 16-bit weights of the call.
+ *  - Weights are stored out x in (row j of a projection produces output
+ *    feature j).  The stacked gate/up projection of an expert holds the gate
+ *    rows 0..I-1 followed by the up rows I..2I-1.
+ *  - Device-side waits are bounded.  A wait that runs out records
+ *    MOE_ERR_TIMEOUT in a device status word that moe_device_status() reads.
+ */
+#ifndef BIT_EXPERT_GEMM_B200_MOE_H_
+#define BIT_EXPERT_GEMM_B200_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, index out of range   */
+  MOE_ERR_UNSUPPORTED = 2, /* a shape the kernels do not handle (see each call) */
+  MOE_ERR_WORKSPACE = 3,   /* ws too small or misaligned                          */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed                          */
+  MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out                  */
+};
+
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_F16 = 1 };
+
+/* Operation ids for moe_workspace_size(). */
+enum {
+  MOE_OP_ROUTE_TOPK = 0,
+  MOE_OP_PERMUTE = 1,
+  MOE_OP_SWIGLU_BF16 = 2,
+  MOE_OP_SWIGLU_AWQ_G32 = 3,
+  MOE_OP_SWIGLU_NVFP4 = 4,
+  MOE_OP_REFILL = 5,
+  MOE_OP_NVFP4_QUANTIZE = 6
+};
+
+/* Version of this header's ABI. */
+MOE_API int moe_abi_version(void);
+
+/* Message of the last failed call on this host thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* Synchronises `stream`, returns the device status word of the current
+ * device (MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait ran out,
+ * or MOE_ERR_INVALID_ARG if a kernel met an out-of-range index), and clears
+ * it when `clear` is non-zero.  This is the only call that synchronises. */
+MOE_API int moe_device_status(int clear, void* stream);
+
+/* Bytes of workspace that operation `op` needs for the given sizes
+ * (T tokens, hidden size H, E experts, k_slots selected slots per token,
+ * intermediate width I).  Returns 0 for an unknown op.  The result is an
+ * upper bound valid for any routing of those sizes. */
+MOE_API size_t moe_workspace_size(int op, int T, int H, int E, int k_slots, int I);
+
+/* ---------------------------------------------------------------------------
+ * Router, softmax over all E experts, top-k, renormalised weights [ARCH].
+ *
+ *   l[t, e]  = sum_h x[t, h] * w_router[e, h] + bias[e]      (FP32 accumulate)
+ *   S_t      = the k experts of largest l (equivalently of largest softmax
+ *              probability), ties to the lower expert index, in descending
+ *              order; with extra = 1 the rank-(k+1) expert r_t is appended
+ *              (the expert Refill-RMS promotes [RAZOR]).
+ *   topk_w   = softmax(l)[S] / sum softmax(l)[S]  (sums to 1 over the k slots)
+ *
+ * x [T, H] and w_router [E, H] are 16-bit (dtype); bias [E] FP32 or NULL.
+ * Outputs: topk_idx [T, k+extra] int32, topk_w [T, k] FP32, topk_logit
+ * [T, k+extra] FP32 (the logits l of the selected experts, bias included; may
+ * be NULL).  Limits: 1 <= k, k + extra <= 16, k + extra <= E <= 1024,
+ * H % 64 == 0.  Workspace: MOE_OP_ROUTE_TOPK.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_route_topk(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k,
+                   int extra, int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Permutation of the (token, slot) assignments by expert: histogram,
+ * exclusive scan, scatter.  The order is deterministic: expert blocks in
+ * ascending expert id, and inside one expert ascending token index (every
+ * token selects an expert at most once).
+ *
+ * topk_idx [T, k_slots] int32 in [0, E) -> expert_offsets [E+1] int32
+ * (expert e owns permuted rows expert_offsets[e] .. expert_offsets[e+1]-1),
+ * row_token [T*k_slots] int32 (token of each permuted row), slot_row
+ * [T, k_slots] int32 (permuted row of each assignment).  An index outside
+ * [0, E) is skipped and recorded as MOE_ERR_INVALID_ARG in the device status
+ * word; duplicate experts within one token's slots are not allowed.
+ * Limits: E <= 1024, k_slots <= 16.  Workspace: MOE_OP_PERMUTE.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_permute(const int32_t* topk_idx, int T, int k_slots, int E, int32_t* expert_offsets, int32_t* row_token,
+                int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Grouped SwiGLU expert FFN with 16-bit weights [ARCH]:
+ *   for every expert e and every permuted row r of e (expert_offsets):
+ *     g = x[row_token[r]] . Wg_e^T,  u = x[row_token[r]] . Wu_e^T   (FP32 acc)
+ *     h = silu(g) * u,  silu(g) = g / (1 + exp(-g)), rounded to dtype
+ *     f[r] = h . Wd_e^T                                            (FP32 acc)
+ *
+ * x [T, H] dtype; row_token [rows] int32, or NULL for the identity (rows
+ * must then equal T: this computes a dense expert such as the shared expert
+ * with E = 1 and expert_offsets = {0, T}); expert_offsets [E+1] int32 on the
+ * device, expert_offsets[E] == rows; w_gate_up [E, 2I, H] dtype; w_down
+ * [E, H, I] dtype; f [rows, H], FP32 when out_fp32 != 0, else dtype.
+ * Limits: H % 64 == 0, I % 64 == 0, E <= 1024.  Workspace:
+ * MOE_OP_SWIGLU_BF16 (holds the gathered rows and h).
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
+                            int rows, int H, int I, int E, const void* w_gate_up, const void* w_down, int dtype,
+                            int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Grouped SwiGLU expert FFN with AWQ W4A16 asymmetric group-32 weights [AWQ].
+ * Same maths as moe_grouped_swiglu_bf16 with FP16 activations, h rounded to
+ * FP16, and each weight dequantised exactly as
+ *     W[k, n] = fp16_rn((q[k, n] - z[k/32, n]) * s[k/32, n])
+ * (the inverse of the card's code rule).  Layout per projection with input
+ * dim K and output dim N, input-major ("GEMM" orientation):
+ *     qweight [K, N/8] int32: word w of row k holds the codes of output
+ *             columns 8w .. 8w+7, column 8w+i in bits 4i .. 4i+3;
+ *     qzeros  [K/32, N/8] int32, packed the same way;
+ *     scales  [K/32, N] FP16.
+ * Gate/up projection: K = H, N = 2I (gate columns 0..I-1, up I..2I-1):
+ *   qw_gu [E, H, 2I/8], qz_gu [E, H/32, 2I/8], sc_gu [E, H/32, 2I].
+ * Down projection: K = I, N = H: qw_d [E, I, H/8], qz_d [E, I/32, H/8],
+ *   sc_d [E, I/32, H].
+ * x [T, H] FP16; f [rows, H], FP32 when out_fp32 != 0, else FP16.
+ * Limits: H % 64 == 0, I % 64 == 0.  Workspace: MOE_OP_SWIGLU_AWQ_G32.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
+                               int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
+                               const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
+                               int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * NVFP4 quantisation of `batch` tensors [rows, K] of 16-bit values [NVFP4]
+ * (decode-direction scales, every rounding decision in FP32 IEEE
+ * round-to-nearest-even, in this order):
+ *     s_g = amax(|V|) / 2688            (or global_scale_in[b] when given)
+ *     s_b = e4m3_rn_satfinite(amax(|block of 16 along K|) / (6 * s_g))
+ *     c   = e2m1_rn_satfinite(v / (e4m3(s_b) * s_g)),  c = +0 if e4m3(s_b)*s_g == 0
+ * v [batch, rows, K] dtype; codes [batch, rows, K/2] uint8 (element 2j in the
+ * low nibble); sf [batch, rows, K/16] uint8 E4M3; global_scale_out [batch]
+ * FP32 (device).  global_scale_in [batch] FP32 device or NULL (dynamic).
+ * Limits: K % 16 == 0.  Workspace: MOE_OP_NVFP4_QUANTIZE.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const float* global_scale_in,
+                       uint8_t* codes, uint8_t* sf, float* global_scale_out, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Grouped SwiGLU expert FFN with NVFP4 W4A4 weights [NVFP4].  The gathered
+ * activations are quantised to NVFP4 on the fly (moe_nvfp4_quantize's rule
+ * over the whole [rows, H] input), GEMM1 runs on FP4 x FP4 with E4M3 block
+ * scales and FP32 accumulation, h = silu(g) * u is quantised again (over the
+ * whole [rows, I] intermediate) and GEMM2 runs the same way.
+ * Weights as produced by moe_nvfp4_quantize:
+ *   w_gu [E, 2I, H/2], sf_gu [E, 2I, H/16], gs_gu [E, 2] (gate, up);
+ *   w_d  [E, H, I/2],  sf_d  [E, H, I/16],  gs_d  [E].
+ * act_gs_in [2] FP32 device (static global scales of x and h) or NULL
+ * (dynamic amax); act_gs_out [2] receives the scales used (may be NULL).
+ * x [T, H] BF16; f [rows, H], FP32 when out_fp32 != 0, else BF16.
+ * Limits: H % 128 == 0, I % 128 == 0.  Workspace: MOE_OP_SWIGLU_NVFP4.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
+                             int rows, int H, int I, int E, const uint8_t* w_gu, const uint8_t* sf_gu,
+                             const float* gs_gu, const uint8_t* w_d, const uint8_t* sf_d, const float* gs_d,
+                             const float* act_gs_in, float* act_gs_out, int out_fp32, void* f, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Weighted combine [ARCH]:
+ *   y[t] = sum_{j<k} topk_w[t, j] * f[slot_row[t, j]]  (+ gate[t] * shared[t])
+ * summed in FP32 in slot order, rounded once to dtype.
+ * f [rows, H] (FP32 when f_fp32 != 0, else dtype); slot_row [T, k_slots]
+ * (k <= k_slots; extra slots are ignored); topk_w [T, k] FP32; shared_out
+ * [T, H] dtype or NULL; shared_gate [T] FP32 or NULL (gate 1); y [T, H] dtype.
+ * Limits: H % 8 == 0.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_combine(const void* f, int f_fp32, const int32_t* slot_row, int k_slots, const float* topk_w,
+                const void* shared_out, const float* shared_gate, int T, int k, int H, int dtype, void* y,
+                void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Refill-RMS accumulation, fused with the combine of a (k+1)-slot pass
+ * [RAZOR].  For token t with selected set S (slots 0..k-1) and promoted
+ * expert r (slot k), with p_j = exp(l_j - l_0) from topk_logit:
+ *   Z = sum_S p,  U = sum_S p_j f_j,  y = U / Z
+ *   for each e in S:  delta_e = (U - p_e f_e + p_r f_r) / (Z - p_e + p_r) - y
+ *                     sum_sq[e] += ||delta_e||_2^2,  count[e] += 1
+ * (the layer output change when e is removed and r promoted; the shared
+ * expert cancels).  Statistics are additive across calls: sum_sq [E] FP64 and
+ * count [E] int64 are read and updated in place and must be initialised by
+ * the caller (zeros for a fresh pass).  The per-expert sums are formed in a
+ * fixed order (deterministic for a given routing).
+ * f [rows, H] (FP32 when f_fp32 != 0, else dtype), rows = T*(k+1) permuted
+ * rows of the (k+1)-slot pass; slot_row, topk_idx, topk_logit [T, k+1];
+ * expert_offsets [E+1] of that pass.  y_out [T, H] dtype or NULL receives
+ * y (+ shared_out when given).  Limits: k + 1 <= 16, H % 8 == 0.
+ * Workspace: MOE_OP_REFILL.
+ * ------------------------------------------------------------------------- */
+MOE_API int razor_refill_rms_accumulate(const void* f, int f_fp32, const int32_t* slot_row, const int32_t* topk_idx,
+                                const float* topk_logit, const int32_t* expert_offsets, int T, int k, int H, int E,
+                                double* sum_sq, int64_t* count, const void* shared_out, void* y_out, int dtype,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Refill-RMS selection [RAZOR]: score_e = sqrt(sum_sq[e] / count[e]) (0 when
+ * count[e] == 0), rank by (score descending, expert index ascending), keep the
+ * first `keep`.  kept_idx [keep] int32 receives the kept original indices in
+ * ascending order ("output order" of the sliced checkpoint); ranking [E]
+ * int32 (the full order) and score [E] FP64 may be NULL.
+ * Limits: 1 <= E <= 1024, 0 <= keep <= E.
+ * ------------------------------------------------------------------------- */
+MOE_API int razor_select(const double* sum_sq, const int64_t* count, int E, int keep, int32_t* kept_idx, int32_t* ranking,
+                 double* score, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BIT_EXPERT_GEMM_B200_MOE_H_ */

@@ -1,0 +1,66 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point the header declares, sizes workspaces, and rejects bad
+arguments before launching anything."""
+
+import ctypes
+
+import pytest
+
+from bit_expert_gemm_b200 import abi
+
+
+def test_library_exports_every_header_symbol():
+    lib = abi.load()
+    names = abi.header_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(abi._SIGS)  # the binding covers exactly the header
+    assert lib.moe_abi_version() == 1
+
+
+def test_workspace_sizes():
+    lib = abi.load()
+    assert lib.moe_workspace_size(abi.MOE_OP_ROUTE_TOPK, 8192, 2048, 512, 10, 640) >= 8192 * 512 * 4
+    big = lib.moe_workspace_size(abi.MOE_OP_SWIGLU_BF16, 8192, 2048, 512, 10, 640)
+    assert big >= 81920 * (2048 + 640) * 2
+    assert lib.moe_workspace_size(abi.MOE_OP_PERMUTE, 32768, 2048, 512, 11, 640) >= 512 * 1024 * 8
+    assert lib.moe_workspace_size(99, 1, 1, 1, 1, 1) == 0
+    assert lib.moe_workspace_size(abi.MOE_OP_ROUTE_TOPK, -1, 1, 1, 1, 1) == 0
+
+
+def _code(fn, *args):
+    return getattr(abi.load(), fn)(*args)
+
+
+@pytest.mark.parametrize("k,extra,E,H", [(0, 0, 16, 256), (17, 0, 512, 256), (10, 1, 10, 256), (2, 0, 2048, 256),
+                                         (2, 0, 16, 100), (2, 3, 16, 256)])
+def test_route_rejects_bad_shapes(k, extra, E, H):
+    rc = _code("moe_route_topk", None, 4, H, None, None, E, k, extra, 0, None, None, None, None, 0, None)
+    assert rc in (abi.MOE_ERR_UNSUPPORTED, abi.MOE_ERR_INVALID_ARG)
+    assert abi.load().moe_last_error().decode()
+
+
+def test_calls_reject_null_pointers_and_bad_sizes():
+    assert _code("moe_route_topk", None, 4, 256, None, None, 16, 2, 0, 0, None, None, None, None, 0, None) == \
+        abi.MOE_ERR_INVALID_ARG
+    assert _code("moe_permute", None, 4, 2, 2000, None, None, None, None, 0, None) == abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_permute", None, 4, 2, 16, None, None, None, None, 0, None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("moe_grouped_swiglu_bf16", None, None, None, 4, 8, 100, 64, 4, None, None, 0, 0, None, None, 0,
+                 None) == abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_grouped_swiglu_bf16", None, None, None, 4, 8, 256, 64, 4, None, None, 0, 0, None, None, 0,
+                 None) == abi.MOE_ERR_INVALID_ARG  # identity rows need rows == T
+    assert _code("moe_combine", None, 0, None, 2, None, None, None, 4, 3, 256, 0, None, None) == \
+        abi.MOE_ERR_INVALID_ARG  # k > k_slots
+    assert _code("razor_select", None, None, 16, 17, None, None, None, None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("razor_select", None, None, 0, 0, None, None, None, None) == abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_nvfp4_quantize", None, 1, 4, 24, 0, None, None, None, None, None, 0, None) == \
+        abi.MOE_ERR_UNSUPPORTED
+
+
+def test_zero_sized_calls_are_no_ops():
+    # nothing to do: returns OK without touching the device
+    assert _code("moe_route_topk", None, 0, 256, None, None, 16, 2, 0, 0, None, None, None, None, 0, None) == abi.MOE_OK
+    assert _code("moe_grouped_swiglu_bf16", None, ctypes.c_void_p(16), None, 0, 0, 256, 64, 4, None, None, 0, 0, None,
+                 None, 0, None) == abi.MOE_OK
+    assert _code("moe_combine", None, 0, None, 2, None, None, None, 0, 2, 256, 0, None, None) == abi.MOE_OK

@@ -1,0 +1,155 @@
+"""GPU parity of each C-ABI operation against the CPU oracle, element by
+element on seeded inputs.  Integer outputs (routing indices where the logit
+margin exceeds 1e-3, permutations, kept sets, rankings) must match bit for
+bit; floating-point outputs must stay within the normwise relative error
+max|gpu - oracle| / max|oracle| <= 2e-2 that BF16 outputs are held to."""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from bit_expert_gemm_b200 import abi, synth
+from oracle import moe, razor
+from tests.helpers import f64, rel_err
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL_BF16 = 2e-2
+
+
+def _wl(**kw):
+    return dataclasses.replace(synth.WORKLOADS["tiny"], **kw)
+
+
+@pytest.mark.parametrize("T,E,ks", [(0, 16, 2), (1, 512, 10), (7, 16, 2), (64, 512, 10), (1000, 512, 11),
+                                    (4099, 64, 3), (8192, 512, 10), (33, 1024, 16)])
+def test_permute_bit_exact(T, E, ks):
+    idx = synth.make_routing(max(T, 1), E, ks, seed=T + E)[:T].contiguous()
+    off, rt, sr = abi.moe_permute(idx.to(DEV), E)
+    want = moe.permute(idx.numpy().astype(np.int64), E)
+    torch.cuda.synchronize()
+    assert np.array_equal(off.cpu().numpy(), want["offsets"])
+    assert np.array_equal(rt.cpu().numpy(), want["row_token"])
+    assert np.array_equal(sr.cpu().numpy(), want["slot_row"])
+    assert abi.moe_device_status() == 0
+
+
+def test_permute_reports_out_of_range_index():
+    idx = synth.make_routing(16, 16, 2, seed=1).clone()
+    idx[3, 1] = 16  # outside [0, E)
+    abi.moe_permute(idx.to(DEV), 16)
+    assert abi.moe_device_status(clear=True) == abi.MOE_ERR_INVALID_ARG
+    assert abi.moe_device_status() == 0
+
+
+ROUTE_CASES = [
+    # T, H, E, k, extra, bias_std, act  (T >= 256 and E % 64 == 0 take the tensor-core logits path)
+    (64, 256, 16, 2, 0, 1.0, "bf16"),
+    (64, 256, 16, 2, 1, 1.0, "bf16"),
+    (1, 2048, 512, 10, 0, 1.5, "bf16"),
+    (64, 2048, 512, 10, 1, 1.5, "bf16"),
+    (1024, 2048, 512, 10, 0, 1.5, "bf16"),
+    (300, 512, 384, 10, 1, 1.5, "bf16"),
+    (520, 2048, 512, 10, 0, 1.5, "f16"),
+    (32, 2048, 512, 10, 0, 1.5, "f16"),
+]
+
+
+@pytest.mark.parametrize("T,H,E,k,extra,bstd,act", ROUTE_CASES)
+def test_route_topk(T, H, E, k, extra, bstd, act):
+    wl = _wl(H=H, E=E, k=k, bias_std=bstd, act=act)
+    w = synth.make_weights(wl, seed=3, device=DEV)
+    x = synth.make_tokens(wl, T, seed=3, device=DEV)
+    idx, wt, lg = abi.moe_route_topk(x, w["w_router"], w["bias"], k, extra)
+    r = moe.route(f64(x), f64(w["w_router"]), f64(w["bias"]), k, extra)
+    ok = r["margin"] > 1e-3
+    assert ok.mean() > 0.8
+    gi = idx.cpu().numpy()
+    assert np.array_equal(gi[ok], r["idx"][ok])
+    assert np.allclose(wt.cpu().numpy()[ok], r["w"][ok], atol=2e-5, rtol=1e-4)
+    want_logit = np.take_along_axis(r["logits"], gi.astype(np.int64), 1)
+    assert np.allclose(lg.cpu().numpy(), want_logit, atol=2e-3, rtol=1e-4)
+    assert np.allclose(wt.cpu().numpy().sum(1), 1.0, atol=1e-5)
+
+
+def _ffn_case(T, H, I, E, k, act, seed):
+    wl = _wl(H=H, I=I, E=E, k=k, act=act)
+    w = synth.make_weights(wl, seed=seed, device=DEV)
+    if act == "f16":  # 16-bit expert weights follow the activation dtype
+        w["w_gate_up"] = w["w_gate_up"].to(torch.float16)
+        w["w_down"] = w["w_down"].to(torch.float16)
+    x = synth.make_tokens(wl, T, seed=seed, device=DEV)
+    idx = synth.make_routing(T, E, k, seed=seed)
+    return wl, w, x, idx
+
+
+FFN_CASES = [
+    # T, H, I, E, k, act, out_fp32
+    (37, 256, 64, 16, 2, "bf16", False),
+    (300, 512, 128, 8, 3, "bf16", False),
+    (2000, 1024, 256, 32, 4, "bf16", True),
+    (1, 2048, 640, 512, 10, "bf16", False),
+    (64, 2048, 640, 512, 10, "bf16", False),
+    (700, 2048, 640, 64, 10, "bf16", False),
+    (129, 512, 192, 5, 2, "f16", False),
+]
+
+
+@pytest.mark.parametrize("T,H,I,E,k,act,out_fp32", FFN_CASES)
+def test_grouped_swiglu_16bit(T, H, I, E, k, act, out_fp32):
+    wl, w, x, idx = _ffn_case(T, H, I, E, k, act, seed=T + I)
+    off, rt, sr = abi.moe_permute(idx.to(DEV), E)
+    rows = T * k
+    f = abi.moe_grouped_swiglu_bf16(x, rt, off, rows, w["w_gate_up"], w["w_down"], out_fp32=out_fp32)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0
+    perm = moe.permute(idx.numpy().astype(np.int64), E)
+    xs = f64(x)
+    gu, wd = w["w_gate_up"], w["w_down"]
+    ref, _ = moe.routed_outputs(xs, perm, lambda e: (f64(gu[e, :I]), f64(gu[e, I:]), f64(wd[e])))
+    got = f64(f)
+    gsr = sr.cpu().numpy()
+    g_rows = got[gsr.ravel()]
+    r_rows = ref[perm["slot_row"].ravel()]
+    err = rel_err(g_rows, r_rows)
+    assert err <= TOL_BF16, err
+    assert err < 1e-2
+
+
+def test_dense_expert_identity_rows():
+    wl, w, x, _ = _ffn_case(300, 512, 128, 1, 1, "bf16", seed=5)
+    off = torch.tensor([0, 300], dtype=torch.int32, device=DEV)
+    f = abi.moe_grouped_swiglu_bf16(x, None, off, 300, w["w_sh_gate_up"].unsqueeze(0), w["w_sh_down"].unsqueeze(0))
+    sg = f64(w["w_sh_gate_up"])
+    ref, _ = moe.swiglu_expert(f64(x), sg[:64], sg[64:], f64(w["w_sh_down"]))
+    assert rel_err(f64(f), ref) < 1e-2
+
+
+@pytest.mark.parametrize("T,H,E,k,ks,f32", [(1, 2048, 512, 10, 10, False), (300, 512, 16, 3, 4, False),
+                                            (257, 2048, 64, 10, 11, True)])
+def test_combine(T, H, E, k, ks, f32):
+    idx = synth.make_routing(T, E, ks, seed=T)
+    off, rt, sr = abi.moe_permute(idx.to(DEV), E)
+    wl = _wl(H=H)
+    f = synth.make_tokens(wl, T * ks, seed=11, device=DEV)
+    if f32:
+        f = f.float() * 3
+    shared = synth.make_tokens(wl, T, seed=12, device=DEV)
+    wt = synth.make_weights_topk(T, k, seed=T).to(DEV)
+    y = abi.moe_combine(f, sr, wt, shared_out=shared)
+    ref = moe.combine(f64(f), sr.cpu().numpy(), wt.double().cpu().numpy(), f64(shared))
+    assert rel_err(f64(y), ref) < 1e-2
+
+
+@pytest.mark.parametrize("E", [1, 16, 256, 512, 1000, 1024])
+def test_select_bit_exact(E):
+    for seed in range(3):
+        ss, cc = synth.make_refill_stats(E, seed)
+        for keep in sorted({0, 1, E // 2, min(E, 256), E}):
+            kept, ranking, score = abi.razor_select(ss.to(DEV), cc.to(DEV), keep)
+            k_ref, r_ref, s_ref = razor.select(ss.numpy(), cc.numpy(), keep)
+            assert np.array_equal(score.cpu().numpy(), s_ref)
+            assert np.array_equal(ranking.cpu().numpy(), r_ref)
+            assert np.array_equal(kept.cpu().numpy(), k_ref)
