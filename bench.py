@@ -28,7 +28,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -51,6 +50,8 @@ WORKLOADS = {
     "bf16_decode_t8": ("bf16", 8, "forward"),
     "bf16_decode_t64": ("bf16", 64, "forward"),
     "bf16_h2560_prefill": ("bf16_h2560", 8192, "forward"),
+    # small case of the same kernels for full ncu captures (64 experts, 2048 tokens)
+    "profile_e64_t2048": ("profile_e64", 2048, "forward"),
     "refill": ("refill", 32768, "refill"),
 }
 
@@ -108,54 +109,53 @@ class Dist:
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
-              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
-              "clocks_event_reasons.sw_power_cap"]
+    """Polls the SM clock and the clock-event (throttle) reasons through NVML
+    every 2 ms while the timed region runs."""
+
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
     def __init__(self, device_index: int):
-        self.proc = None
-        self.lines = []
+        self.sm, self.mx, self.bits = [], [], 0
+        self.err = None
+        self.stop_flag = threading.Event()
         try:
-            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", uuid, "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except Exception:
-            self.proc = None
+            import pynvml
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.get_reasons = get
+            self.mx.append(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        except Exception as e:  # no NVML: report it instead of a number
+            self.err = f"NVML unavailable: {e}"
+
+    def _sample(self):
+        self.sm.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        self.bits |= int(self.get_reasons(self.h))
+
+    def _run(self):
+        while not self.stop_flag.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def stop(self) -> dict:
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self.err:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err]}
+        self.stop_flag.set()
+        self.t.join(timeout=1)
+        self._sample()
+        reasons = sorted(n for n, b in self.REASONS.items() if self.bits & b)
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": max(self.mx), "reasons": reasons,
+                "samples": len(self.sm)}
 
 
 def measured_peaks() -> dict:
@@ -342,7 +342,7 @@ def run_native(args, dist: Dist) -> None:
         "expert_ffn_ms": round(ffn_ms, 4),
     }
     if dist.rank == 0 and not args.no_cpu_baseline:
-        n = args.cpu_sample_tokens or (8 if kind == "refill" else 16)
+        n = args.cpu_sample_tokens or (96 if kind == "refill" else 192)
         tps, dt = oracle_tokens_per_s(wl, w, xs[0], min(n, T), kind)
         line["cpu_baseline"] = {"value": round(tps, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"first {min(n, T)} tokens of one batch of the same workload, full layer "

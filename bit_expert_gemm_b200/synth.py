@@ -58,6 +58,9 @@ WORKLOADS: Dict[str, Workload] = {
     # RAZOR Refill-RMS scoring pass: one packed row of 32768 tokens
     "refill": Workload("refill", H=2048, E=512, k=10, I=640, I_sh=640, bias_std=1.5, fmt="bf16", act="bf16",
                        T_prefill=32768, keep=256),
+    # small case of the prefill kernels, sized for full profiler captures
+    "profile_e64": Workload("profile_e64", H=2048, E=64, k=10, I=640, I_sh=640, bias_std=1.5, fmt="bf16", act="bf16",
+                            T_prefill=2048),
     # extra, non-graded: the residual width the model's fact sheet states
     "bf16_h2560": Workload("bf16_h2560", H=2560, E=512, k=10, I=640, I_sh=640, bias_std=1.5, fmt="bf16",
                            act="bf16", T_prefill=8192),
