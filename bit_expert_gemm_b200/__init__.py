@@ -9,6 +9,7 @@ function-for-function in `abi`; `MoELayer` chains those calls into a layer.
 
 from . import abi, synth  # noqa: F401
 from .abi import (  # noqa: F401
+    moe_awq_dequant_g32,
     moe_combine,
     moe_device_status,
     moe_grouped_swiglu_awq_g32,

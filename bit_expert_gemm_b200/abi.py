@@ -48,6 +48,7 @@ _SIGS = {
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "moe_grouped_swiglu_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _SZ, _P]),
     "moe_grouped_swiglu_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "moe_awq_dequant_g32": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_nvfp4_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_grouped_swiglu_nvfp4": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ,
                                       _P]),
@@ -198,6 +199,24 @@ def moe_grouped_swiglu_awq_g32(x, row_token, expert_offsets, rows: int, qw_gu, q
           _p(qz_gu), _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), int(out_fp32), _p(f), _p(ws), ws.numel(),
           _stream(stream))
     return f
+
+
+def moe_awq_dequant_g32(qweight, qzeros, scales, out=None, stream=None):
+    """qweight [B, K, N/8] (or [K, N/8]) -> FP16 [B, K, N]: the exact weights
+    the AWQ GEMM multiplies with."""
+    squeeze = qweight.dim() == 2
+    qw = qweight.unsqueeze(0) if squeeze else qweight
+    qz = qzeros.unsqueeze(0) if squeeze else qzeros
+    sc = scales.unsqueeze(0) if squeeze else scales
+    B, K, W = qw.shape
+    N = W * 8
+    _need(qw, torch.int32, "qweight")
+    _need(qz, torch.int32, "qzeros")
+    _need(sc, torch.float16, "scales")
+    if out is None:
+        out = torch.empty((B, K, N), dtype=torch.float16, device=qw.device)
+    _call("moe_awq_dequant_g32", _p(qw), _p(qz), _p(sc), B, K, N, _p(out), _stream(stream))
+    return out[0] if squeeze else out
 
 
 def moe_nvfp4_quantize(v, global_scale_in=None, codes=None, sf=None, global_scale_out=None, ws=None, stream=None):

@@ -32,6 +32,8 @@ int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* o
                        int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
                        const int32_t* qz_d, const void* sc_d, int out_fp32, void* f, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
+int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N, void* out,
+                cudaStream_t stream);
 size_t nvfp4_quant_ws_bytes(int batch, int rows, int K);
 int nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const float* gs_in, uint8_t* codes,
                    uint8_t* sf, float* gs_out, void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -101,7 +103,7 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Tile-width choice of a grouped GEMM from host-known sizes only: the widest
 // tile that still gives at least one tile per SM for an upper bound of the
 // number of row tiles.
-static int pick_bn(int rows, int groups, int n_out, bool swiglu) {
+int pick_bn(int rows, int groups, int n_out, bool swiglu) {
   const long mt = (rows + 127) / 128 + (groups < rows ? groups : rows);
   const int cands[3] = {256, 128, 64};
   int last_ok = 0;
@@ -260,6 +262,17 @@ int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const in
               "moe_grouped_swiglu_awq_g32: null pointer");
   return grouped_swiglu_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
                             out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int moe_awq_dequant_g32(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N,
+                        void* out, void* stream) {
+  MOE_REQUIRE(batch >= 0 && K >= 0 && N >= 0 && K % 32 == 0 && N % 8 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_awq_dequant_g32: need K %% 32 == 0 and N %% 8 == 0 (K=%d N=%d)", K, N);
+  if (long(batch) * K * N == 0) return MOE_OK;
+  MOE_REQUIRE(qweight && qzeros && scales && out, MOE_ERR_INVALID_ARG, "moe_awq_dequant_g32: null pointer");
+  MOE_REQUIRE(aligned16(scales) && aligned16(out), MOE_ERR_INVALID_ARG,
+              "moe_awq_dequant_g32: scales / out must be 16-byte aligned");
+  return awq_dequant(qweight, qzeros, scales, batch, K, N, out, static_cast<cudaStream_t>(stream));
 }
 
 int moe_nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const float* global_scale_in,

@@ -21,6 +21,8 @@ int cuda_status(cudaError_t e, const char* what);
 int* device_status_ptr();            // device address of the status word of the current device
 int num_sms();                       // SMs of the current device
 unsigned long long wait_limit_ns();  // bound of every device-side wait
+// Tile width of a grouped GEMM from host-known sizes (abi.cu).
+int pick_bn(int rows, int groups, int n_out, bool swiglu);
 
 #define MOE_CHECK_CUDA(call)                                   \
   do {                                                         \
@@ -290,6 +292,42 @@ struct Pack2<__half> {
     return __half22float2(v);
   }
 };
+
+// AWQ dequantisation of one packed word: codes q_j (nibble j of W, output
+// column 8w+j), zero points z_j (nibble j of Z) and FP16 scales s_j (S holds
+// s_0..s_7) -> the 8 FP16 values fp16_rn((q_j - z_j) * s_j), as 4 packed
+// pairs (j = 2m low half, 2m+1 high half).  0x6400 | q is the FP16 value
+// 1024 + q, so one subtraction of two such values gives q - z exactly; the
+// single FP16 multiplication then rounds once, to nearest even.
+__device__ __forceinline__ uint32_t awq_pair_1024(uint32_t w, int m) {
+  return ((w >> (8 * m)) & 0xFu) | (((w >> (8 * m + 4)) & 0xFu) << 16) | 0x64006400u;
+}
+__device__ __forceinline__ uint4 awq_dequant8(uint32_t W, uint32_t Z, uint4 S) {
+  const uint32_t sp[4] = {S.x, S.y, S.z, S.w};
+  uint32_t r[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    uint32_t q = awq_pair_1024(W, m), z = awq_pair_1024(Z, m);
+    __half2 d = __hsub2(*reinterpret_cast<__half2*>(&q), *reinterpret_cast<__half2*>(&z));
+    __half2 v = __hmul2(d, *reinterpret_cast<const __half2*>(&sp[m]));
+    r[m] = *reinterpret_cast<uint32_t*>(&v);
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// Shared-memory matrix descriptor of an MN-major operand in the 128-byte
+// swizzled layout: atoms of 64 16-bit elements along MN by 8 rows along K
+// (1024 bytes, 16-byte chunk index XOR (k mod 8)); atoms along K are
+// `sbo` bytes apart, atoms along MN `lbo` bytes apart.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((smem_addr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 

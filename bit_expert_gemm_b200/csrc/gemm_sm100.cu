@@ -10,15 +10,43 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_TILE_BYTES = BM * BK * 2;
-constexpr int kThreads = 192;
+constexpr int kBaseThreads = 192;    // producer, UMMA issuer, 4 epilogue warps
+constexpr int kDequantThreads = 256;  // 8 AWQ dequantisation warps
+constexpr int kSmemBudget = 196 * 1024;
 
-template <int BN>
+enum { W_DENSE = 0, W_AWQ = 1 };
+
+template <int BN, int EPI, int WQ>
 struct GemmCfg {
   static constexpr int B_TILE_BYTES = BN * BK * 2;
-  static constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
-  static constexpr int STAGES = (196 * 1024) / STAGE_BYTES > 8 ? 8 : (196 * 1024) / STAGE_BYTES;
+  // AWQ staging per stage, one TMA box per output half (gate / up for SwiGLU):
+  // codes [64][W2] words, scales [2][8*W2] FP16, zeros [2][W2] words.  Every
+  // box starts on a 128-byte boundary (a requirement of tensor copies).
+  static constexpr int NBOX = (EPI == EPI_SWIGLU) ? 2 : 1;
+  static constexpr int W2 = BN / 8 / NBOX;
+  static constexpr int CODE_BOX = WQ ? BK * W2 * 4 : 0;
+  static constexpr int SCALE_BOX = WQ ? (2 * W2 * 8 * 2 + 127) / 128 * 128 : 0;
+  static constexpr int ZERO_BOX = WQ ? (2 * W2 * 4 + 127) / 128 * 128 : 0;
+  static constexpr int CODE_OFF = A_TILE_BYTES + B_TILE_BYTES;
+  static constexpr int SCALE_OFF = CODE_OFF + NBOX * CODE_BOX;
+  static constexpr int ZERO_OFF = SCALE_OFF + NBOX * SCALE_BOX;
+  static constexpr int RAW_BYTES = ZERO_OFF + NBOX * ZERO_BOX;
+  static constexpr int STAGE_BYTES = (RAW_BYTES + 1023) / 1024 * 1024;  // keep every tile 1024-byte aligned
+  static constexpr int TX_BYTES =
+      A_TILE_BYTES + (WQ ? NBOX * (BK * W2 * 4 + 2 * W2 * 8 * 2 + 2 * W2 * 4) : B_TILE_BYTES);
+  static constexpr int STAGES = kSmemBudget / STAGE_BYTES > 8 ? 8 : kSmemBudget / STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // +1024: alignment slack
   static constexpr uint32_t TMEM_COLS = 2 * BN;                    // two accumulators
+  static constexpr int THREADS = kBaseThreads + (WQ ? kDequantThreads : 0);
+  // MN-major B tile (AWQ): 64-element atoms along N are LBO apart, 8-row K groups SBO apart
+  static constexpr uint32_t B_SBO = 1024;
+  static constexpr uint32_t B_LBO = (BK / 8) * 1024;
+  static_assert(STAGE_BYTES % 1024 == 0 && A_TILE_BYTES % 1024 == 0 && B_TILE_BYTES % 1024 == 0,
+                "swizzled tiles must stay 1024-byte aligned");
+  static_assert(CODE_BOX % 128 == 0 && SCALE_BOX % 128 == 0 && ZERO_BOX % 128 == 0 && CODE_OFF % 128 == 0 &&
+                    SCALE_OFF % 128 == 0 && ZERO_OFF % 128 == 0,
+                "every TMA destination must be 128-byte aligned");
+  static_assert(W2 * 4 >= 16, "TMA boxes need at least 16 bytes per row");
 };
 
 struct TileMap {
@@ -32,15 +60,13 @@ __device__ void build_tile_table(const GemmArgs& a, int* goff, int* tile_start, 
   const int tid = threadIdx.x;
   for (int i = tid; i <= G; i += blockDim.x) goff[i] = a.group_offsets ? a.group_offsets[i] : (i == 0 ? 0 : a.rows);
   __syncthreads();
-  // each thread owns a contiguous chunk of groups
-  const int per = (G + blockDim.x - 1) / blockDim.x;
+  const int per = (G + blockDim.x - 1) / blockDim.x;  // each thread owns a contiguous chunk of groups
   const int g0 = tid * per;
   int local = 0;
   for (int g = g0; g < g0 + per && g < G; ++g) {
     int n = goff[g + 1] - goff[g];
     local += (n > 0 ? (n + BM - 1) / BM : 0);
   }
-  // block exclusive scan of `local`
   const int lane = tid & 31, warp = tid >> 5;
   int incl = local;
 #pragma unroll
@@ -77,30 +103,49 @@ __device__ __forceinline__ TileMap decode_tile(int L, int nt, const int* tile_st
   return t;
 }
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs args) {
-  using Cfg = GemmCfg<BN>;
+// Tensor maps of the B source.  Dense: b = the weight matrix.  AWQ: codes,
+// scales, zeros (b unused).
+struct BMaps {
+  CUtensorMap b, codes, scales, zeros;
+};
+
+template <int BN, int EPI, int WQ>
+__global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ>::THREADS, 1)
+    k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps bm, const GemmArgs args) {
+  using Cfg = GemmCfg<BN, EPI, WQ>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int BNH = (EPI == EPI_SWIGLU) ? BN / 2 : BN;  // output columns per tile
+  constexpr int WC = BN / 8;                               // AWQ code words per K row of the tile
+  constexpr int W2 = Cfg::W2;                              // words per TMA box (gate / up halves)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], bready_bar[STAGES], tfull_bar[2],
+      tempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ int goff[kGemmMaxGroups + 1];
   __shared__ int tile_start[kGemmMaxGroups + 1];
-  __shared__ int warp_sums[kThreads / 32];
+  __shared__ int warp_sums[Cfg::THREADS / 32];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   auto smA = [&](int s) { return smem + s * Cfg::STAGE_BYTES; };
   auto smB = [&](int s) { return smem + s * Cfg::STAGE_BYTES + A_TILE_BYTES; };
+  // AWQ staging box `half` (0: gate / all, 1: up) of stage s
+  auto smCodes = [&](int s, int half) {
+    return reinterpret_cast<uint32_t*>(smA(s) + Cfg::CODE_OFF + half * Cfg::CODE_BOX);
+  };
+  auto smScales = [&](int s, int half) {
+    return reinterpret_cast<uint16_t*>(smA(s) + Cfg::SCALE_OFF + half * Cfg::SCALE_BOX);
+  };
+  auto smZeros = [&](int s, int half) {
+    return reinterpret_cast<uint32_t*>(smA(s) + Cfg::ZERO_OFF + half * Cfg::ZERO_BOX);
+  };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
+      mbar_init(&bready_bar[s], kDequantThreads / 32);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
@@ -112,7 +157,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    if (WQ) {
+      tma_prefetch_desc(&bm.codes);
+      tma_prefetch_desc(&bm.scales);
+      tma_prefetch_desc(&bm.zeros);
+    } else {
+      tma_prefetch_desc(&bm.b);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, Cfg::TMEM_COLS);
@@ -142,15 +193,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileMap t = decode_tile(L, nt, tile_start, G);
         const int a_row = goff[t.g] + t.m * BM;
         const int b_row = t.g * args.b_rows_per_group + t.n * BNH;
+        const int col0 = t.n * BNH;  // AWQ: first output column of the tile (gate half)
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
+          mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
           tma_load_2d(smA(stage), &tmA, &full_bar[stage], kb * BK, a_row);
-          if (EPI == EPI_SWIGLU) {
-            tma_load_2d(smB(stage), &tmB, &full_bar[stage], kb * BK, b_row);
-            tma_load_2d(smB(stage) + BNH * BK * 2, &tmB, &full_bar[stage], kb * BK, b_row + args.up_offset);
+          if (WQ) {
+            const int crow = t.g * args.K + kb * BK;          // code rows (input dim)
+            const int grow = t.g * (args.K / 32) + kb * (BK / 32);  // scale / zero rows (groups)
+            tma_load_2d(smCodes(stage, 0), &bm.codes, &full_bar[stage], col0 / 8, crow);
+            tma_load_2d(smScales(stage, 0), &bm.scales, &full_bar[stage], col0, grow);
+            tma_load_2d(smZeros(stage, 0), &bm.zeros, &full_bar[stage], col0 / 8, grow);
+            if (EPI == EPI_SWIGLU) {
+              const int c1 = args.up_offset + col0;
+              tma_load_2d(smCodes(stage, 1), &bm.codes, &full_bar[stage], c1 / 8, crow);
+              tma_load_2d(smScales(stage, 1), &bm.scales, &full_bar[stage], c1, grow);
+              tma_load_2d(smZeros(stage, 1), &bm.zeros, &full_bar[stage], c1 / 8, grow);
+            }
+          } else if (EPI == EPI_SWIGLU) {
+            tma_load_2d(smB(stage), &bm.b, &full_bar[stage], kb * BK, b_row);
+            tma_load_2d(smB(stage) + BNH * BK * 2, &bm.b, &full_bar[stage], kb * BK, b_row + args.up_offset);
           } else {
-            tma_load_2d(smB(stage), &tmB, &full_bar[stage], kb * BK, b_row);
+            tma_load_2d(smB(stage), &bm.b, &full_bar[stage], kb * BK, b_row);
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -166,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- UMMA issuer ----------------
-      const uint32_t idesc = idesc_f16(args.bf16, BM, BN);
+      const uint32_t idesc = idesc_f16(args.bf16, BM, BN) | (WQ ? (1u << 16) : 0u);  // AWQ: B is MN-major
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -178,12 +242,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem_base + uint32_t(acc * BN);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
+          if (WQ && !mbar_wait(&bready_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = sdesc_kmajor_sw128(smem_u32(smA(stage)));
-          const uint64_t bd = sdesc_kmajor_sw128(smem_u32(smB(stage)));
+          if (WQ) {
+            const uint64_t bd = sdesc_mnmajor_sw128(smem_u32(smB(stage)), Cfg::B_LBO, Cfg::B_SBO);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_f16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < BK / 16; ++kk)  // 16 K = two 8-row groups = 2 * SBO bytes
+              umma_f16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * (2 * Cfg::B_SBO >> 4)), idesc, (kb | kk) != 0);
+          } else {
+            const uint64_t bd = sdesc_kmajor_sw128(smem_u32(smB(stage)));
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_f16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+          }
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -197,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(&drain_bar, 0, &never, nullptr, lim);
     }
-  } else {
+  } else if (warp < 6) {
     // ---------------- epilogue: warps 2..5 ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int row_in_tile = q * 32 + lane;
@@ -265,6 +337,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+  } else if (WQ) {
+    // ---------------- AWQ dequantisation: warps 6..13 ----------------
+    // Thread (wc, r0) turns code word column wc (output columns 8wc..8wc+7)
+    // of K rows r0, r0 + RP, ... into one 16-byte chunk of the MN-major B tile
+    // per row.
+    const int dt = threadIdx.x - kBaseThreads;
+    const int wc = dt % WC;
+    const int r0 = dt / WC;
+    constexpr int RP = kDequantThreads / WC;  // rows per pass
+    const int half = (EPI == EPI_SWIGLU && wc >= W2) ? 1 : 0;
+    const int wl = wc - half * W2;
+    const uint32_t chunk = uint32_t(wc & 7);
+    const uint32_t atom_off = uint32_t(wc >> 3) * Cfg::B_LBO;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { L = total; break; }
+        const uint32_t* codes = smCodes(stage, half) + wl;
+        const uint16_t* sc = smScales(stage, half) + wl * 8;
+        const uint32_t* zr = smZeros(stage, half) + wl;
+        const uint4 s0 = *reinterpret_cast<const uint4*>(sc);
+        const uint4 s1 = *reinterpret_cast<const uint4*>(sc + W2 * 8);
+        const uint32_t z0 = zr[0], z1 = zr[W2];
+        uint8_t* btile = smB(stage) + atom_off;
+#pragma unroll 4
+        for (int r = r0; r < BK; r += RP) {
+          const uint32_t w = codes[r * W2];
+          const uint4 v = r < 32 ? awq_dequant8(w, z0, s0) : awq_dequant8(w, z1, s1);
+          const uint32_t off = uint32_t(r >> 3) * Cfg::B_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
+          *reinterpret_cast<uint4*>(btile + off) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bready_bar[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
   }
 
   tc_fence_before();
@@ -294,45 +404,66 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+// 2-D tensor map of a row-major [rows, cols] matrix of `esize`-byte elements,
+// box [box_rows, box_cols].
+int make_tmap_2d(CUtensorMap* map, const void* base, int rows, int cols, int esize, int box_rows, int box_cols,
+                 CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = get_encode_fn();
+  MOE_REQUIRE(enc != nullptr, MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  MOE_REQUIRE((reinterpret_cast<uintptr_t>(base) & 15) == 0, MOE_ERR_INVALID_ARG, "operand is not 16-byte aligned");
+  MOE_REQUIRE((size_t(cols) * esize) % 16 == 0, MOE_ERR_UNSUPPORTED, "row pitch of %d bytes is not a multiple of 16",
+              cols * esize);
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * esize};
+  cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUtensorMapDataType dt = esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                      : (esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8);
+  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MOE_REQUIRE(r == CUDA_SUCCESS, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a [%d, %d] operand, box [%d, %d]",
+              int(r), rows, cols, box_rows, box_cols);
+  return MOE_OK;
+}
+
 }  // namespace
 
 // 2-D tensor map of a row-major [rows, cols] 16-bit matrix, box [box_rows, 64]
 // with the 128-byte swizzle (the K-major UMMA operand layout).
 int make_tmap_16bit_sw128(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
-  EncodeTiledFn enc = get_encode_fn();
-  MOE_REQUIRE(enc != nullptr, MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  MOE_REQUIRE((reinterpret_cast<uintptr_t>(base) & 15) == 0, MOE_ERR_INVALID_ARG, "operand is not 16-byte aligned");
-  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
-  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  MOE_REQUIRE(r == CUDA_SUCCESS, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a [%d, %d] operand", int(r),
-              rows, cols);
-  return MOE_OK;
+  return make_tmap_2d(map, base, rows, cols, 2, box_rows, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int BN, int EPI>
-static int launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, cudaStream_t stream) {
-  using Cfg = GemmCfg<BN>;
+template <int BN, int EPI, int WQ>
+static int launch_bn(const CUtensorMap& ta, const BMaps& bmaps, const GemmArgs& args, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN, EPI, WQ>;
   static bool attr_set[64] = {false};  // per device
-  auto kern = k_grouped_gemm<BN, EPI>;
+  auto kern = k_grouped_gemm<BN, EPI, WQ>;
   int dev = 0;
   MOE_CHECK_CUDA(cudaGetDevice(&dev));
   if (dev >= 64 || !attr_set[dev]) {
     MOE_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     if (dev < 64) attr_set[dev] = true;
   }
-  int grid = num_sms();
-  kern<<<grid, kThreads, Cfg::SMEM_BYTES, stream>>>(ta, tb, args);
+  kern<<<num_sms(), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, bmaps, args);
   MOE_CHECK_CUDA(cudaGetLastError());
   return MOE_OK;
 }
 
-int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_total, const GemmArgs& args, int epi,
-                        int bn, cudaStream_t stream) {
+template <int WQ>
+static int dispatch(const CUtensorMap& ta, const BMaps& bm, const GemmArgs& args, int epi, int bn,
+                    cudaStream_t stream) {
+  if (epi == EPI_SWIGLU) {
+    if (bn == 256) return launch_bn<256, EPI_SWIGLU, WQ>(ta, bm, args, stream);
+    if (bn == 128) return launch_bn<128, EPI_SWIGLU, WQ>(ta, bm, args, stream);
+    return launch_bn<64, EPI_SWIGLU, WQ>(ta, bm, args, stream);
+  }
+  if (bn == 256) return launch_bn<256, EPI_STORE, WQ>(ta, bm, args, stream);
+  if (bn == 128) return launch_bn<128, EPI_STORE, WQ>(ta, bm, args, stream);
+  return launch_bn<64, EPI_STORE, WQ>(ta, bm, args, stream);
+}
+
+static int check_common(const GemmArgs& args, int epi, int bn) {
   MOE_REQUIRE(args.K % BK == 0 && args.K > 0, MOE_ERR_UNSUPPORTED, "GEMM K=%d is not a positive multiple of 64",
               args.K);
   MOE_REQUIRE(args.G >= 1 && args.G <= kGemmMaxGroups, MOE_ERR_UNSUPPORTED, "GEMM group count %d outside [1, %d]",
@@ -341,20 +472,48 @@ int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_tot
   const int bnh = epi == EPI_SWIGLU ? bn / 2 : bn;
   MOE_REQUIRE(args.n_out % bnh == 0, MOE_ERR_UNSUPPORTED, "output width %d is not a multiple of the tile (%d)",
               args.n_out, bnh);
+  return MOE_OK;
+}
+
+int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_total, const GemmArgs& args, int epi,
+                        int bn, cudaStream_t stream) {
+  int rc = check_common(args, epi, bn);
+  if (rc) return rc;
   if (a_rows == 0) return MOE_OK;
-  CUtensorMap ta, tb;
-  int rc = make_tmap_16bit_sw128(&ta, A, a_rows, args.K, BM);
+  const int bnh = epi == EPI_SWIGLU ? bn / 2 : bn;
+  CUtensorMap ta;
+  BMaps bm;
+  memset(&bm, 0, sizeof(bm));
+  rc = make_tmap_16bit_sw128(&ta, A, a_rows, args.K, BM);
   if (rc) return rc;
-  rc = make_tmap_16bit_sw128(&tb, B, b_rows_total, args.K, bnh);
+  rc = make_tmap_16bit_sw128(&bm.b, B, b_rows_total, args.K, bnh);
   if (rc) return rc;
-  if (epi == EPI_SWIGLU) {
-    if (bn == 256) return launch_bn<256, EPI_SWIGLU>(ta, tb, args, stream);
-    if (bn == 128) return launch_bn<128, EPI_SWIGLU>(ta, tb, args, stream);
-    return launch_bn<64, EPI_SWIGLU>(ta, tb, args, stream);
-  }
-  if (bn == 256) return launch_bn<256, EPI_STORE>(ta, tb, args, stream);
-  if (bn == 128) return launch_bn<128, EPI_STORE>(ta, tb, args, stream);
-  return launch_bn<64, EPI_STORE>(ta, tb, args, stream);
+  return dispatch<W_DENSE>(ta, bm, args, epi, bn, stream);
+}
+
+int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, const int32_t* qzeros,
+                            const void* scales, int n_total, const GemmArgs& args, int epi, int bn,
+                            cudaStream_t stream) {
+  int rc = check_common(args, epi, bn);
+  if (rc) return rc;
+  MOE_REQUIRE(args.bf16 == 0, MOE_ERR_UNSUPPORTED, "AWQ GEMM runs on FP16 activations");
+  MOE_REQUIRE(args.K % 32 == 0, MOE_ERR_UNSUPPORTED, "AWQ K=%d is not a multiple of the group size 32", args.K);
+  if (a_rows == 0) return MOE_OK;
+  const int bnh = epi == EPI_SWIGLU ? bn / 2 : bn;
+  MOE_REQUIRE(bnh % 32 == 0, MOE_ERR_UNSUPPORTED, "AWQ tile half-width %d is not a multiple of 32", bnh);
+  CUtensorMap ta;
+  BMaps bm;
+  memset(&bm, 0, sizeof(bm));
+  rc = make_tmap_16bit_sw128(&ta, A, a_rows, args.K, BM);
+  if (rc) return rc;
+  const int G = args.G;
+  rc = make_tmap_2d(&bm.codes, qweight, G * args.K, n_total / 8, 4, BK, bnh / 8, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+  rc = make_tmap_2d(&bm.scales, scales, G * (args.K / 32), n_total, 2, 2, bnh, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+  rc = make_tmap_2d(&bm.zeros, qzeros, G * (args.K / 32), n_total / 8, 4, 2, bnh / 8, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+  return dispatch<W_AWQ>(ta, bm, args, epi, bn, stream);
 }
 
 }  // namespace moe

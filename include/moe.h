@@ -182,6 +182,16 @@ MOE_API int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, 
                                int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * AWQ dequantisation [AWQ], the same device code the grouped GEMM runs on
+ * each weight tile: out[b, k, n] = fp16_rn((q - z) * s) for `batch` stacked
+ * projections in the layout above (qweight [batch, K, N/8], qzeros
+ * [batch, K/32, N/8], scales [batch, K/32, N]); out [batch, K, N] FP16,
+ * input-major like the stored codes.  Limits: K % 32 == 0, N % 8 == 0.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_awq_dequant_g32(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K,
+                                int N, void* out, void* stream);
+
+/* ---------------------------------------------------------------------------
  * NVFP4 quantisation of `batch` tensors [rows, K] of 16-bit values [NVFP4]
  * (decode-direction scales, every rounding decision in FP32 IEEE
  * round-to-nearest-even, in this order):

@@ -1,0 +1,119 @@
+"""AWQ W4A16 group-32 experts on the GPU against the oracle: dequantised
+weights bit for bit, grouped SwiGLU and whole layers within the 5e-2
+normwise bound of the 4-bit paths (the oracle computes in float64 with its
+own dequantised FP16 weights)."""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from bit_expert_gemm_b200 import MoELayer, abi, synth
+from oracle import awq, moe
+from tests.helpers import f64, rel_err
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL_4BIT = 5e-2
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+@pytest.mark.parametrize("E,K,N", [(3, 64, 64), (2, 2048, 1280), (2, 640, 2048), (1, 96, 24)])
+def test_awq_dequant_bit_exact(E, K, N):
+    wl = dataclasses.replace(synth.WORKLOADS["awq_g32"], H=K, I=N // 2, E=E)
+    w = synth.make_weights(wl, seed=K + N, device=DEV)
+    got = abi.moe_awq_dequant_g32(w["qw_gu"], w["qz_gu"], w["sc_gu"])
+    torch.cuda.synchronize()
+    for e in range(E):
+        ref = awq.dequant(_np(w["qw_gu"][e]), _np(w["qz_gu"][e]), _np(w["sc_gu"][e]))
+        g = _np(got[e].view(torch.int16)).view(np.uint16)
+        r = ref.astype(np.float16).view(np.uint16)
+        assert np.array_equal(g, r)
+
+
+def _awq_expert_fn(w, I):
+    cache = {}
+    host = {k: _np(w[k]) for k in ("qw_gu", "qz_gu", "sc_gu", "qw_d", "qz_d", "sc_d")}
+
+    def ew(e):
+        if e not in cache:
+            cache[e] = awq.expert_weights_out_in(host["qw_gu"], host["qz_gu"], host["sc_gu"], host["qw_d"],
+                                                 host["qz_d"], host["sc_d"], e, I)
+        return cache[e]
+
+    return ew
+
+
+FFN_CASES = [
+    # T, H, I, E, k
+    (37, 256, 64, 16, 2),
+    (300, 512, 128, 8, 3),
+    (1, 2048, 640, 512, 10),
+    (32, 2048, 640, 512, 10),
+    (700, 2048, 640, 64, 10),
+]
+
+
+@pytest.mark.parametrize("T,H,I,E,k", FFN_CASES)
+def test_grouped_swiglu_awq(T, H, I, E, k):
+    wl = dataclasses.replace(synth.WORKLOADS["awq_g32"], H=H, I=I, E=E, k=k)
+    w = synth.make_weights(wl, seed=T + I, device=DEV)
+    x = synth.make_tokens(wl, T, seed=T, device=DEV)
+    idx = synth.make_routing(T, E, k, seed=T + 1)
+    off, rt, sr = abi.moe_permute(idx.to(DEV), E)
+    f = abi.moe_grouped_swiglu_awq_g32(x, rt, off, T * k, w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"], w["qz_d"],
+                                       w["sc_d"], out_fp32=True)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0
+    perm = moe.permute(idx.numpy().astype(np.int64), E)
+    ref, _ = moe.routed_outputs(f64(x), perm, _awq_expert_fn(w, I))
+    g_rows = f64(f)[sr.cpu().numpy().ravel()]
+    r_rows = ref[perm["slot_row"].ravel()]
+    err = rel_err(g_rows, r_rows)
+    assert err <= TOL_4BIT, err
+    assert err < 1e-2  # FP16 h rounding only
+
+
+@pytest.fixture(scope="module")
+def awq_layer():
+    wl = synth.WORKLOADS["awq_g32"]
+    return wl, synth.make_weights(wl, seed=0, device=DEV)
+
+
+def _oracle(wl, w, x):
+    sh = f64(w["w_sh_gate_up"])
+    I = wl.I_sh
+    return moe.moe_layer(f64(x), f64(w["w_router"]), f64(w["bias"]), wl.k, _awq_expert_fn(w, wl.I),
+                         (sh[:I], sh[I:], f64(w["w_sh_down"])))
+
+
+@pytest.mark.parametrize("T", [1, 8, 32])
+def test_awq_layer_decode(awq_layer, T):
+    wl, w = awq_layer
+    layer = MoELayer(w, wl.k, "awq_g32", T_max=T)
+    x = synth.make_tokens(wl, T, seed=0, device=DEV)
+    y = layer.forward(x)
+    ref = _oracle(wl, w, x)
+    ok = ref["route"]["margin"] > 1e-3
+    assert ok.any()
+    err = rel_err(f64(y)[ok], ref["y"][ok])
+    assert err <= TOL_4BIT, err
+
+
+def test_awq_layer_prefill_sampled(awq_layer):
+    wl, w = awq_layer
+    T = wl.T_prefill
+    layer = MoELayer(w, wl.k, "awq_g32", T_max=T)
+    x = synth.make_tokens(wl, T, seed=0, device=DEV)
+    y = layer.forward(x)
+    torch.cuda.synchronize()
+    sample = np.concatenate([np.random.default_rng(1).choice(T, 16, replace=False), [0, T - 1]])
+    ref = _oracle(wl, w, x[torch.as_tensor(sample, device=DEV)])
+    ok = ref["route"]["margin"] > 1e-3
+    err = rel_err(f64(y)[sample][ok], ref["y"][ok])
+    assert err <= TOL_4BIT, err
+    assert abi.moe_device_status() == 0
