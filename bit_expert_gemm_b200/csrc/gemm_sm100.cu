@@ -434,6 +434,12 @@ int make_tmap_16bit_sw128(CUtensorMap* map, const void* base, int rows, int cols
   return make_tmap_2d(map, base, rows, cols, 2, box_rows, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// 2-D tensor map of a row-major [rows, cols_bytes] byte matrix (packed FP4),
+// box [box_rows, 128 bytes] with the 128-byte swizzle.
+int make_tmap_2d_u8_sw128(CUtensorMap* map, const void* base, int rows, int cols_bytes, int box_rows) {
+  return make_tmap_2d(map, base, rows, cols_bytes, 1, box_rows, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 template <int BN, int EPI, int WQ>
 static int launch_bn(const CUtensorMap& ta, const BMaps& bmaps, const GemmArgs& args, cudaStream_t stream) {
   using Cfg = GemmCfg<BN, EPI, WQ>;

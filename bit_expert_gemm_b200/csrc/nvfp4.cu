@@ -1,20 +1,191 @@
-// NVFP4 W4A4 quantisation and grouped SwiGLU (kernels follow in a later change).
+// NVFP4 W4A4: per-tensor amax, group-16 quantisation (E2M1 codes, E4M3 block
+// scales, FP32 global scale), and the grouped SwiGLU built on the
+// block-scaled tcgen05 GEMM (gemm_nvfp4.cu).
 #include "common.cuh"
+#include "nvfp4.cuh"
 
 namespace moe {
 
-size_t nvfp4_quant_ws_bytes(int batch, int rows, int K) { (void)batch; (void)rows; (void)K; return 256; }
-size_t nvfp4_ws_bytes(int rows, int H, int I, int E) { (void)rows; (void)H; (void)I; (void)E; return 256; }
+int gather_rows(const void* x, const int32_t* row_token, int rows, int H, void* out, cudaStream_t stream);
 
-int nvfp4_quantize(const void*, int, int, int, int, const float*, uint8_t*, uint8_t*, float*, void*, size_t,
-                   cudaStream_t) {
-  return set_error(MOE_ERR_UNSUPPORTED, "moe_nvfp4_quantize: not built in this library version");
+struct Nvfp4GemmArgs;  // gemm_nvfp4.cu
+int launch_grouped_gemm_nvfp4(const uint8_t* A, const uint8_t* sfa, int a_rows, const uint8_t* B, const uint8_t* sfb,
+                              int b_rows_total, const int* group_offsets, int G, int rows, int K, int n_out,
+                              int b_rows_per_group, int up_offset, int swiglu, const float* gs_act,
+                              const float* gs_w, int gs_w_stride, void* out, int ldo, int out_fp32, float* amax_out,
+                              cudaStream_t stream);
+
+// amax[b] = max |v| over tensor b of `batch` tensors of `n` 16-bit values
+// (stored as float bits: non-negative floats order like integers).
+template <typename T16>
+__global__ void __launch_bounds__(256) k_amax(const T16* __restrict__ v, long n, int batch, unsigned* __restrict__ amax) {
+  const int b = blockIdx.y;
+  const uint4* p = reinterpret_cast<const uint4*>(v + b * n);
+  const long nv = n / 8;
+  float m = 0.0f;
+  for (long i = long(blockIdx.x) * blockDim.x + threadIdx.x; i < nv; i += long(gridDim.x) * blockDim.x) {
+    uint4 q = __ldg(p + i);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = Pack2<T16>::unpack(w[j]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax + b, __float_as_uint(m));
 }
 
-int grouped_swiglu_nvfp4(const void*, const int32_t*, const int32_t*, int, int, int, int, int, const uint8_t*,
-                         const uint8_t*, const float*, const uint8_t*, const uint8_t*, const float*, const float*,
-                         float*, int, void*, void*, size_t, cudaStream_t) {
-  return set_error(MOE_ERR_UNSUPPORTED, "moe_grouped_swiglu_nvfp4: not built in this library version");
+// One thread per block of 16 values of row r of tensor b.  Source row of
+// output row r: row_token[r] when given (a gather), else r.  s_g = gs_in[b]
+// when given, else amax[b] / 2688; thread 0 of each tensor writes gs_out[b].
+template <typename T16>
+__global__ void __launch_bounds__(256) k_nvfp4_quant(const T16* __restrict__ v, const int32_t* __restrict__ row_token,
+                                                     int rows, int K, long src_tensor_stride,
+                                                     const float* __restrict__ gs_in,
+                                                     const unsigned* __restrict__ amax, uint8_t* __restrict__ codes,
+                                                     uint8_t* __restrict__ sf, float* __restrict__ gs_out) {
+  const int b = blockIdx.y;
+  const int nb = K / 16;
+  const long i = long(blockIdx.x) * blockDim.x + threadIdx.x;
+  const float s_g = gs_in ? gs_in[b] : nvfp4_global_scale(__uint_as_float(amax[b]));
+  if (i == 0 && gs_out) gs_out[b] = s_g;
+  if (i >= long(rows) * nb) return;
+  const int r = int(i / nb);
+  const int blk = int(i - long(r) * nb);
+  const long src_row = row_token ? row_token[r] : r;
+  const uint4* src = reinterpret_cast<const uint4*>(v + b * src_tensor_stride + src_row * K + blk * 16);
+  float x[16];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint4 q = __ldg(src + h);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = Pack2<T16>::unpack(w[j]);
+      x[8 * h + 2 * j] = f.x;
+      x[8 * h + 2 * j + 1] = f.y;
+    }
+  }
+  uint32_t c[2];
+  const uint32_t s = nvfp4_quant_block(x, s_g, c);
+  const long out_row = long(b) * rows + r;
+  *reinterpret_cast<uint2*>(codes + out_row * (K / 2) + blk * 8) = make_uint2(c[0], c[1]);
+  sf[out_row * nb + blk] = uint8_t(s);
+}
+
+// amax_n > 0: reduce amax over the first amax_n values of each tensor
+// first; amax_n == 0: amax already holds it (or gs_in is given).
+template <typename T16>
+static int quant_impl(const void* v, const int32_t* row_token, int batch, int rows, int K, long src_tensor_stride,
+                      long amax_n, const float* gs_in, unsigned* amax, uint8_t* codes, uint8_t* sf, float* gs_out,
+                      cudaStream_t stream) {
+  const T16* src = static_cast<const T16*>(v);
+  if (!gs_in && amax_n > 0) {
+    MOE_CHECK_CUDA(cudaMemsetAsync(amax, 0, sizeof(unsigned) * batch, stream));
+    const long nv = amax_n / 8;
+    const int gx = int(std::min<long>((nv + 255) / 256, long(num_sms()) * 8));
+    k_amax<T16><<<dim3(gx > 0 ? gx : 1, batch), 256, 0, stream>>>(src, amax_n, batch, amax);
+    MOE_CHECK_CUDA(cudaGetLastError());
+  }
+  const long n = long(rows) * (K / 16);
+  if (n == 0) return MOE_OK;
+  k_nvfp4_quant<T16><<<dim3(int((n + 255) / 256), batch), 256, 0, stream>>>(src, row_token, rows, K,
+                                                                               src_tensor_stride, gs_in, amax, codes,
+                                                                               sf, gs_out);
+  MOE_CHECK_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+static int quantize_rows(const void* v, int dtype, const int32_t* row_token, int batch, int rows, int K,
+                         long src_tensor_stride, long amax_n, const float* gs_in, unsigned* amax, uint8_t* codes,
+                         uint8_t* sf, float* gs_out, cudaStream_t stream) {
+  if (dtype == MOE_DTYPE_BF16)
+    return quant_impl<__nv_bfloat16>(v, row_token, batch, rows, K, src_tensor_stride, amax_n, gs_in, amax, codes, sf,
+                                     gs_out, stream);
+  return quant_impl<__half>(v, row_token, batch, rows, K, src_tensor_stride, amax_n, gs_in, amax, codes, sf, gs_out,
+                            stream);
+}
+
+size_t nvfp4_quant_ws_bytes(int batch, int rows, int K) {
+  (void)rows;
+  (void)K;
+  WsCounter c;
+  c.take<unsigned>(size_t(batch > 0 ? batch : 1));
+  return c.used;
+}
+
+int nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const float* gs_in, uint8_t* codes,
+                   uint8_t* sf, float* gs_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  WsCarver carve(ws, ws_bytes);
+  unsigned* amax = carve.take<unsigned>(size_t(batch));
+  MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_nvfp4_quantize: workspace of %zu bytes is too small", ws_bytes);
+  const long n = long(rows) * K;
+  return quantize_rows(v, dtype, nullptr, batch, rows, K, n, n, gs_in, amax, codes, sf, gs_out, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Grouped SwiGLU with NVFP4 weights and on-the-fly NVFP4 activations:
+//   amax(x) -> quantise gathered rows -> GEMM1 (+SwiGLU, h in BF16, amax(h))
+//   -> quantise h -> GEMM2.
+// ---------------------------------------------------------------------------
+struct Nvfp4Ws {
+  uint8_t *xq, *xsf, *hq, *hsf;
+  uint16_t* h;
+  unsigned* amax;  // [2]: x, h
+  float* gs;       // [2]: x, h
+};
+
+template <typename C>
+static void carve_nvfp4(C& c, int rows, int H, int I) {
+  c.template take<uint8_t>(size_t(rows) * H / 2);
+  c.template take<uint8_t>(size_t(rows) * H / 16);
+  c.template take<uint8_t>(size_t(rows) * I / 2);
+  c.template take<uint8_t>(size_t(rows) * I / 16);
+  c.template take<uint16_t>(size_t(rows) * I);
+  c.template take<unsigned>(2);
+  c.template take<float>(2);
+}
+
+size_t nvfp4_ws_bytes(int rows, int H, int I, int E) {
+  (void)E;
+  WsCounter c;
+  carve_nvfp4(c, rows, H, I);
+  return c.used;
+}
+
+int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
+                         int I, int E, const uint8_t* w_gu, const uint8_t* sf_gu, const float* gs_gu,
+                         const uint8_t* w_d, const uint8_t* sf_d, const float* gs_d, const float* act_gs_in,
+                         float* act_gs_out, int out_fp32, void* f, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  WsCarver carve(ws, ws_bytes);
+  Nvfp4Ws w;
+  w.xq = carve.take<uint8_t>(size_t(rows) * H / 2);
+  w.xsf = carve.take<uint8_t>(size_t(rows) * H / 16);
+  w.hq = carve.take<uint8_t>(size_t(rows) * I / 2);
+  w.hsf = carve.take<uint8_t>(size_t(rows) * I / 16);
+  w.h = carve.take<uint16_t>(size_t(rows) * I);
+  w.amax = carve.take<unsigned>(2);
+  w.gs = carve.take<float>(2);
+  MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_grouped_swiglu_nvfp4: workspace of %zu bytes is too small", ws_bytes);
+  if (rows == 0) return MOE_OK;
+  // x: amax over the whole [T, H] input, quantise the gathered rows
+  int rc = quantize_rows(x, MOE_DTYPE_BF16, row_token, 1, rows, H, 0, long(T) * H, act_gs_in, w.amax, w.xq, w.xsf,
+                         w.gs, stream);
+  if (rc) return rc;
+  MOE_CHECK_CUDA(cudaMemsetAsync(w.amax + 1, 0, sizeof(unsigned), stream));
+  rc = launch_grouped_gemm_nvfp4(w.xq, w.xsf, rows, w_gu, sf_gu, E * 2 * I, offsets, E, rows, H, I, 2 * I, I, 1, w.gs,
+                                 gs_gu, 2, w.h, I, 0, reinterpret_cast<float*>(w.amax + 1), stream);
+  if (rc) return rc;
+  rc = quantize_rows(w.h, MOE_DTYPE_BF16, nullptr, 1, rows, I, 0, 0, act_gs_in ? act_gs_in + 1 : nullptr, w.amax + 1,
+                     w.hq, w.hsf, w.gs + 1, stream);
+  if (rc) return rc;
+  rc = launch_grouped_gemm_nvfp4(w.hq, w.hsf, rows, w_d, sf_d, E * H, offsets, E, rows, I, H, H, 0, 0, w.gs + 1, gs_d,
+                                 1, f, H, out_fp32, nullptr, stream);
+  if (rc) return rc;
+  if (act_gs_out) MOE_CHECK_CUDA(cudaMemcpyAsync(act_gs_out, w.gs, 2 * sizeof(float), cudaMemcpyDeviceToDevice, stream));
+  return MOE_OK;
 }
 
 }  // namespace moe

@@ -22,6 +22,23 @@ import torch
 from . import abi
 
 
+def prepare_nvfp4_weights(w: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
+    """Adds NVFP4 copies of the 16-bit expert weights, quantised by the
+    library (moe_nvfp4_quantize): gate, up and down of every expert are
+    separate tensors with their own global scale.
+    w_gu [E, 2I, H/2], sf_gu [E, 2I, H/16], gs_gu [E, 2]; w_d [E, H, I/2],
+    sf_d [E, H, I/16], gs_d [E]."""
+    gu, wd = w["w_gate_up"], w["w_down"]
+    E, I2, H = gu.shape
+    I = I2 // 2
+    c, sf, gs = abi.moe_nvfp4_quantize(gu.reshape(2 * E, I, H))
+    out = dict(w)
+    out["w_gu"], out["sf_gu"], out["gs_gu"] = c.reshape(E, I2, H // 2), sf.reshape(E, I2, H // 16), gs.reshape(E, 2)
+    c, sf, gs = abi.moe_nvfp4_quantize(wd)
+    out["w_d"], out["sf_d"], out["gs_d"] = c, sf, gs
+    return out
+
+
 class MoELayer:
     def __init__(self, weights: Dict[str, torch.Tensor], k: int, fmt: str = "bf16", T_max: int = 8192,
                  extra: int = 0, device: Optional[torch.device] = None):
@@ -38,6 +55,8 @@ class MoELayer:
         elif fmt == "awq_g32":
             self.I = weights["qw_gu"].shape[2] * 8 // 2
         elif fmt == "nvfp4":
+            if "w_gu" not in weights:
+                self.w = weights = prepare_nvfp4_weights(weights)
             self.I = weights["w_gu"].shape[1] // 2
         else:
             raise ValueError(fmt)

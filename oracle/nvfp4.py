@@ -92,3 +92,73 @@ def fake_quant(v: np.ndarray, s_g=None) -> np.ndarray:
     """quantise -> dequantise, float64."""
     c, sb, g = quantize(v, s_g)
     return dequant(c, sb, g)
+
+
+def routed_outputs_w4a4(x: np.ndarray, perm: dict, expert_weights_deq, act_gs=None):
+    """Routed expert outputs of an NVFP4 W4A4 layer, float64.
+
+    x [T, H] holds the 16-bit activations (as float64).  The activations are
+    quantised as one tensor (global scale over all of x, or act_gs[0]); each
+    expert runs SwiGLU on its rows with its dequantised weights
+    (expert_weights_deq(e) -> (w_gate [I,H], w_up [I,H], w_down [H,I])); the
+    intermediate h of all permuted rows is quantised as one tensor (global
+    scale over all rows, or act_gs[1]) before the down projection.  h is a
+    16-bit activation tensor like every other activation of the layer: it is
+    rounded to BF16 before its amax and its codes are taken, so that the
+    quantisation decisions are made in the same precision as the kernel's.
+    Returns (f [rows, H], h [rows, I] before rounding, (s_x, s_h))."""
+    from . import moe
+    from .formats import bf16_to_f64, f32_to_bf16
+
+    x32 = np.asarray(x, np.float64).astype(np.float32)
+    s_x = None if act_gs is None else np.float32(act_gs[0])
+    xq = fake_quant(x32, s_x)
+    s_x = global_scale(x32) if act_gs is None else np.float32(act_gs[0])
+    offsets, row_token = perm["offsets"], perm["row_token"]
+    E = len(offsets) - 1
+    R = len(row_token)
+    h_all = None
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if a == b:
+            continue
+        wg, wu, _ = expert_weights_deq(e)
+        xe = xq[row_token[a:b]]
+        he = moe.silu(xe @ wg.T) * (xe @ wu.T)
+        if h_all is None:
+            h_all = np.zeros((R, he.shape[1]), np.float64)
+        h_all[a:b] = he
+    h32 = bf16_to_f64(f32_to_bf16(h_all.astype(np.float32))).astype(np.float32)
+    s_h = global_scale(h32) if act_gs is None else np.float32(act_gs[1])
+    hq = fake_quant(h32, s_h)
+    f = None
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if a == b:
+            continue
+        _, _, wd = expert_weights_deq(e)
+        fe = hq[a:b] @ wd.T
+        if f is None:
+            f = np.zeros((R, fe.shape[1]), np.float64)
+        f[a:b] = fe
+    return f, h_all, (s_x, s_h)
+
+
+def quantize_expert_weights(w_gate_up: np.ndarray, w_down: np.ndarray):
+    """Per-(expert, projection) quantisation of 16-bit weights given as
+    float64 arrays w_gate_up [E, 2I, H] (gate rows then up rows) and w_down
+    [E, H, I]: gate, up and down of each expert are separate tensors with
+    their own global scale.  Returns a function e -> dequantised float64
+    (w_gate, w_up, w_down) and the raw (codes, scale codes, global scale)
+    triples as dict[(e, name)]."""
+    E, I2, _ = w_gate_up.shape
+    I = I2 // 2
+    raw = {}
+    deq = {}
+    for e in range(E):
+        parts = {"gate": w_gate_up[e, :I], "up": w_gate_up[e, I:], "down": w_down[e]}
+        for name, wmat in parts.items():
+            c, sb, g = quantize(wmat.astype(np.float32))
+            raw[(e, name)] = (c, sb, g)
+            deq[(e, name)] = dequant(c, sb, g)
+    return (lambda e: (deq[(e, "gate")], deq[(e, "up")], deq[(e, "down")])), raw

@@ -111,3 +111,36 @@ def test_nvfp4_static_scale_saturates():
     v = np.array([[100.0] + [0.0] * 15], np.float32)
     c, sb, g = nvfp4.quantize(v, s_g=np.float32(1e-3))  # 6*448*1e-3 = 2.688 < 100
     assert sb[0, 0] == 0x7E and c[0, 0] == 0x7
+
+
+def test_w4a4_experts_compose_pinned_pieces():
+    """The W4A4 expert path equals the pinned SwiGLU expert run on the
+    globally fake-quantised activations, with h fake-quantised as ONE tensor
+    over all permuted rows (not per expert) before the down projection."""
+    from oracle import moe
+    rng = np.random.default_rng(7)
+    T, H, I, E, k = 24, 64, 32, 3, 2
+    x = rng.standard_normal((T, H)).astype(np.float32).astype(np.float64)
+    wgu = rng.standard_normal((E, 2 * I, H)) / 8
+    wd = rng.standard_normal((E, H, I)) / 6
+    deq, _ = nvfp4.quantize_expert_weights(wgu, wd)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+    perm = moe.permute(idx, E)
+    f, h, (s_x, s_h) = nvfp4.routed_outputs_w4a4(x, perm, deq)
+    xq = nvfp4.fake_quant(x.astype(np.float32))
+    h_ref = np.zeros_like(h)
+    for e in range(E):
+        a, b = perm["offsets"][e], perm["offsets"][e + 1]
+        _, h_ref[a:b] = moe.swiglu_expert(xq[perm["row_token"][a:b]], *deq(e))
+    assert np.allclose(h, h_ref, rtol=1e-12, atol=1e-12)
+    # h is rounded to BF16 (torch's rounding) before it is quantised, as one tensor
+    h16 = torch.from_numpy(h.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    assert s_h == nvfp4.global_scale(h16)  # one scale for all rows
+    hq = nvfp4.fake_quant(h16)
+    for e in range(E):
+        a, b = perm["offsets"][e], perm["offsets"][e + 1]
+        assert np.allclose(f[a:b], hq[a:b] @ deq(e)[2].T, rtol=1e-12, atol=1e-12)
+    # a static activation scale is used as given (a power-of-two factor would be
+    # absorbed exactly by the block scales; a 20x smaller one saturates them)
+    f2, _, (sx2, sh2) = nvfp4.routed_outputs_w4a4(x, perm, deq, act_gs=(s_x / 20, s_h / 20))
+    assert sx2 == np.float32(s_x / 20) and not np.allclose(f2, f)
