@@ -307,8 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 16; ++i) {
               const float h0 = silu_f(gv[2 * i] * sg) * (uv[2 * i] * su);
               const float h1 = silu_f(gv[2 * i + 1] * sg) * (uv[2 * i + 1] * su);
-              hmax = fmaxf(hmax, fmaxf(fabsf(h0), fabsf(h1)));
               pk[i] = Pack2<__nv_bfloat16>::pack(h0, h1);
+              // the amax is taken on the stored BF16 values, the ones that get quantised
+              const float2 r = Pack2<__nv_bfloat16>::unpack(pk[i]);
+              hmax = fmaxf(hmax, fmaxf(fabsf(r.x), fabsf(r.y)));
             }
             uint16_t* dst = reinterpret_cast<uint16_t*>(args.out) + out_row * size_t(args.ldo) + t.n * (BN / 2) + c * 32;
 #pragma unroll
