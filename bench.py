@@ -49,6 +49,11 @@ WORKLOADS = {
     "bf16_decode_t1": ("bf16", 1, "forward"),
     "bf16_decode_t8": ("bf16", 8, "forward"),
     "bf16_decode_t64": ("bf16", 64, "forward"),
+    "awq_prefill": ("awq_g32", 8192, "forward"),
+    "awq_decode_t1": ("awq_g32", 1, "forward"),
+    "awq_decode_t8": ("awq_g32", 8, "forward"),
+    "awq_decode_t32": ("awq_g32", 32, "forward"),
+    "nvfp4_prefill": ("nvfp4", 16384, "forward"),
     "bf16_h2560_prefill": ("bf16_h2560", 8192, "forward"),
     # small case of the same kernels for full ncu captures (64 experts, 2048 tokens)
     "profile_e64_t2048": ("profile_e64", 2048, "forward"),
@@ -64,6 +69,7 @@ def parse():
     p.add_argument("--workload", default="bf16_prefill", choices=sorted(WORKLOADS))
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-graph", action="store_true", help="launch the C-ABI calls eagerly instead of a CUDA graph")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=0, help="oracle sample size (0: automatic)")
     return p.parse_args()
@@ -180,7 +186,7 @@ def blas_threads() -> int:
 
 def oracle_tokens_per_s(wl, w, x: torch.Tensor, n_tokens: int, kind: str):
     """Runs the float64 oracle on the first n_tokens tokens; returns (tokens/s, seconds)."""
-    from oracle import moe, razor
+    from oracle import awq, moe, nvfp4, razor
 
     I = wl.I
 
@@ -188,11 +194,20 @@ def oracle_tokens_per_s(wl, w, x: torch.Tensor, n_tokens: int, kind: str):
         return t.detach().float().cpu().double().numpy()
 
     cache = {}
+    if wl.fmt == "awq_g32":
+        host = {k: w[k].cpu().numpy() for k in EXPERT_KEYS["awq_g32"]}
 
     def ew(e):
         if e not in cache:
-            g = to64(w["w_gate_up"][e])
-            cache[e] = (g[:I], g[I:], to64(w["w_down"][e]))
+            if wl.fmt == "awq_g32":
+                cache[e] = awq.expert_weights_out_in(host["qw_gu"], host["qz_gu"], host["sc_gu"], host["qw_d"],
+                                                     host["qz_d"], host["sc_d"], e, I)
+            else:
+                g = to64(w["w_gate_up"][e])
+                ws = (g[:I], g[I:], to64(w["w_down"][e]))
+                if wl.fmt == "nvfp4":
+                    ws = tuple(nvfp4.fake_quant(m.astype(np.float32)) for m in ws)
+                cache[e] = ws
         return cache[e]
 
     xs = to64(x[:n_tokens])
@@ -207,6 +222,11 @@ def oracle_tokens_per_s(wl, w, x: torch.Tensor, n_tokens: int, kind: str):
         s, c = np.zeros(wl.E), np.zeros(wl.E, np.int64)
         razor.accumulate(s, c, d, r["idx"], wl.k)
         razor.select(s, c, wl.keep)
+    elif wl.fmt == "nvfp4":
+        r = moe.route(xs, wr, b, wl.k)
+        perm = moe.permute(r["idx"], wl.E)
+        f, _, _ = nvfp4.routed_outputs_w4a4(xs, perm, ew)
+        moe.combine(f, perm["slot_row"], r["w"], moe.swiglu_expert(xs, *shared)[0])
     else:
         moe.moe_layer(xs, wr, b, wl.k, ew, shared)
     dt = time.perf_counter() - t0
@@ -216,6 +236,49 @@ def oracle_tokens_per_s(wl, w, x: torch.Tensor, n_tokens: int, kind: str):
 # ---------------------------------------------------------------------------
 def expert_flops(rows: int, H: int, I: int) -> float:
     return 2.0 * rows * 3 * H * I
+
+
+EXPERT_KEYS = {"bf16": ("w_gate_up", "w_down"), "awq_g32": ("qw_gu", "qz_gu", "sc_gu", "qw_d", "qz_d", "sc_d"),
+               "nvfp4": ("w_gu", "sf_gu", "gs_gu", "w_d", "sf_d", "gs_d")}
+KERNEL_NAMES = {"bf16": "moe_grouped_swiglu_bf16 (row gather + GEMM1/SwiGLU + GEMM2, tcgen05 kind::f16)",
+                "awq_g32": "moe_grouped_swiglu_awq_g32 (row gather + dequantising GEMM1/SwiGLU + GEMM2, tcgen05 "
+                           "kind::f16)",
+                "nvfp4": "moe_grouped_swiglu_nvfp4 (activation quantisation + GEMM1/SwiGLU + h quantisation + GEMM2, "
+                         "tcgen05 kind::mxf4nvf4)"}
+
+
+def expert_roofline(wl, layer, T, rows, ffn_ms, peaks) -> dict:
+    """Roofline of the routed expert call: tensor-bound (algorithmic FLOPs)
+    for prefill-sized batches, HBM-bound (bytes of the distinct experts the
+    batch touches) for decode-sized ones."""
+    w = layer.w
+    keys = EXPERT_KEYS[wl.fmt]
+    per_expert = sum(w[k].numel() * w[k].element_size() for k in keys) / wl.E
+    counts = torch.diff(layer.offsets.to(torch.int64)).cpu()
+    touched = int((counts > 0).sum())
+    expert_bytes = touched * per_expert
+    flops = expert_flops(rows, wl.H, wl.I)
+    if T >= 256:
+        if wl.fmt == "nvfp4":
+            base = peaks.get("bf16_tflops_sustained")
+            peak = 4.0 * base if base else 4.0 * 1400.0
+            src = ("derived: 4 x measured sustained BF16 (MEASURED_PEAKS.json bf16_tflops_sustained) x the nominal "
+                   "FP4:BF16 ratio 9/2.25")
+        else:
+            peak = peaks.get("bf16_tflops_sustained", 1400.0)
+            src = ("measured (MEASURED_PEAKS.json bf16_tflops_sustained: kernel timed inside a multi-second loop; "
+                   "FP16 runs at the BF16 rate)")
+        achieved = flops / (ffn_ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None, "kernel": KERNEL_NAMES[wl.fmt],
+                "work_per_launch": f"{flops / 1e9:.1f} GFLOP = 2*rows*3*H*I, rows={rows}", "peak_source": src,
+                "experts_touched": touched}
+    peak = peaks.get("hbm_gbs", 6650.0)
+    achieved = expert_bytes / (ffn_ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None, "kernel": KERNEL_NAMES[wl.fmt],
+            "work_per_launch": f"{expert_bytes / 1e6:.2f} MB = {touched} experts x {per_expert / 1e6:.3f} MB",
+            "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)", "experts_touched": touched}
 
 
 def run_native(args, dist: Dist) -> None:
@@ -236,22 +299,13 @@ def run_native(args, dist: Dist) -> None:
     kept = torch.empty(max(wl.keep, 1), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
-    ffn_ev = []
-
-    def step(i: int, record: bool):
-        x = xs[i % n_batches]
-        if kind == "refill":
-            layer.route(x)
-        else:
-            layer.route(x)
-        if record:
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+    def step(x, ev=None):
+        layer.route(x)
+        if ev:
+            ev[0].record()
         f = layer.experts(x)
-        if record:
-            e1.record(stream)
-            ffn_ev.append((e0, e1))
+        if ev:
+            ev[1].record()
         sh = layer.shared_expert(x)
         if kind == "refill":
             abi.razor_refill_rms_accumulate(f, layer.slot_row[:T], layer.topk_idx[:T], layer.topk_logit[:T],
@@ -261,8 +315,22 @@ def run_native(args, dist: Dist) -> None:
         else:
             abi.moe_combine(f, layer.slot_row[:T], layer.topk_w[:T], shared_out=sh, y=layer.y[:T])
 
+    # one CUDA graph per token batch; each holds timing events around the
+    # routed expert call (external event nodes, read after the timed region)
+    ev_pairs = [(torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n_batches)]
+    graphs = None
+    if not args.no_graph:
+        graphs = [layer.capture(xs[b], lambda x, ev=ev_pairs[b]: step(x, ev)) for b in range(n_batches)]
+
+    def run(i):
+        if graphs:
+            graphs[i % n_batches].replay()
+        else:
+            step(xs[i % n_batches], ev_pairs[i % n_batches])
+
     for i in range(args.warmup):
-        step(i, False)
+        run(i)
     torch.cuda.synchronize()
     assert abi.moe_device_status() == 0, "device status after warm-up"
 
@@ -273,15 +341,16 @@ def run_native(args, dist: Dist) -> None:
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        step(i, True)
+        run(i)
     t_end.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
     clk = clocks.stop()
     ms_local = t_start.elapsed_time(t_end) / args.steps
     ms = dist.max(ms_local)
-    ffn_ms = statistics.mean(a.elapsed_time(b) for a, b in ffn_ev)
-    ffn_ms = dist.max(ffn_ms)
+    # the expert call of the last replay of every batch's graph (inside the timed region)
+    used = sorted({i % n_batches for i in range(max(0, args.steps - n_batches), args.steps)})
+    ffn_ms = dist.max(statistics.mean(ev_pairs[b][0].elapsed_time(ev_pairs[b][1]) for b in used))
     status = abi.moe_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -290,17 +359,7 @@ def run_native(args, dist: Dist) -> None:
     tokens = T * dist.world
     value = tokens / (ms / 1e3)
     peaks = measured_peaks()
-    peak_kind = "bf16_tflops_sustained"
-    peak = peaks.get(peak_kind)
-    peak_note = "measured (MEASURED_PEAKS.json bf16_tflops_sustained: kernel timed inside a multi-second loop)"
-    if peak is None:
-        peak, peak_note = 1400.0, "fallback (no MEASURED_PEAKS.json)"
-    achieved = expert_flops(rows, wl.H, wl.I) / (ffn_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
-                "kernel": "moe_grouped_swiglu_bf16 (row gather + GEMM1/SwiGLU + GEMM2)",
-                "work_per_launch": f"{expert_flops(rows, wl.H, wl.I) / 1e9:.1f} GFLOP = 2*rows*3*H*I, rows={rows}",
-                "peak_source": peak_note}
+    roofline = expert_roofline(wl, layer, T, rows, ffn_ms, peaks)
 
     # end-to-end through the public API: pinned host x -> y in pinned host memory
     e2e = None
@@ -308,33 +367,46 @@ def run_native(args, dist: Dist) -> None:
         xh = [xs[b].cpu().pin_memory() for b in range(n_batches)]
         yh = torch.empty((T, wl.H), dtype=layer.y.dtype).pin_memory()
         xd = torch.empty_like(xs[0])
+        g_e2e = None if args.no_graph else layer.capture(xd)
+
+        def e2e_step(i):
+            xd.copy_(xh[i % n_batches], non_blocking=True)
+            if g_e2e is not None:
+                g_e2e.replay()
+            else:
+                layer.forward(xd)
+            yh.copy_(layer.y[:T], non_blocking=True)
+
         for i in range(max(2, args.warmup)):
-            layer.forward_host(xh[i % n_batches], yh, xd)
+            e2e_step(i)
         dist.barrier()
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for i in range(args.steps):
-            layer.forward_host(xh[i % n_batches], yh, xd)
+            e2e_step(i)
         b.record(stream)
         torch.cuda.synchronize()
         dist.barrier()
         e2e_ms = dist.max(a.elapsed_time(b) / args.steps)
         e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
                "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
-               "d2h_bytes_per_step": int(yh.numel() * yh.element_size())}
+               "d2h_bytes_per_step": int(yh.numel() * yh.element_size()),
+               "path": "pinned host x -> H2D copy -> layer (CUDA graph of the C-ABI calls) -> D2H copy of y"}
 
-    launches_per_step = 2 + 4 + 3 + 2 + (2 if kind == "refill" else 1)  # route, permute, experts, shared, combine/refill+reduce
-    if kind == "refill":
-        launches_per_step += 1  # selection
+    # kernels per step: route (logits + top-k), permute (4), experts, shared (2), combine / refill (+ reduce, select)
+    launches_per_step = 2 + 4 + (5 if wl.fmt == "nvfp4" else 3) + 2 + (3 if kind == "refill" else 1)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) tokens, N(0,1/sqrt(fan_in)) weights)",
+        "vs_baseline": None, "dtype": {"bf16": "bf16", "awq_g32": "f16 x int4 (AWQ g32)",
+                                       "nvfp4": "fp4 e2m1 x fp4 e2m1 (NVFP4)"}[wl.fmt],
+        "data": "synthetic (seeded N(0,1) tokens, N(0,1/sqrt(fan_in)) weights)",
         "config": {"workload": f"{args.workload}: T={T} H={wl.H} E={wl.E} k={wl.k} I={wl.I} shared={wl.I_sh} "
                                f"fmt={wl.fmt}" + (" +Refill-RMS accumulate/select" if kind == "refill" else ""),
                    "tokens_per_step_per_gpu": T, "parallelism": f"dp{dist.world} (replicas, no collective)",
+                   "launch": "eager C-ABI calls" if args.no_graph else "one CUDA graph per step (the C-ABI calls)",
                    "l2": f"{n_batches} rotating token batches ({n_batches * x_bytes / 2**20:.0f} MiB) and "
                          f"{wl.E} experts of weights ({sum(t.numel() * t.element_size() for t in w.values()) / 2**30:.1f} GiB), "
                          "both larger than the 126 MB L2"},

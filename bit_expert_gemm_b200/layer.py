@@ -11,6 +11,11 @@ forward_host(xh, yh)     pinned host x -> y in pinned host memory (copies in
                          the stream, for end-to-end measurements)
 refill_pass(x, stats)    one Refill-RMS scoring pass (k+1 slots), adds to the
                          statistics and returns y
+capture(x, fn)           records one pass (forward, or any callable over the
+                         layer's buffers) into a CUDA graph bound to the
+                         device buffer x; replaying the graph re-runs the
+                         pass on whatever x then holds, without host work
+                         between the kernels
 """
 
 from __future__ import annotations
@@ -138,6 +143,24 @@ class MoELayer:
         y = self.y[:T]
         abi.moe_combine(f, self.slot_row[:T], self.topk_w[:T], shared_out=sh, y=y)
         return y
+
+    def capture(self, x: torch.Tensor, fn=None, warmup: int = 1) -> "torch.cuda.CUDAGraph":
+        """CUDA graph of fn(x) (default: forward).  Every launch of the pass
+        has fixed pointers (the layer's buffers, x) and host-side arguments,
+        so the graph replays it exactly; the pass is run `warmup` times first
+        so that one-time host set-up (function attributes, cached offsets)
+        happens outside the capture."""
+        fn = fn or self.forward
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for _ in range(warmup):
+                fn(x)
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(x)
+        return g
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, x_dev: torch.Tensor) -> None:
         """Pinned host x -> device -> forward -> pinned host y, all enqueued on
