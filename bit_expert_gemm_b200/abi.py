@@ -46,6 +46,7 @@ _SIGS = {
     "moe_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "moe_route_topk": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_grouped_swiglu_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _SZ, _P]),
     "moe_grouped_swiglu_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "moe_awq_dequant_g32": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
@@ -164,6 +165,23 @@ def moe_permute(topk_idx, E: int, expert_offsets=None, row_token=None, slot_row=
     if ws is None:
         ws = workspace(MOE_OP_PERMUTE, T, 0, E, ks, 0, dev)
     _call("moe_permute", _p(topk_idx), T, ks, E, _p(expert_offsets), _p(row_token), _p(slot_row), _p(ws), ws.numel(),
+          _stream(stream))
+    return expert_offsets, row_token, slot_row
+
+
+def moe_permute_noalloc(topk_idx, E: int, expert_offsets=None, row_token=None, slot_row=None, stream=None):
+    """moe_permute with the library's fixed scratch array instead of a
+    workspace, for callers that cannot allocate device memory."""
+    _need(topk_idx, torch.int32, "topk_idx")
+    T, ks = topk_idx.shape
+    dev = topk_idx.device
+    if expert_offsets is None:
+        expert_offsets = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    if row_token is None:
+        row_token = torch.empty((T * ks,), dtype=torch.int32, device=dev)
+    if slot_row is None:
+        slot_row = torch.empty((T, ks), dtype=torch.int32, device=dev)
+    _call("moe_permute_noalloc", _p(topk_idx), T, ks, E, _p(expert_offsets), _p(row_token), _p(slot_row),
           _stream(stream))
     return expert_offsets, row_token, slot_row
 

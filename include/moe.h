@@ -140,6 +140,27 @@ MOE_API int moe_permute(const int32_t* topk_idx, int T, int k_slots, int E, int3
                 int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_permute without a workspace argument.  The pages have no counterpart:
+ * this exists for callers that only receive input and output buffers from
+ * the framework hosting them (a plug-in interface without an allocator, a
+ * runtime with its own fixed memory pool, a latency-critical step where a
+ * cudaMalloc could synchronise the device) and so cannot pass scratch memory.
+ * Same arguments, outputs and order as moe_permute.  Its scratch is a fixed
+ * array of about 4 MiB inside the library's device image, held on every GPU
+ * that loads the library until the process exits; the call allocates and
+ * frees nothing.  Limit: E * ceil(T/32) <= 524288 (e.g. E = 512 experts,
+ * T = 32768 tokens); larger batches are rejected with MOE_ERR_UNSUPPORTED
+ * (use moe_permute with a workspace).  The first call on a device looks up
+ * the array's device address with that device current; make that first call
+ * before any stream capture.  All calls on a device share the array and it
+ * keeps the last call's contents (the part that must start at zero is
+ * cleared on the call's stream); calls whose work overlaps on the GPU, e.g.
+ * on unordered streams, race on it.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_permute_noalloc(const int32_t* topk_idx, int T, int k_slots, int E, int32_t* expert_offsets,
+                                int32_t* row_token, int32_t* slot_row, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Grouped SwiGLU expert FFN with 16-bit weights [ARCH]:
  *   for every expert e and every permuted row r of e (expert_offsets):
  *     g = x[row_token[r]] . Wg_e^T,  u = x[row_token[r]] . Wu_e^T   (FP32 acc)
