@@ -120,17 +120,15 @@ static int swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* o
                        int E, const void* w_gu, const void* w_d, int dtype, int out_fp32, void* f, void* ws,
                        size_t ws_bytes, cudaStream_t stream) {
   WsCarver carve(ws, ws_bytes);
-  void* xp = row_token ? carve.take<uint16_t>(size_t(rows) * H) : nullptr;
   uint16_t* h = carve.take<uint16_t>(size_t(rows) * I);
   MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_grouped_swiglu_bf16: workspace of %zu bytes is too small", ws_bytes);
   if (rows == 0) return MOE_OK;
+  // GEMM1 gathers its A rows (x[row_token[r]]) itself: no permuted copy of x
   const void* a = x;
-  if (row_token) {
-    int rc = gather_rows(x, row_token, rows, H, xp, stream);
-    if (rc) return rc;
-    a = xp;
-  }
   GemmArgs g1{};
+  g1.row_token = row_token;
+  g1.a_src = x;
+  g1.a_src_rows = T;
   g1.group_offsets = offsets;
   g1.G = E;
   g1.rows = rows;
@@ -148,6 +146,9 @@ static int swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* o
   int rc = launch_grouped_gemm(a, rows, w_gu, E * 2 * I, g1, EPI_SWIGLU, pick_bn(rows, E, I, true), stream);
   if (rc) return rc;
   GemmArgs g2 = g1;
+  g2.row_token = nullptr;
+  g2.a_src = nullptr;
+  g2.a_src_rows = 0;
   g2.K = I;
   g2.n_out = H;
   g2.b_rows_per_group = H;
@@ -187,7 +188,6 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k_slots, int I) {
     case MOE_OP_PERMUTE: return permute_ws_bytes(T, E);
     case MOE_OP_SWIGLU_BF16: {
       WsCounter c;
-      c.take<uint16_t>(size_t(rows) * H);
       c.take<uint16_t>(size_t(rows) * I);
       return c.used;
     }

@@ -12,11 +12,13 @@ constexpr int BK = 64;
 constexpr int A_TILE_BYTES = BM * BK * 2;
 constexpr int kBaseThreads = 192;    // producer, UMMA issuer, 4 epilogue warps
 constexpr int kDequantThreads = 256;  // 8 AWQ dequantisation warps
+constexpr int kGatherThreads = 128;   // 4 row-gather warps (A rows loaded through row_token)
+constexpr int kStoreStride = 128 + 16;  // epilogue staging: bytes per row of a 32-column chunk, padded
 constexpr int kSmemBudget = 196 * 1024;
 
 enum { W_DENSE = 0, W_AWQ = 1 };
 
-template <int BN, int EPI, int WQ>
+template <int BN, int EPI, int WQ, int AG>
 struct GemmCfg {
   static constexpr int B_TILE_BYTES = BN * BK * 2;
   // AWQ staging per stage, one TMA box per output half (gate / up for SwiGLU):
@@ -32,12 +34,16 @@ struct GemmCfg {
   static constexpr int ZERO_OFF = SCALE_OFF + NBOX * SCALE_BOX;
   static constexpr int RAW_BYTES = ZERO_OFF + NBOX * ZERO_BOX;
   static constexpr int STAGE_BYTES = (RAW_BYTES + 1023) / 1024 * 1024;  // keep every tile 1024-byte aligned
+  // bytes the TMA brings per stage (a gathered A tile arrives through cp.async instead)
   static constexpr int TX_BYTES =
-      A_TILE_BYTES + (WQ ? NBOX * (BK * W2 * 4 + 2 * W2 * 8 * 2 + 2 * W2 * 4) : B_TILE_BYTES);
+      (AG ? 0 : A_TILE_BYTES) + (WQ ? NBOX * (BK * W2 * 4 + 2 * W2 * 8 * 2 + 2 * W2 * 4) : B_TILE_BYTES);
   static constexpr int STAGES = kSmemBudget / STAGE_BYTES > 8 ? 8 : kSmemBudget / STAGE_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // +1024: alignment slack
+  static constexpr int STORE_BYTES = 4 * 32 * kStoreStride;   // epilogue staging, 32 rows per epilogue warp
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + STORE_BYTES;  // +1024: alignment slack
   static constexpr uint32_t TMEM_COLS = 2 * BN;                    // two accumulators
-  static constexpr int THREADS = kBaseThreads + (WQ ? kDequantThreads : 0);
+  static constexpr int GATHER_WARP0 = (kBaseThreads + (WQ ? kDequantThreads : 0)) / 32;
+  static constexpr int THREADS = kBaseThreads + (WQ ? kDequantThreads : 0) + (AG ? kGatherThreads : 0);
+  static constexpr uint32_t FULL_ARRIVALS = 1 + (AG ? kGatherThreads : 0);
   // MN-major B tile (AWQ): 64-element atoms along N are LBO apart, 8-row K groups SBO apart
   static constexpr uint32_t B_SBO = 1024;
   static constexpr uint32_t B_LBO = (BK / 8) * 1024;
@@ -103,16 +109,45 @@ __device__ __forceinline__ TileMap decode_tile(int L, int nt, const int* tile_st
   return t;
 }
 
+// Epilogue store of a 32-row x RB-byte chunk held one row per lane: the rows
+// go through the warp's staging area so that every store instruction writes
+// whole contiguous row segments (RB/16 lanes per row) instead of 16 bytes of
+// 32 different rows.  Rows r >= nvalid are not written.
+template <int RB>
+__device__ __forceinline__ void warp_store_rows(uint8_t* stg, const uint32_t* vals, int nvalid, uint8_t* gbase,
+                                                size_t pitch, int lane) {
+  uint4* mine = reinterpret_cast<uint4*>(stg + lane * kStoreStride);
+#pragma unroll
+  for (int i = 0; i < RB / 16; ++i) mine[i] = make_uint4(vals[4 * i], vals[4 * i + 1], vals[4 * i + 2], vals[4 * i + 3]);
+  __syncwarp();
+  constexpr int LPR = RB / 16, RPP = 32 / LPR;
+  const int seg = lane % LPR;
+#pragma unroll
+  for (int p = 0; p < LPR; ++p) {
+    const int r = p * RPP + lane / LPR;
+    const uint4 v = *reinterpret_cast<const uint4*>(stg + r * kStoreStride + seg * 16);
+    if (r < nvalid) st_global_v4(gbase + size_t(r) * pitch + seg * 16, v.x, v.y, v.z, v.w);
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Tensor maps of the B source.  Dense: b = the weight matrix.  AWQ: codes,
 // scales, zeros (b unused).
 struct BMaps {
   CUtensorMap b, codes, scales, zeros;
 };
 
-template <int BN, int EPI, int WQ>
-__global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ>::THREADS, 1)
+template <int BN, int EPI, int WQ, int AG>
+__global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ, AG>::THREADS, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps bm, const GemmArgs args) {
-  using Cfg = GemmCfg<BN, EPI, WQ>;
+  using Cfg = GemmCfg<BN, EPI, WQ, AG>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int BNH = (EPI == EPI_SWIGLU) ? BN / 2 : BN;  // output columns per tile
   constexpr int WC = BN / 8;                               // AWQ code words per K row of the tile
@@ -143,7 +178,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ>::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], Cfg::FULL_ARRIVALS);
       mbar_init(&empty_bar[s], 1);
       mbar_init(&bready_bar[s], kDequantThreads / 32);
     }
@@ -197,7 +232,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ>::THREADS, 1)
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
-          tma_load_2d(smA(stage), &tmA, &full_bar[stage], kb * BK, a_row);
+          if (!AG) tma_load_2d(smA(stage), &tmA, &full_bar[stage], kb * BK, a_row);
           if (WQ) {
             const int crow = t.g * args.K + kb * BK;          // code rows (input dim)
             const int grow = t.g * (args.K / 32) + kb * (BK / 32);  // scale / zero rows (groups)
@@ -272,15 +307,20 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ>::THREADS, 1)
   } else if (warp < 6) {
     // ---------------- epilogue: warps 2..5 ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const int row_in_tile = q * 32 + lane;
+    uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES + (warp - 2) * 32 * kStoreStride;
+    const size_t esize = args.out_fp32 ? 4 : 2;
+    const size_t pitch = size_t(args.ldo) * esize;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
       TileMap t = decode_tile(L, nt, tile_start, G);
       const int n_g = goff[t.g + 1] - goff[t.g];
-      const size_t out_row = size_t(goff[t.g]) + size_t(t.m) * BM + row_in_tile;
+      const size_t row0 = size_t(goff[t.g]) + size_t(t.m) * BM + q * 32;  // this warp's first output row
       // rows past the group, or (with inconsistent offsets) past the output, are not written
-      const bool valid = t.m * BM + row_in_tile < n_g && out_row < size_t(args.rows);
+      int nvalid = n_g - (t.m * BM + q * 32);
+      nvalid = nvalid < 0 ? 0 : (nvalid > 32 ? 32 : nvalid);
+      if (row0 + nvalid > size_t(args.rows)) nvalid = row0 < size_t(args.rows) ? int(size_t(args.rows) - row0) : 0;
+      uint8_t* gtile = reinterpret_cast<uint8_t*>(args.out) + row0 * pitch;
       if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag, status, lim)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
@@ -289,46 +329,35 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ>::THREADS, 1)
         for (int c = 0; c < BNH / 32; ++c) {
           float gv[32], uv[32];
           tmem_ld32x2(tb + c * 32, tb + BNH + c * 32, gv, uv);
-          if (valid) {
-            uint32_t pk[16];
+          uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float h0 = silu_f(gv[2 * i]) * uv[2 * i];
-              float h1 = silu_f(gv[2 * i + 1]) * uv[2 * i + 1];
-              pk[i] = args.bf16 ? Pack2<__nv_bfloat16>::pack(h0, h1) : Pack2<__half>::pack(h0, h1);
-            }
-            uint16_t* dst = reinterpret_cast<uint16_t*>(args.out) + out_row * size_t(args.ldo) + t.n * BNH + c * 32;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) st_global_v4(dst + 8 * v, pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int i = 0; i < 16; ++i) {
+            float h0 = silu_f(gv[2 * i]) * uv[2 * i];
+            float h1 = silu_f(gv[2 * i + 1]) * uv[2 * i + 1];
+            pk[i] = args.bf16 ? Pack2<__nv_bfloat16>::pack(h0, h1) : Pack2<__half>::pack(h0, h1);
           }
+          warp_store_rows<64>(stg, pk, nvalid, gtile + size_t(t.n * BNH + c * 32) * 2, pitch, lane);
         }
       } else {
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
           tmem_ld32(tb + c * 32, v);
-          if (valid) {
-            const int col0 = t.n * BN + c * 32;
-            if (args.bias) {
+          const int col0 = t.n * BN + c * 32;
+          if (args.bias) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] += __ldg(args.bias + col0 + i);
-            }
-            if (args.out_fp32) {
-              float* dst = reinterpret_cast<float*>(args.out) + out_row * size_t(args.ldo) + col0;
+            for (int i = 0; i < 32; ++i) v[i] += __ldg(args.bias + col0 + i);
+          }
+          if (args.out_fp32) {
+            warp_store_rows<128>(stg, reinterpret_cast<const uint32_t*>(v), nvalid, gtile + size_t(col0) * 4, pitch,
+                                 lane);
+          } else {
+            uint32_t pk[16];
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                st_global_v4(dst + 4 * i, __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
-                             __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
-            } else {
-              uint32_t pk[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                pk[i] = args.bf16 ? Pack2<__nv_bfloat16>::pack(v[2 * i], v[2 * i + 1])
-                                  : Pack2<__half>::pack(v[2 * i], v[2 * i + 1]);
-              uint16_t* dst = reinterpret_cast<uint16_t*>(args.out) + out_row * size_t(args.ldo) + col0;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) st_global_v4(dst + 8 * i, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-            }
+            for (int i = 0; i < 16; ++i)
+              pk[i] = args.bf16 ? Pack2<__nv_bfloat16>::pack(v[2 * i], v[2 * i + 1])
+                                : Pack2<__half>::pack(v[2 * i], v[2 * i + 1]);
+            warp_store_rows<64>(stg, pk, nvalid, gtile + size_t(col0) * 2, pitch, lane);
           }
         }
       }
@@ -337,7 +366,48 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ>::THREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
-  } else if (WQ) {
+  } else if (AG && warp >= Cfg::GATHER_WARP0) {
+    // ---------------- A row gather: 4 warps ----------------
+    // Thread gt copies 16-byte chunk (gt % 8) of tile rows gt/8, gt/8 + 16, ...
+    // of A = a_src[row_token[row]] into the 128-byte-swizzled K-major layout
+    // (chunk index XOR row mod 8) that the TMA would write; rows past the
+    // problem are zero-filled.  Each thread then arrives on the stage's full
+    // barrier once its copies have landed.
+    const int gt = threadIdx.x - Cfg::GATHER_WARP0 * 32;
+    const int chunk = gt & 7;
+    const int rbase = gt >> 3;
+    const uint8_t* src = static_cast<const uint8_t*>(args.a_src);
+    const size_t src_pitch = size_t(args.K) * 2;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      TileMap t = decode_tile(L, nt, tile_start, G);
+      const int a_row = goff[t.g] + t.m * BM;
+      int tok[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = a_row + rbase + 16 * i;
+        int tk = r < args.rows ? __ldg(args.row_token + r) : -1;
+        tok[i] = (tk >= 0 && tk < args.a_src_rows) ? tk : -1;
+      }
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
+        const uint32_t dst0 = smem_u32(smA(stage));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = rbase + 16 * i;
+          const uint32_t dst = dst0 + uint32_t(r * 128 + ((chunk ^ (r & 7)) << 4));
+          const uint8_t* g = src + (tok[i] >= 0 ? size_t(tok[i]) * src_pitch + size_t(kb) * 128 + chunk * 16 : 0);
+          cp_async_16_zfill(dst, g, tok[i] >= 0 ? 16u : 0u);
+        }
+        cp_async_arrive_noinc(&full_bar[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // every copy has landed before the CTA exits
+  } else if (WQ && warp < Cfg::GATHER_WARP0) {
     // ---------------- AWQ dequantisation: warps 6..13 ----------------
     // Thread (wc, r0) turns code word column wc (output columns 8wc..8wc+7)
     // of K rows r0, r0 + RP, ... into one 16-byte chunk of the MN-major B tile
@@ -440,11 +510,11 @@ int make_tmap_2d_u8_sw128(CUtensorMap* map, const void* base, int rows, int cols
   return make_tmap_2d(map, base, rows, cols_bytes, 1, box_rows, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int BN, int EPI, int WQ>
+template <int BN, int EPI, int WQ, int AG>
 static int launch_bn(const CUtensorMap& ta, const BMaps& bmaps, const GemmArgs& args, cudaStream_t stream) {
-  using Cfg = GemmCfg<BN, EPI, WQ>;
+  using Cfg = GemmCfg<BN, EPI, WQ, AG>;
   static bool attr_set[64] = {false};  // per device
-  auto kern = k_grouped_gemm<BN, EPI, WQ>;
+  auto kern = k_grouped_gemm<BN, EPI, WQ, AG>;
   int dev = 0;
   MOE_CHECK_CUDA(cudaGetDevice(&dev));
   if (dev >= 64 || !attr_set[dev]) {
@@ -456,17 +526,17 @@ static int launch_bn(const CUtensorMap& ta, const BMaps& bmaps, const GemmArgs& 
   return MOE_OK;
 }
 
-template <int WQ>
+template <int WQ, int AG>
 static int dispatch(const CUtensorMap& ta, const BMaps& bm, const GemmArgs& args, int epi, int bn,
                     cudaStream_t stream) {
   if (epi == EPI_SWIGLU) {
-    if (bn == 256) return launch_bn<256, EPI_SWIGLU, WQ>(ta, bm, args, stream);
-    if (bn == 128) return launch_bn<128, EPI_SWIGLU, WQ>(ta, bm, args, stream);
-    return launch_bn<64, EPI_SWIGLU, WQ>(ta, bm, args, stream);
+    if (bn == 256) return launch_bn<256, EPI_SWIGLU, WQ, AG>(ta, bm, args, stream);
+    if (bn == 128) return launch_bn<128, EPI_SWIGLU, WQ, AG>(ta, bm, args, stream);
+    return launch_bn<64, EPI_SWIGLU, WQ, AG>(ta, bm, args, stream);
   }
-  if (bn == 256) return launch_bn<256, EPI_STORE, WQ>(ta, bm, args, stream);
-  if (bn == 128) return launch_bn<128, EPI_STORE, WQ>(ta, bm, args, stream);
-  return launch_bn<64, EPI_STORE, WQ>(ta, bm, args, stream);
+  if (bn == 256) return launch_bn<256, EPI_STORE, WQ, AG>(ta, bm, args, stream);
+  if (bn == 128) return launch_bn<128, EPI_STORE, WQ, AG>(ta, bm, args, stream);
+  return launch_bn<64, EPI_STORE, WQ, AG>(ta, bm, args, stream);
 }
 
 static int check_common(const GemmArgs& args, int epi, int bn) {
@@ -490,11 +560,20 @@ int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_tot
   CUtensorMap ta;
   BMaps bm;
   memset(&bm, 0, sizeof(bm));
-  rc = make_tmap_16bit_sw128(&ta, A, a_rows, args.K, BM);
+  if (args.row_token) {
+    // A rows are gathered in the kernel; the map over the source only keeps the parameter valid
+    MOE_REQUIRE(args.a_src != nullptr && args.a_src_rows > 0, MOE_ERR_INVALID_ARG, "gathered GEMM without a source");
+    MOE_REQUIRE((reinterpret_cast<uintptr_t>(args.a_src) & 15) == 0, MOE_ERR_INVALID_ARG,
+                "gathered rows are not 16-byte aligned");
+    rc = make_tmap_16bit_sw128(&ta, args.a_src, args.a_src_rows, args.K, BM);
+  } else {
+    rc = make_tmap_16bit_sw128(&ta, A, a_rows, args.K, BM);
+  }
   if (rc) return rc;
   rc = make_tmap_16bit_sw128(&bm.b, B, b_rows_total, args.K, bnh);
   if (rc) return rc;
-  return dispatch<W_DENSE>(ta, bm, args, epi, bn, stream);
+  if (args.row_token) return dispatch<W_DENSE, 1>(ta, bm, args, epi, bn, stream);
+  return dispatch<W_DENSE, 0>(ta, bm, args, epi, bn, stream);
 }
 
 int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, const int32_t* qzeros,
@@ -519,7 +598,8 @@ int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, c
   if (rc) return rc;
   rc = make_tmap_2d(&bm.zeros, qzeros, G * (args.K / 32), n_total / 8, 4, 2, bnh / 8, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
-  return dispatch<W_AWQ>(ta, bm, args, epi, bn, stream);
+  MOE_REQUIRE(args.row_token == nullptr, MOE_ERR_UNSUPPORTED, "AWQ GEMM reads pre-gathered rows");
+  return dispatch<W_AWQ, 0>(ta, bm, args, epi, bn, stream);
 }
 
 }  // namespace moe

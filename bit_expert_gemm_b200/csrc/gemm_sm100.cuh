@@ -35,6 +35,11 @@ struct GemmArgs {
   int bf16;              // 1: BF16 operands, 0: FP16
   int* status;
   unsigned long long limit_ns;
+  // Row gather of A (optional): A row r of the grouped problem is row
+  // row_token[r] of a_src [a_src_rows, K]; nullptr: A is read as stored.
+  const int* row_token;
+  const void* a_src;
+  int a_src_rows;
 };
 
 // Host launcher (gemm_sm100.cu).  A [a_rows, K] and B [b_rows_total, K] are
