@@ -240,7 +240,8 @@ def expert_flops(rows: int, H: int, I: int) -> float:
 
 EXPERT_KEYS = {"bf16": ("w_gate_up", "w_down"), "awq_g32": ("qw_gu", "qz_gu", "sc_gu", "qw_d", "qz_d", "sc_d"),
                "nvfp4": ("w_gu", "sf_gu", "gs_gu", "w_d", "sf_d", "gs_d")}
-KERNEL_NAMES = {"bf16": "moe_grouped_swiglu_bf16 (row gather + GEMM1/SwiGLU + GEMM2, tcgen05 kind::f16)",
+KERNEL_NAMES = {"bf16": "moe_experts_bf16 (routed + shared experts: GEMM1/SwiGLU + GEMM2, tcgen05 kind::f16; "
+                        "decode-sized batches stream the weights as the M operand)",
                 "awq_g32": "moe_grouped_swiglu_awq_g32 (row gather + dequantising GEMM1/SwiGLU + GEMM2, tcgen05 "
                            "kind::f16)",
                 "nvfp4": "moe_grouped_swiglu_nvfp4 (activation quantisation + GEMM1/SwiGLU + h quantisation + GEMM2, "
@@ -258,6 +259,11 @@ def expert_roofline(wl, layer, T, rows, ffn_ms, peaks) -> dict:
     touched = int((counts > 0).sum())
     expert_bytes = touched * per_expert
     flops = expert_flops(rows, wl.H, wl.I)
+    with_shared = layer.ws_exp is not None  # the timed call also runs the shared expert
+    if with_shared:
+        sh_bytes = sum(w[k].numel() * w[k].element_size() for k in ("w_sh_gate_up", "w_sh_down"))
+        expert_bytes += sh_bytes
+        flops += expert_flops(T, wl.H, wl.I_sh)
     if T >= 256:
         if wl.fmt == "nvfp4":
             base = peaks.get("bf16_tflops_sustained")
@@ -271,13 +277,15 @@ def expert_roofline(wl, layer, T, rows, ffn_ms, peaks) -> dict:
         achieved = flops / (ffn_ms / 1e3) / 1e12
         return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": None, "kernel": KERNEL_NAMES[wl.fmt],
-                "work_per_launch": f"{flops / 1e9:.1f} GFLOP = 2*rows*3*H*I, rows={rows}", "peak_source": src,
+                "work_per_launch": f"{flops / 1e9:.1f} GFLOP = 2*rows*3*H*I, rows={rows}"
+                                   + (f" + shared expert on {T} tokens" if with_shared else ""), "peak_source": src,
                 "experts_touched": touched}
     peak = peaks.get("hbm_gbs", 6650.0)
     achieved = expert_bytes / (ffn_ms / 1e3) / 1e9
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": None, "kernel": KERNEL_NAMES[wl.fmt],
-            "work_per_launch": f"{expert_bytes / 1e6:.2f} MB = {touched} experts x {per_expert / 1e6:.3f} MB",
+            "work_per_launch": f"{expert_bytes / 1e6:.2f} MB = {touched} experts x {per_expert / 1e6:.3f} MB"
+                               + (" + the shared expert" if with_shared else ""),
             "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)", "experts_touched": touched}
 
 
@@ -303,10 +311,9 @@ def run_native(args, dist: Dist) -> None:
         layer.route(x)
         if ev:
             ev[0].record()
-        f = layer.experts(x)
+        f, sh = layer.experts_and_shared(x)
         if ev:
             ev[1].record()
-        sh = layer.shared_expert(x)
         if kind == "refill":
             abi.razor_refill_rms_accumulate(f, layer.slot_row[:T], layer.topk_idx[:T], layer.topk_logit[:T],
                                             layer.offsets, sum_sq, count, shared_out=sh, y_out=layer.y[:T],
@@ -339,14 +346,28 @@ def run_native(args, dist: Dist) -> None:
     clocks = ClockSampler(dist.local)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    # Decode-sized steps touch fewer weight bytes than L2 holds (the popular
+    # experts would stay cached from step to step): flush L2 before every
+    # timed step and time each step with its own events, flush excluded.
+    # Prefill steps stream GBs, larger than L2: one bracket over all steps.
+    flush_l2 = T < 256
+    l2_flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush_l2 else None
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start.record(stream)
     for i in range(args.steps):
+        if flush_l2:
+            l2_flush.zero_()
+        step_ev[i][0].record(stream)
         run(i)
+        step_ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
     clk = clocks.stop()
-    ms_local = t_start.elapsed_time(t_end) / args.steps
+    if flush_l2:
+        ms_local = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
+    else:
+        ms_local = t_start.elapsed_time(t_end) / args.steps
     ms = dist.max(ms_local)
     # the expert call of the last replay of every batch's graph (inside the timed region)
     used = sorted({i % n_batches for i in range(max(0, args.steps - n_batches), args.steps)})
@@ -383,13 +404,22 @@ def run_native(args, dist: Dist) -> None:
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
         a.record(stream)
         for i in range(args.steps):
+            if flush_l2:
+                l2_flush.zero_()
+            e2e_ev[i][0].record(stream)
             e2e_step(i)
+            e2e_ev[i][1].record(stream)
         b.record(stream)
         torch.cuda.synchronize()
         dist.barrier()
-        e2e_ms = dist.max(a.elapsed_time(b) / args.steps)
+        if flush_l2:
+            e2e_ms = dist.max(sum(p.elapsed_time(q) for p, q in e2e_ev) / args.steps)
+        else:
+            e2e_ms = dist.max(a.elapsed_time(b) / args.steps)
         e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
                "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
                "d2h_bytes_per_step": int(yh.numel() * yh.element_size()),
@@ -407,9 +437,11 @@ def run_native(args, dist: Dist) -> None:
                                f"fmt={wl.fmt}" + (" +Refill-RMS accumulate/select" if kind == "refill" else ""),
                    "tokens_per_step_per_gpu": T, "parallelism": f"dp{dist.world} (replicas, no collective)",
                    "launch": "eager C-ABI calls" if args.no_graph else "one CUDA graph per step (the C-ABI calls)",
-                   "l2": f"{n_batches} rotating token batches ({n_batches * x_bytes / 2**20:.0f} MiB) and "
-                         f"{wl.E} experts of weights ({sum(t.numel() * t.element_size() for t in w.values()) / 2**30:.1f} GiB), "
-                         "both larger than the 126 MB L2"},
+                   "l2": (f"L2 flushed (a {2 * L2_BYTES >> 20} MiB write) before every timed step; each step timed "
+                          "with its own CUDA events, the flush excluded" if T < 256 else
+                          f"{n_batches} rotating token batches ({n_batches * x_bytes / 2**20:.0f} MiB) and "
+                          f"{sum(t.numel() * t.element_size() for t in w.values()) / 2**30:.1f} GiB of expert "
+                          "weights per step's reach, both larger than the 126 MB L2")},
         "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
         "expert_ffn_ms": round(ffn_ms, 4),
     }

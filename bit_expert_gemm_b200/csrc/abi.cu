@@ -35,6 +35,10 @@ int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* o
 int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N, void* out,
                 cudaStream_t stream);
 size_t nvfp4_quant_ws_bytes(int batch, int rows, int K);
+size_t decode_ws_bytes(int rows, int T, int I);
+int decode_experts_16bit(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
+                         int E, const void* w_gu, const void* w_d, const void* w_sh_gu, const void* w_sh_d, int dtype,
+                         int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, cudaStream_t stream);
 int nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const float* gs_in, uint8_t* codes,
                    uint8_t* sf, float* gs_out, void* ws, size_t ws_bytes, cudaStream_t stream);
 size_t nvfp4_ws_bytes(int rows, int H, int I, int E);
@@ -159,6 +163,45 @@ static int swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* o
   return launch_grouped_gemm(h, rows, w_d, E * H, g2, EPI_STORE, pick_bn(rows, E, H, false), stream);
 }
 
+// Dense SwiGLU expert on all T rows of x (the shared expert): GEMM1 + SwiGLU
+// into h_ws [T, I], GEMM2 into out [T, H].
+static int dense_swiglu(const void* x, int T, int H, int I, const void* w_gu, const void* w_d, int dtype, void* out,
+                        uint16_t* h_ws, cudaStream_t stream) {
+  GemmArgs g1{};
+  g1.group_offsets = nullptr;
+  g1.G = 1;
+  g1.rows = T;
+  g1.K = H;
+  g1.n_out = I;
+  g1.b_rows_per_group = 2 * I;
+  g1.up_offset = I;
+  g1.out = h_ws;
+  g1.ldo = I;
+  g1.bf16 = dtype == MOE_DTYPE_BF16;
+  g1.status = device_status_ptr();
+  g1.limit_ns = wait_limit_ns();
+  int rc = launch_grouped_gemm(x, T, w_gu, 2 * I, g1, EPI_SWIGLU, pick_bn(T, 1, I, true), stream);
+  if (rc) return rc;
+  GemmArgs g2 = g1;
+  g2.K = I;
+  g2.n_out = H;
+  g2.b_rows_per_group = H;
+  g2.up_offset = 0;
+  g2.out = out;
+  g2.ldo = H;
+  return launch_grouped_gemm(h_ws, T, w_d, H, g2, EPI_STORE, pick_bn(T, 1, H, false), stream);
+}
+
+static constexpr int kDecodeMaxT = 128;
+
+static size_t experts_ws_bytes(int T, int rows, int H, int I) {
+  (void)H;
+  if (T <= kDecodeMaxT) return decode_ws_bytes(rows, T, I);
+  WsCounter c;
+  c.take<uint16_t>(size_t(rows > T ? rows : T) * I);
+  return c.used;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -192,6 +235,7 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k_slots, int I) {
       return c.used;
     }
     case MOE_OP_SWIGLU_AWQ_G32: return awq_ws_bytes(rows, H, I, E);
+    case MOE_OP_EXPERTS_BF16: return experts_ws_bytes(T, rows, H, I);
     case MOE_OP_SWIGLU_NVFP4: return nvfp4_ws_bytes(rows, H, I, E);
     case MOE_OP_REFILL: return refill_ws_bytes(T, k_slots > 0 ? k_slots - 1 : 0);
     case MOE_OP_NVFP4_QUANTIZE: return nvfp4_quant_ws_bytes(1, T, H);
@@ -246,6 +290,37 @@ int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, const int32
               "moe_grouped_swiglu_bf16: operands must be 16-byte aligned");
   return swiglu_bf16(x, row_token, expert_offsets, T, rows, H, I, E, w_gate_up, w_down, dtype, out_fp32, f, ws,
                      ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int moe_experts_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows, int H,
+                     int I, int E, const void* w_gate_up, const void* w_down, const void* w_sh_gate_up,
+                     const void* w_sh_down, int dtype, int out_fp32, void* f, void* shared_out, void* ws,
+                     size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG, "moe_experts_bf16: bad sizes");
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_experts_bf16: dtype %d",
+              dtype);
+  MOE_REQUIRE(H > 0 && I > 0 && H % 128 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_experts_bf16: need H %% 128 == 0 and I %% 64 == 0 (H=%d I=%d)", H, I);
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(x && row_token && expert_offsets && w_gate_up && w_down && w_sh_gate_up && w_sh_down && f && shared_out,
+              MOE_ERR_INVALID_ARG, "moe_experts_bf16: null pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(w_gate_up) && aligned16(w_down) && aligned16(w_sh_gate_up) &&
+                  aligned16(w_sh_down) && aligned16(f) && aligned16(shared_out),
+              MOE_ERR_INVALID_ARG, "moe_experts_bf16: operands must be 16-byte aligned");
+  MOE_REQUIRE(ws_bytes >= experts_ws_bytes(T, rows, H, I), MOE_ERR_WORKSPACE,
+              "moe_experts_bf16: workspace of %zu bytes is too small (need %zu)", ws_bytes,
+              experts_ws_bytes(T, rows, H, I));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T <= kDecodeMaxT)
+    return decode_experts_16bit(x, row_token, expert_offsets, T, rows, H, I, E, w_gate_up, w_down, w_sh_gate_up,
+                                w_sh_down, dtype, out_fp32, f, shared_out, ws, ws_bytes, st);
+  int rc = MOE_OK;
+  if (rows > 0) {
+    rc = swiglu_bf16(x, row_token, expert_offsets, T, rows, H, I, E, w_gate_up, w_down, dtype, out_fp32, f, ws,
+                     ws_bytes, st);
+    if (rc) return rc;
+  }
+  return dense_swiglu(x, T, H, I, w_sh_gate_up, w_sh_down, dtype, shared_out, static_cast<uint16_t*>(ws), st);
 }
 
 int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,

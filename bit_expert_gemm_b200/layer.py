@@ -91,6 +91,14 @@ class MoELayer:
         self.ws_perm = abi.workspace(abi.MOE_OP_PERMUTE, T_max, H, E, ks, 0, d)
         self.ws_ffn = abi.workspace(op, T_max, H, E, ks, self.I, d)
         self.ws_sh = abi.workspace(abi.MOE_OP_SWIGLU_BF16, T_max, H, 1, 1, self.I_sh, d)
+        if self.fmt == "bf16" and self.I_sh == self.I:
+            # routed + shared experts in one call: big enough for the decode path
+            # (T <= 128) and the prefill path
+            need = max(abi.moe_workspace_size(abi.MOE_OP_EXPERTS_BF16, t, H, E, ks, self.I)
+                       for t in {T_max, min(T_max, 128)})
+            self.ws_exp = torch.empty(max(256, need), dtype=torch.uint8, device=d)
+        else:
+            self.ws_exp = None
         self.ws_refill = abi.workspace(abi.MOE_OP_REFILL, T_max, H, E, ks, 0, d)
         self._sh_off = {}
 
@@ -134,12 +142,26 @@ class MoELayer:
                                     self.w["w_sh_down"].unsqueeze(0), out_fp32=False, f=sh, ws=self.ws_sh)
         return sh
 
+    def experts_and_shared(self, x: torch.Tensor):
+        """Routed expert rows f and the shared expert's output; one C-ABI call
+        (moe_experts_bf16) for 16-bit weights."""
+        if self.ws_exp is None:
+            return self.experts(x), self.shared_expert(x)
+        T = x.shape[0]
+        rows = T * (self.k + self.extra)
+        f = self.f[:rows]
+        sh = self.shared[:T]
+        w = self.w
+        abi.moe_experts_bf16(x, self.row_token[:rows], self.offsets, rows, w["w_gate_up"], w["w_down"],
+                             w["w_sh_gate_up"], w["w_sh_down"], out_fp32=f.dtype == torch.float32, f=f,
+                             shared_out=sh, ws=self.ws_exp)
+        return f, sh
+
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         T = x.shape[0]
         assert T <= self.T_max and self.extra == 0
         self.route(x)
-        f = self.experts(x)
-        sh = self.shared_expert(x)
+        f, sh = self.experts_and_shared(x)
         y = self.y[:T]
         abi.moe_combine(f, self.slot_row[:T], self.topk_w[:T], shared_out=sh, y=y)
         return y
@@ -175,8 +197,7 @@ class MoELayer:
         T = x.shape[0]
         assert self.extra == 1
         self.route(x)
-        f = self.experts(x)
-        sh = self.shared_expert(x)
+        f, sh = self.experts_and_shared(x)
         y = self.y[:T]
         abi.razor_refill_rms_accumulate(f, self.slot_row[:T], self.topk_idx[:T], self.topk_logit[:T], self.offsets,
                                         sum_sq, count, shared_out=sh, y_out=y, ws=self.ws_refill)

@@ -81,7 +81,8 @@ enum {
   MOE_OP_SWIGLU_AWQ_G32 = 3,
   MOE_OP_SWIGLU_NVFP4 = 4,
   MOE_OP_REFILL = 5,
-  MOE_OP_NVFP4_QUANTIZE = 6
+  MOE_OP_NVFP4_QUANTIZE = 6,
+  MOE_OP_EXPERTS_BF16 = 7
 };
 
 /* Version of this header's ABI. */
@@ -178,6 +179,24 @@ MOE_API int moe_permute_noalloc(const int32_t* topk_idx, int T, int k_slots, int
 MOE_API int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
                             int rows, int H, int I, int E, const void* w_gate_up, const void* w_down, int dtype,
                             int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Routed experts and the shared expert of one layer in one call [ARCH]: the
+ * routed part is moe_grouped_swiglu_bf16 (f [rows, H]), the shared part the
+ * same SwiGLU on every token with w_sh_gate_up [2I, H] and w_sh_down [H, I]
+ * (shared_out [T, H] dtype; the shared expert has the routed experts' width
+ * I).  For T <= 128 (decode) both run as weight-streaming tensor-core GEMMs
+ * with the weights as the M operand and the few tokens as N, routed and
+ * shared work items in the same two launches: the first applies SwiGLU in its
+ * epilogue and writes h [rows + T, I] (dtype) to the workspace, the second
+ * reads it back.  Larger T uses the grouped prefill GEMMs.  row_token is
+ * required.
+ * Limits: H % 128 == 0, I % 64 == 0.  Workspace: MOE_OP_EXPERTS_BF16.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_experts_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows,
+                             int H, int I, int E, const void* w_gate_up, const void* w_down, const void* w_sh_gate_up,
+                             const void* w_sh_down, int dtype, int out_fp32, void* f, void* shared_out, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Grouped SwiGLU expert FFN with AWQ W4A16 asymmetric group-32 weights [AWQ].

@@ -23,7 +23,10 @@ def test_workspace_sizes():
     lib = abi.load()
     assert lib.moe_workspace_size(abi.MOE_OP_ROUTE_TOPK, 8192, 2048, 512, 10, 640) >= 8192 * 512 * 4
     big = lib.moe_workspace_size(abi.MOE_OP_SWIGLU_BF16, 8192, 2048, 512, 10, 640)
-    assert big >= 81920 * (2048 + 640) * 2
+    assert big >= 81920 * 640 * 2  # h between the GEMMs (GEMM1 gathers x rows itself)
+    # routed + shared experts: h [rows, I] for prefill, h [rows + T, I] (shared rows appended) for decode
+    assert lib.moe_workspace_size(abi.MOE_OP_EXPERTS_BF16, 8192, 2048, 512, 10, 640) >= 81920 * 640 * 2
+    assert lib.moe_workspace_size(abi.MOE_OP_EXPERTS_BF16, 64, 2048, 512, 10, 640) >= (640 + 64) * 640 * 2  # 16-bit h
     assert lib.moe_workspace_size(abi.MOE_OP_PERMUTE, 32768, 2048, 512, 11, 640) >= 512 * 1024 * 8
     assert lib.moe_workspace_size(99, 1, 1, 1, 1, 1) == 0
     assert lib.moe_workspace_size(abi.MOE_OP_ROUTE_TOPK, -1, 1, 1, 1, 1) == 0

@@ -153,3 +153,30 @@ def test_select_bit_exact(E):
             assert np.array_equal(score.cpu().numpy(), s_ref)
             assert np.array_equal(ranking.cpu().numpy(), r_ref)
             assert np.array_equal(kept.cpu().numpy(), k_ref)
+
+
+@pytest.mark.parametrize("T,H,I,E,k,out_fp32", [(1, 2048, 640, 512, 10, False), (8, 512, 128, 16, 4, False),
+                                                (64, 2048, 640, 64, 10, True), (128, 256, 64, 16, 2, False),
+                                                (300, 512, 128, 8, 3, False)])
+def test_experts_routed_and_shared(T, H, I, E, k, out_fp32):
+    """moe_experts_bf16: the decode path (T <= 128: weight-streaming GEMMs with
+    the shared expert as one more group) and the prefill path (T > 128)."""
+    wl = _wl(H=H, I=I, I_sh=I, E=E, k=k)
+    w = synth.make_weights(wl, seed=T + 7, device=DEV)
+    x = synth.make_tokens(wl, T, seed=T + 7, device=DEV)
+    idx = synth.make_routing(T, E, k, seed=T + 8)
+    off, rt, sr = abi.moe_permute(idx.to(DEV), E)
+    f, sh = abi.moe_experts_bf16(x, rt, off, T * k, w["w_gate_up"], w["w_down"], w["w_sh_gate_up"], w["w_sh_down"],
+                                 out_fp32=out_fp32)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0
+    perm = moe.permute(idx.numpy().astype(np.int64), E)
+    xs = f64(x)
+    gu, wd = w["w_gate_up"], w["w_down"]
+    ref, _ = moe.routed_outputs(xs, perm, lambda e: (f64(gu[e, :I]), f64(gu[e, I:]), f64(wd[e])))
+    err = rel_err(f64(f)[sr.cpu().numpy().ravel()], ref[perm["slot_row"].ravel()])
+    assert err < 1e-2, err
+    sg = f64(w["w_sh_gate_up"])
+    sref, _ = moe.swiglu_expert(xs, sg[:I], sg[I:], f64(w["w_sh_down"]))
+    err_sh = rel_err(f64(sh), sref)
+    assert err_sh < 1e-2, err_sh
