@@ -248,15 +248,22 @@ KERNEL_NAMES = {"bf16": "moe_experts_bf16 (routed + shared experts: GEMM1/SwiGLU
                          "tcgen05 kind::mxf4nvf4)"}
 
 
-def expert_roofline(wl, layer, T, rows, ffn_ms, peaks) -> dict:
+def _count_step_kernels(layer, x, step) -> int:
+    layer.capture(x, step, warmup=0)
+    return layer.graph_kernels
+
+
+def expert_roofline(wl, layers, T, rows, ffn_ms, peaks) -> dict:
     """Roofline of the routed expert call: tensor-bound (algorithmic FLOPs)
     for prefill-sized batches, HBM-bound (bytes of the distinct experts the
-    batch touches) for decode-sized ones."""
+    batch touches, averaged over the timed units' last routings) for
+    decode-sized ones."""
+    layer = layers[0]
     w = layer.w
     keys = EXPERT_KEYS[wl.fmt]
     per_expert = sum(w[k].numel() * w[k].element_size() for k in keys) / wl.E
-    counts = torch.diff(layer.offsets.to(torch.int64)).cpu()
-    touched = int((counts > 0).sum())
+    touched_each = [int((torch.diff(lay.offsets.to(torch.int64)).cpu() > 0).sum()) for lay in layers]
+    touched = statistics.mean(touched_each)
     expert_bytes = touched * per_expert
     flops = expert_flops(rows, wl.H, wl.I)
     with_shared = layer.ws_exp is not None  # the timed call also runs the shared expert
@@ -284,7 +291,7 @@ def expert_roofline(wl, layer, T, rows, ffn_ms, peaks) -> dict:
     achieved = expert_bytes / (ffn_ms / 1e3) / 1e9
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": None, "kernel": KERNEL_NAMES[wl.fmt],
-            "work_per_launch": f"{expert_bytes / 1e6:.2f} MB = {touched} experts x {per_expert / 1e6:.3f} MB"
+            "work_per_launch": f"{expert_bytes / 1e6:.2f} MB = {touched:.1f} experts x {per_expert / 1e6:.3f} MB"
                                + (" + the shared expert" if with_shared else ""),
             "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)", "experts_touched": touched}
 
@@ -294,49 +301,75 @@ def run_native(args, dist: Dist) -> None:
     wl = synth.WORKLOADS[wname]
     dev = torch.device("cuda", dist.local)
     torch.cuda.set_device(dev)
-    w = synth.make_weights(wl, seed=0, device=dev)
     extra = 1 if kind == "refill" else 0
-    layer = MoELayer(w, wl.k, wl.fmt, T_max=T, extra=extra)
+    decode = T < 256
+    layers = [MoELayer(synth.make_weights(wl, seed=0, device=dev), wl.k, wl.fmt, T_max=T, extra=extra)]
+    layer_bytes = sum(t.numel() * t.element_size() for t in layers[0].w.values())
+    if decode:
+        # A decode step touches fewer expert bytes than L2 holds.  Rotate
+        # through layers with distinct weights so that, between two uses of
+        # one layer, the others stream at least 3x L2 of expert weights (at
+        # least k routed experts + the shared expert per step): no expert
+        # weight is L2-resident when its layer runs again.
+        per_expert = sum(layers[0].w[k].numel() * layers[0].w[k].element_size() for k in EXPERT_KEYS[wl.fmt]) / wl.E
+        step_min = (wl.k + 1) * per_expert
+        n_layers = max(2, 1 + -(-3 * L2_BYTES // int(step_min)))
+        n_layers = min(n_layers, 24, max(2, int(64e9 // layer_bytes)))
+        for l in range(1, n_layers):
+            layers.append(MoELayer(synth.make_weights(wl, seed=l, device=dev), wl.k, wl.fmt, T_max=T, extra=extra))
+    layer = layers[0]
+    w = layer.w
     # token batches: distinct per rank, rotated so that the inputs of the
     # timed steps exceed the L2 cache
     x_bytes = T * wl.H * 2
     n_batches = max(2, min(8, -(-2 * L2_BYTES // x_bytes)))
     xs = [synth.make_tokens(wl, T, seed=1 + dist.rank, batch=b, device=dev) for b in range(n_batches)]
+    # units of the rotation: (layer, token batch); one CUDA graph each
+    units = ([(layers[l], xs[l % n_batches]) for l in range(len(layers))] if decode else
+             [(layer, xs[b]) for b in range(n_batches)])
+    n_units = len(units)
     sum_sq = torch.zeros(wl.E, dtype=torch.float64, device=dev)
     count = torch.zeros(wl.E, dtype=torch.int64, device=dev)
     kept = torch.empty(max(wl.keep, 1), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(x, ev=None):
-        layer.route(x)
+    def step(lay, x, ev=None):
+        lay.route(x)
         if ev:
             ev[0].record()
-        f, sh = layer.experts_and_shared(x)
+        f, sh = lay.experts_and_shared(x)
         if ev:
             ev[1].record()
         if kind == "refill":
-            abi.razor_refill_rms_accumulate(f, layer.slot_row[:T], layer.topk_idx[:T], layer.topk_logit[:T],
-                                            layer.offsets, sum_sq, count, shared_out=sh, y_out=layer.y[:T],
-                                            ws=layer.ws_refill)
+            abi.razor_refill_rms_accumulate(f, lay.slot_row[:T], lay.topk_idx[:T], lay.topk_logit[:T],
+                                            lay.offsets, sum_sq, count, shared_out=sh, y_out=lay.y[:T],
+                                            ws=lay.ws_refill)
             abi.razor_select(sum_sq, count, wl.keep, kept=kept)
         else:
-            abi.moe_combine(f, layer.slot_row[:T], layer.topk_w[:T], shared_out=sh, y=layer.y[:T])
+            abi.moe_combine(f, lay.slot_row[:T], lay.topk_w[:T], shared_out=sh, y=lay.y[:T])
 
-    # one CUDA graph per token batch; each holds timing events around the
-    # routed expert call (external event nodes, read after the timed region)
+    # one CUDA graph per unit for the timed steps, and a second set holding
+    # timing events around the expert call (external event nodes, read
+    # afterwards) for the expert roofline: event nodes between kernels would
+    # cut the programmatic launch edges of the timed steps
     ev_pairs = [(torch.cuda.Event(enable_timing=True, external=True),
-                 torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n_batches)]
-    graphs = None
+                 torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n_units)]
+    graphs = graphs_ev = None
+    launches_per_step = None
     if not args.no_graph:
-        graphs = [layer.capture(xs[b], lambda x, ev=ev_pairs[b]: step(x, ev)) for b in range(n_batches)]
+        graphs = [lay.capture(x, lambda xx, lay=lay: step(lay, xx)) for lay, x in units]
+        launches_per_step = layer.graph_kernels
+        graphs_ev = [lay.capture(x, lambda xx, lay=lay, ev=ev_pairs[u]: step(lay, xx, ev))
+                     for u, (lay, x) in enumerate(units)]
 
-    def run(i):
+    def run(i, with_events=False):
+        u = i % n_units
         if graphs:
-            graphs[i % n_batches].replay()
+            (graphs_ev if with_events else graphs)[u].replay()
         else:
-            step(xs[i % n_batches], ev_pairs[i % n_batches])
+            step(units[u][0], units[u][1], ev_pairs[u] if with_events else None)
 
-    for i in range(args.warmup):
+    for i in range(max(args.warmup, n_units)):
         run(i)
     torch.cuda.synchronize()
     assert abi.moe_device_status() == 0, "device status after warm-up"
@@ -346,32 +379,36 @@ def run_native(args, dist: Dist) -> None:
     clocks = ClockSampler(dist.local)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    # Decode-sized steps touch fewer weight bytes than L2 holds (the popular
-    # experts would stay cached from step to step): flush L2 before every
-    # timed step and time each step with its own events, flush excluded.
-    # Prefill steps stream GBs, larger than L2: one bracket over all steps.
-    flush_l2 = T < 256
-    l2_flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush_l2 else None
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start.record(stream)
     for i in range(args.steps):
-        if flush_l2:
-            l2_flush.zero_()
-        step_ev[i][0].record(stream)
         run(i)
-        step_ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
     clk = clocks.stop()
-    if flush_l2:
-        ms_local = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
-    else:
-        ms_local = t_start.elapsed_time(t_end) / args.steps
-    ms = dist.max(ms_local)
-    # the expert call of the last replay of every batch's graph (inside the timed region)
-    used = sorted({i % n_batches for i in range(max(0, args.steps - n_batches), args.steps)})
-    ffn_ms = dist.max(statistics.mean(ev_pairs[b][0].elapsed_time(ev_pairs[b][1]) for b in used))
+    ms = dist.max(t_start.elapsed_time(t_end) / args.steps)
+    # expert roofline: the same rotation with events around the expert call;
+    # each unit's last replay
+    for i in range(max(args.steps, n_units)):
+        run(i, with_events=True)
+    torch.cuda.synchronize()
+    ffn_ms = dist.max(statistics.mean(a.elapsed_time(b) for a, b in ev_pairs))
+    # for comparison: decode steps after an L2 flush by a write of 2x L2 (the
+    # flush leaves dirty lines whose write-back and the kernels' cold code
+    # fall inside the step), each step timed alone, the flush excluded
+    flush_ms = None
+    if decode:
+        l2_flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        fl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for i in range(args.steps):
+            l2_flush.zero_()
+            fl_ev[i][0].record(stream)
+            run(i)
+            fl_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        flush_ms = dist.max(sum(a.elapsed_time(b) for a, b in fl_ev) / args.steps)
+        del l2_flush
     status = abi.moe_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -380,53 +417,46 @@ def run_native(args, dist: Dist) -> None:
     tokens = T * dist.world
     value = tokens / (ms / 1e3)
     peaks = measured_peaks()
-    roofline = expert_roofline(wl, layer, T, rows, ffn_ms, peaks)
+    roofline = expert_roofline(wl, [u[0] for u in units], T, rows, ffn_ms, peaks)
 
     # end-to-end through the public API: pinned host x -> y in pinned host memory
     e2e = None
     if not args.no_e2e and kind == "forward":
-        xh = [xs[b].cpu().pin_memory() for b in range(n_batches)]
+        xh = [x.cpu().pin_memory() for _, x in units]
         yh = torch.empty((T, wl.H), dtype=layer.y.dtype).pin_memory()
         xd = torch.empty_like(xs[0])
-        g_e2e = None if args.no_graph else layer.capture(xd)
+        g_e2e = None if args.no_graph else [lay.capture(xd) for lay, _ in units]
 
         def e2e_step(i):
-            xd.copy_(xh[i % n_batches], non_blocking=True)
+            u = i % n_units
+            lay = units[u][0]
+            xd.copy_(xh[u], non_blocking=True)
             if g_e2e is not None:
-                g_e2e.replay()
+                g_e2e[u].replay()
             else:
-                layer.forward(xd)
-            yh.copy_(layer.y[:T], non_blocking=True)
+                lay.forward(xd)
+            yh.copy_(lay.y[:T], non_blocking=True)
 
-        for i in range(max(2, args.warmup)):
+        for i in range(max(2, args.warmup, n_units)):
             e2e_step(i)
         dist.barrier()
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
         a.record(stream)
         for i in range(args.steps):
-            if flush_l2:
-                l2_flush.zero_()
-            e2e_ev[i][0].record(stream)
             e2e_step(i)
-            e2e_ev[i][1].record(stream)
         b.record(stream)
         torch.cuda.synchronize()
         dist.barrier()
-        if flush_l2:
-            e2e_ms = dist.max(sum(p.elapsed_time(q) for p, q in e2e_ev) / args.steps)
-        else:
-            e2e_ms = dist.max(a.elapsed_time(b) / args.steps)
+        e2e_ms = dist.max(a.elapsed_time(b) / args.steps)
         e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
                "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
                "d2h_bytes_per_step": int(yh.numel() * yh.element_size()),
                "path": "pinned host x -> H2D copy -> layer (CUDA graph of the C-ABI calls) -> D2H copy of y"}
 
-    # kernels per step: route (logits + top-k), permute (4), experts, shared (2), combine / refill (+ reduce, select)
-    launches_per_step = 2 + 4 + (5 if wl.fmt == "nvfp4" else 3) + 2 + (3 if kind == "refill" else 1)
+    if launches_per_step is None:  # eager: count one pass's launches from a throw-away capture
+        launches_per_step = _count_step_kernels(layer, xs[0], lambda xx: step(layer, xx))
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -437,14 +467,19 @@ def run_native(args, dist: Dist) -> None:
                                f"fmt={wl.fmt}" + (" +Refill-RMS accumulate/select" if kind == "refill" else ""),
                    "tokens_per_step_per_gpu": T, "parallelism": f"dp{dist.world} (replicas, no collective)",
                    "launch": "eager C-ABI calls" if args.no_graph else "one CUDA graph per step (the C-ABI calls)",
-                   "l2": (f"L2 flushed (a {2 * L2_BYTES >> 20} MiB write) before every timed step; each step timed "
-                          "with its own CUDA events, the flush excluded" if T < 256 else
+                   "l2": (f"{n_units} layers with distinct weights in rotation ({layer_bytes / 2**30:.2f} GiB each); "
+                          "between two uses of a layer the others stream >= 3x the 126 MB L2 of expert weights, "
+                          "so no expert weight is cached when its layer runs again; no flush" if decode else
                           f"{n_batches} rotating token batches ({n_batches * x_bytes / 2**20:.0f} MiB) and "
-                          f"{sum(t.numel() * t.element_size() for t in w.values()) / 2**30:.1f} GiB of expert "
-                          "weights per step's reach, both larger than the 126 MB L2")},
+                          f"{layer_bytes / 2**30:.1f} GiB of expert weights per step's reach, both larger than the "
+                          "126 MB L2")},
         "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
         "expert_ffn_ms": round(ffn_ms, 4),
+        "ms_per_step_after_l2_write_flush": None if flush_ms is None else round(flush_ms, 4),
+        "launches_per_step": launches_per_step,
     }
+    roofline["timing"] = ("CUDA events around the expert call, in a second run of the same rotation right after "
+                          "the timed region; mean over the units")
     if dist.rank == 0 and not args.no_cpu_baseline:
         n = args.cpu_sample_tokens or (96 if kind == "refill" else 192)
         tps, dt = oracle_tokens_per_s(wl, w, xs[0], min(n, T), kind)

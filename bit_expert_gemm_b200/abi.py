@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 MOE_DTYPE_BF16, MOE_DTYPE_F16 = 0, 1
 (MOE_OP_ROUTE_TOPK, MOE_OP_PERMUTE, MOE_OP_SWIGLU_BF16, MOE_OP_SWIGLU_AWQ_G32, MOE_OP_SWIGLU_NVFP4, MOE_OP_REFILL,
- MOE_OP_NVFP4_QUANTIZE, MOE_OP_EXPERTS_BF16) = range(8)
+ MOE_OP_NVFP4_QUANTIZE, MOE_OP_EXPERTS_BF16, MOE_OP_ROUTE_PERMUTE) = range(9)
 
 
 class MoEError(RuntimeError):
@@ -45,6 +45,7 @@ _SIGS = {
     "moe_device_status": (_I, [_I, _P]),
     "moe_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "moe_route_topk": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "moe_route_permute": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_grouped_swiglu_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _SZ, _P]),
@@ -151,6 +152,37 @@ def moe_route_topk(x, w_router, bias, k: int, extra: int = 0, topk_idx=None, top
     _call("moe_route_topk", _p(x), T, H, _p(w_router), _p(bias), E, k, extra, _dtype_code(x), _p(topk_idx),
           _p(topk_w), _p(topk_logit), _p(ws), ws.numel(), _stream(stream))
     return topk_idx, topk_w, topk_logit
+
+
+def moe_route_permute(x, w_router, bias, k: int, extra: int = 0, topk_idx=None, topk_w=None, topk_logit=None,
+                      expert_offsets=None, row_token=None, slot_row=None, ws=None, stream=None):
+    """moe_route_topk then moe_permute of its selection, in one call (one
+    kernel for T <= 128).  Returns (topk_idx, topk_w, topk_logit,
+    expert_offsets, row_token, slot_row)."""
+    T, H = x.shape
+    E = w_router.shape[0]
+    ks = k + extra
+    dev = x.device
+    if topk_idx is None:
+        topk_idx = torch.empty((T, ks), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if topk_logit is None:
+        topk_logit = torch.empty((T, ks), dtype=torch.float32, device=dev)
+    if expert_offsets is None:
+        expert_offsets = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    if row_token is None:
+        row_token = torch.empty((T * ks,), dtype=torch.int32, device=dev)
+    if slot_row is None:
+        slot_row = torch.empty((T, ks), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(MOE_OP_ROUTE_PERMUTE, T, H, E, ks, 0, dev)
+    if bias is not None:
+        _need(bias, torch.float32, "bias")
+    _call("moe_route_permute", _p(x), T, H, _p(w_router), _p(bias), E, k, extra, _dtype_code(x), _p(topk_idx),
+          _p(topk_w), _p(topk_logit), _p(expert_offsets), _p(row_token), _p(slot_row), _p(ws), ws.numel(),
+          _stream(stream))
+    return topk_idx, topk_w, topk_logit, expert_offsets, row_token, slot_row
 
 
 def moe_permute(topk_idx, E: int, expert_offsets=None, row_token=None, slot_row=None, ws=None, stream=None):

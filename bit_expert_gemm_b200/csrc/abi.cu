@@ -16,6 +16,10 @@ int route_topk(const void* x, int T, int H, const void* w_router, const float* b
                int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, void* ws, size_t ws_bytes,
                cudaStream_t stream);
 size_t permute_ws_bytes(int T, int E);
+size_t route_permute_ws_bytes(int T, int E);
+int route_permute(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
+                  int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, int32_t* offsets,
+                  int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes, cudaStream_t stream);
 int permute(const int32_t* topk_idx, int T, int ks, int E, int32_t* offsets, int32_t* row_token, int32_t* slot_row,
             void* ws, size_t ws_bytes, cudaStream_t stream);
 int gather_rows(const void* x, const int32_t* row_token, int rows, int H, void* out, cudaStream_t stream);
@@ -100,6 +104,15 @@ unsigned long long wait_limit_ns() {
     lim = (ms > 0 ? (unsigned long long)ms : 5000ull) * 1000000ull;
   }
   return lim;
+}
+
+bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* s = getenv("BIT_EXPERT_GEMM_PDL");
+    on = (s && s[0] == '0') ? 0 : 1;
+  }
+  return on != 0;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -229,6 +242,7 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k_slots, int I) {
   switch (op) {
     case MOE_OP_ROUTE_TOPK: return route_ws_bytes(T, E);
     case MOE_OP_PERMUTE: return permute_ws_bytes(T, E);
+    case MOE_OP_ROUTE_PERMUTE: return route_permute_ws_bytes(T, E);
     case MOE_OP_SWIGLU_BF16: {
       WsCounter c;
       c.take<uint16_t>(size_t(rows) * I);
@@ -270,6 +284,29 @@ int moe_permute(const int32_t* topk_idx, int T, int k_slots, int E, int32_t* exp
   MOE_REQUIRE(long(T) * k_slots < (1l << 31), MOE_ERR_UNSUPPORTED, "moe_permute: T*k_slots overflows int32");
   return permute(topk_idx, T, k_slots, E, expert_offsets, row_token, slot_row, ws, ws_bytes,
                  static_cast<cudaStream_t>(stream));
+}
+
+int moe_route_permute(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
+                      int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, int32_t* expert_offsets,
+                      int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(T >= 0 && H > 0 && E > 0, MOE_ERR_INVALID_ARG, "moe_route_permute: bad sizes T=%d H=%d E=%d", T, H, E);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_route_permute: dtype %d",
+              dtype);
+  MOE_REQUIRE(extra == 0 || extra == 1, MOE_ERR_INVALID_ARG, "moe_route_permute: extra must be 0 or 1");
+  MOE_REQUIRE(k >= 1 && k + extra <= 16 && k + extra <= E, MOE_ERR_UNSUPPORTED,
+              "moe_route_permute: need 1 <= k, k+extra <= 16 and <= E (k=%d extra=%d E=%d)", k, extra, E);
+  MOE_REQUIRE(E <= 1024, MOE_ERR_UNSUPPORTED, "moe_route_permute: E=%d > 1024", E);
+  MOE_REQUIRE(H % 64 == 0, MOE_ERR_UNSUPPORTED, "moe_route_permute: H=%d is not a multiple of 64", H);
+  MOE_REQUIRE(long(T) * (k + extra) < (1l << 31), MOE_ERR_UNSUPPORTED, "moe_route_permute: T*(k+extra) overflows");
+  MOE_REQUIRE(expert_offsets != nullptr, MOE_ERR_INVALID_ARG, "moe_route_permute: expert_offsets is null");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) return permute(topk_idx, 0, k + extra, E, expert_offsets, row_token, slot_row, ws, ws_bytes, st);
+  MOE_REQUIRE(x && w_router && topk_idx && topk_w && row_token && slot_row, MOE_ERR_INVALID_ARG,
+              "moe_route_permute: null pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(w_router), MOE_ERR_INVALID_ARG,
+              "moe_route_permute: x / w_router not 16-byte aligned");
+  return route_permute(x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w, topk_logit, expert_offsets,
+                       row_token, slot_row, ws, ws_bytes, st);
 }
 
 int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows,

@@ -33,17 +33,28 @@ template <typename T16, bool F32>
 __global__ void __launch_bounds__(256) k_combine(const void* __restrict__ f, const int32_t* __restrict__ slot_row,
                                                  int ks, const float* __restrict__ w, const T16* __restrict__ shared,
                                                  const float* __restrict__ gate, int k, int H, T16* __restrict__ y) {
+  griddep_wait();  // f comes from the kernel just before (programmatic dependent launch)
+  griddep_launch_dependents();
   const int t = blockIdx.x;
   const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
   if (c >= H) return;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int j = 0; j < k; ++j) {
-    const int r = slot_row[size_t(t) * ks + j];
-    const float wj = w[size_t(t) * k + j];
-    float v[4];
-    load4<T16, F32>(f, size_t(r), H, c, v);
+  // all slots' rows and weights first, so that the k row loads are in flight together
+  int r[16];
+  float wj[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
+  for (int j = 0; j < 16; ++j) {
+    r[j] = j < k ? __ldg(slot_row + size_t(t) * ks + j) : 0;
+    wj[j] = j < k ? __ldg(w + size_t(t) * k + j) : 0.0f;
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j < k && r[j] >= 0) {  // -1: an assignment the permutation rejected
+      float v[4];
+      load4<T16, F32>(f, size_t(r[j]), H, c, v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(wj[j], v[i], acc[i]);
+    }
   }
   if (shared) {
     const float g = gate ? gate[t] : 1.0f;
@@ -62,19 +73,19 @@ int combine(const void* f, int f_fp32, const int32_t* slot_row, int ks, const fl
   if (dtype == MOE_DTYPE_BF16) {
     using T16 = __nv_bfloat16;
     if (f_fp32)
-      k_combine<T16, true><<<grid, 256, 0, stream>>>(f, slot_row, ks, w, static_cast<const T16*>(shared), gate, k, H,
-                                                     static_cast<T16*>(y));
+      MOE_CHECK_CUDA(launch_pdl(k_combine<T16, true>, grid, dim3(256), 0, stream, f, slot_row, ks, w,
+                                static_cast<const T16*>(shared), gate, k, H, static_cast<T16*>(y)));
     else
-      k_combine<T16, false><<<grid, 256, 0, stream>>>(f, slot_row, ks, w, static_cast<const T16*>(shared), gate, k, H,
-                                                      static_cast<T16*>(y));
+      MOE_CHECK_CUDA(launch_pdl(k_combine<T16, false>, grid, dim3(256), 0, stream, f, slot_row, ks, w,
+                                static_cast<const T16*>(shared), gate, k, H, static_cast<T16*>(y)));
   } else {
     using T16 = __half;
     if (f_fp32)
-      k_combine<T16, true><<<grid, 256, 0, stream>>>(f, slot_row, ks, w, static_cast<const T16*>(shared), gate, k, H,
-                                                     static_cast<T16*>(y));
+      MOE_CHECK_CUDA(launch_pdl(k_combine<T16, true>, grid, dim3(256), 0, stream, f, slot_row, ks, w,
+                                static_cast<const T16*>(shared), gate, k, H, static_cast<T16*>(y)));
     else
-      k_combine<T16, false><<<grid, 256, 0, stream>>>(f, slot_row, ks, w, static_cast<const T16*>(shared), gate, k, H,
-                                                      static_cast<T16*>(y));
+      MOE_CHECK_CUDA(launch_pdl(k_combine<T16, false>, grid, dim3(256), 0, stream, f, slot_row, ks, w,
+                                static_cast<const T16*>(shared), gate, k, H, static_cast<T16*>(y)));
   }
   MOE_CHECK_CUDA(cudaGetLastError());
   return MOE_OK;

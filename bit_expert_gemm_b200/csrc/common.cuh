@@ -37,6 +37,36 @@ int pick_bn(int rows, int groups, int n_out, bool swiglu);
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch
+//
+// A kernel launched with launch_pdl may start while the kernel before it on
+// the stream is still running.  Every kernel so launched follows one rule:
+// its prologue touches no output of the previous kernel; then it executes
+// griddep_wait() (the previous kernel has completed and its writes are
+// visible), then griddep_launch_dependents() (its own dependent may start).
+// So when a kernel starts, everything two kernels back on the stream has
+// completed, and it may read those outputs before its own wait.  Without the
+// launch attribute both instructions return at once.
+// ---------------------------------------------------------------------------
+bool pdl_enabled();  // false when the environment sets BIT_EXPERT_GEMM_PDL=0 (abi.cu)
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // Carves consecutive 256-byte aligned pieces out of a workspace.
 struct WsCarver {
   char* base;
@@ -69,6 +99,11 @@ struct WsCounter {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void report(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {

@@ -14,12 +14,14 @@
 //   GEMM2 (MODE_DOWN): a work item is 128 rows of W_d; f[r, n] = h[r] . Wd[n].
 // Rows: the routed rows [0, rows) in permuted order, then the shared
 // expert's T rows (identity tokens).  The token operand of both GEMMs is
-// gathered with cp.async (x rows through row_token, or h rows) and signals
-// its stage barrier when the copies land, so the gathers of many K steps are
-// in flight at once.
+// gathered with cp.async (x rows through row_token, or h rows); each gather
+// thread arrives on the stage's full barrier when its copies land, the TMA
+// producer's arrival carries the weight bytes, so one barrier per stage
+// covers both operands and the gathers of many stages are in flight at once.
 //
 // Warp roles: 0 TMA producer (weights), 1 UMMA issuer (TMEM owner),
 // 2..5 epilogue, 6..9 token-operand gather.
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -34,13 +36,20 @@ namespace {
 constexpr int BM = 128;             // weight rows per work item (MMA M)
 constexpr int BK = 64;              // K per pipeline step (one 128-byte swizzle row)
 constexpr int NMAX = 128;           // token rows per group handled in one pass (MMA N <= 128)
-constexpr int A_BYTES = BM * BK * 2;    // 16 KB of weights per step
-constexpr int B_BYTES = NMAX * BK * 2;  // 16 KB of tokens per step (at most)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB of weights per 64-wide K sub-tile
+// A pipeline stage holds ksub K sub-tiles: ksub weight tiles and ksub token
+// tiles of bn_max rows (the largest group rounded up to 16, at most NMAX).
+// With N = 16 tokens an MMA does little work, and the per-stage cost of the
+// issuing thread (barrier waits, commit: several hundred cycles) would cap
+// the weight stream of an SM; ksub > 1 spreads that cost over more bytes.
+// Smaller token tiles leave room for more stages.
+constexpr int MAX_STAGES = 12;
+constexpr int FULL_ARRIVALS = 1 + 128;  // producer (with the TMA bytes) + one per gather thread
 constexpr int XCHG_STRIDE = 33;     // floats per row of the gate/up exchange buffer (bank-conflict padding)
 constexpr int XCHG_BYTES = 64 * XCHG_STRIDE * 4;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + XCHG_BYTES;
+constexpr int SMEM_BYTES = 217 * 1024;  // dynamic; + ~9 KB static stays under the 227 KB per block
+constexpr int STAGE_SPACE = SMEM_BYTES - 1024 - XCHG_BYTES;
+static_assert(STAGE_SPACE >= 6 * (A_BYTES + NMAX * BK * 2), "six full stages must fit");
 constexpr int kThreads = 320;
 constexpr int kGatherThreads = 128;
 constexpr uint32_t TMEM_COLS = 2 * NMAX;  // two accumulators of 128 x NMAX
@@ -66,6 +75,9 @@ struct Args {
   void* shared_out;  // GEMM2: shared rows [T, H] (16-bit)
   int f_fp32;
   int bf16;
+  int bn_max;  // token rows per sub-tile: round16(min(largest group, NMAX))
+  int ksub;    // K sub-tiles (64 wide) per pipeline stage
+  int stages;  // pipeline depth for that stage size
   int* status;
   unsigned long long limit_ns;
 };
@@ -111,7 +123,7 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_decode_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWs, const Args args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[STAGES], bready_bar[STAGES], empty_bar[STAGES], tfull_bar[2],
+  __shared__ __align__(8) uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES], tfull_bar[2],
       tempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
@@ -120,17 +132,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int warp_sums[kThreads / 32];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  auto smA = [&](int s) { return smem + s * STAGE_BYTES; };
-  auto smB = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
-  float* xchg = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+  const int STAGES = args.stages;
+  const int ksub = args.ksub;
+  const int b_sub_bytes = args.bn_max * BK * 2;
+  const int stage_bytes = ksub * (A_BYTES + b_sub_bytes);
+  // sub-tile j of stage s: weights at smA(s) + j * A_BYTES, tokens at smB(s) + j * b_sub_bytes
+  auto smA = [&](int s) { return smem + s * stage_bytes; };
+  auto smB = [&](int s) { return smem + s * stage_bytes + ksub * A_BYTES; };
+  float* xchg = reinterpret_cast<float*>(smem + STAGES * stage_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = args.E, G = E + 1;
   const int MB = args.MB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&bready_bar[s], kGatherThreads);
+      mbar_init(&full_bar[s], FULL_ARRIVALS);
       mbar_init(&empty_bar[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -148,6 +164,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, TMEM_COLS);
     tmem_relinquish();
+  }
+  // Launched as a programmatic dependent: GEMM1's routing comes from the
+  // kernel just before it, so it waits here; GEMM2's routing is two kernels
+  // back (complete when GEMM2 starts), so GEMM2 schedules and streams weights
+  // at once and only its gather of h waits for GEMM1.
+  if (MODE == MODE_GATE_UP) {
+    griddep_wait();
+    griddep_launch_dependents();
   }
   // work items: every group with rows contributes MB blocks of weight rows
   for (int i = threadIdx.x; i <= E; i += blockDim.x) goff[i] = args.offsets[i];
@@ -184,7 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
   const int total = item_start[G];
-  const int KB = args.K / BK;
+  const int KB = args.K / BK;               // 64-wide K sub-tiles per work item
+  const int NS = (KB + ksub - 1) / ksub;     // pipeline stages per work item (the last may be partial)
   int* status = args.status;
   const unsigned long long lim = args.limit_ns;
   auto item_of = [&](int L) {
@@ -209,17 +234,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
         const Item it = item_of(L);
         const CUtensorMap* map = it.g < E ? &tmW : &tmWs;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int ks = 0; ks < NS; ++ks) {
+          const int nsub = min(ksub, KB - ks * ksub);
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], A_BYTES);
-          if (MODE == MODE_GATE_UP) {
-            // 64 gate rows, then the 64 up rows of the same features
-            const int base = it.g < E ? it.g * 2 * args.I : 0;
-            tma_load_2d(smA(stage), map, &full_bar[stage], kb * BK, base + it.mb * 64);
-            tma_load_2d(smA(stage) + 64 * BK * 2, map, &full_bar[stage], kb * BK, base + args.I + it.mb * 64);
-          } else {
-            const int base = it.g < E ? it.g * args.H : 0;
-            tma_load_2d(smA(stage), map, &full_bar[stage], kb * BK, base + it.mb * BM);
+          mbar_arrive_expect_tx(&full_bar[stage], uint32_t(nsub * A_BYTES));
+          for (int j = 0; j < nsub; ++j) {
+            const int kx = (ks * ksub + j) * BK;
+            uint8_t* a = smA(stage) + j * A_BYTES;
+            if (MODE == MODE_GATE_UP) {
+              // 64 gate rows, then the 64 up rows of the same features
+              const int base = it.g < E ? it.g * 2 * args.I : 0;
+              tma_load_2d(a, map, &full_bar[stage], kx, base + it.mb * 64);
+              tma_load_2d(a + 64 * BK * 2, map, &full_bar[stage], kx, base + args.I + it.mb * 64);
+            } else {
+              const int base = it.g < E ? it.g * args.H : 0;
+              tma_load_2d(a, map, &full_bar[stage], kx, base + it.mb * BM);
+            }
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -243,20 +273,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = item_of(L);
         int r0, n;
         group_rows(goff, it.g, E, args.rows, args.T, r0, n);
-        const int npad = (min(n, NMAX) + 15) & ~15;
+        const int npad = (min(n, args.bn_max) + 15) & ~15;
         const uint32_t idesc = idesc_f16(args.bf16, BM, npad);
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, &abort_flag, status, lim)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(acc * NMAX);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int ks = 0; ks < NS; ++ks) {
+          const int nsub = min(ksub, KB - ks * ksub);
           if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
-          if (!mbar_wait(&bready_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t ad = sdesc_kmajor_sw128(smem_u32(smA(stage)));
-          const uint64_t bd = sdesc_kmajor_sw128(smem_u32(smB(stage)));
+          for (int j = 0; j < nsub; ++j) {
+            const uint64_t ad = sdesc_kmajor_sw128(smem_u32(smA(stage) + j * A_BYTES));
+            const uint64_t bd = sdesc_kmajor_sw128(smem_u32(smB(stage) + j * b_sub_bytes));
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_f16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_f16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (ks | j | kk) != 0);
+          }
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -278,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = item_of(L);
       int r0, n;
       group_rows(goff, it.g, E, args.rows, args.T, r0, n);
-      const int nn = min(n, NMAX);
-      if (n > NMAX && warp == 2 && lane == 0) report(status, MOE_ERR_UNSUPPORTED);  // > 128 rows in one group
+      const int nn = min(n, args.bn_max);
+      if (n > args.bn_max && warp == 2 && lane == 0) report(status, MOE_ERR_UNSUPPORTED);  // more rows than the token tile
       // a timed-out wait in one warp must not leave the others at a named barrier
       if (!epilogue_all(mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag, status, lim))) break;
       tc_fence_after();
@@ -346,6 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // XOR row mod 8); rows from the group size up to the next multiple of 16
     // are zero-filled.  Each thread arrives on the stage's barrier once its
     // copies have landed.
+    if (MODE == MODE_DOWN) {  // h is GEMM1's output
+      griddep_wait();
+      griddep_launch_dependents();
+    }
     const int gt = threadIdx.x - 192;
     const int ch = gt & 7;
     const int cb = gt >> 3;
@@ -357,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = item_of(L);
       int r0, n;
       group_rows(goff, it.g, E, args.rows, args.T, r0, n);
-      const int nn = min(n, NMAX);
+      const int nn = min(n, args.bn_max);
       const int npad = (nn + 15) & ~15;
       int row[8];
 #pragma unroll
@@ -374,18 +410,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         row[i] = rr;
       }
       bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int ks = 0; ks < NS; ++ks) {
+        const int nsub = min(ksub, KB - ks * ksub);
         if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
-        const uint32_t bt = smem_u32(smB(stage));
+        for (int j = 0; j < nsub; ++j) {
+          const uint32_t bt = smem_u32(smB(stage) + j * b_sub_bytes);
+          const size_t kbyte = size_t(ks * ksub + j) * 128;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int c = cb + 16 * i;
-          if (c < npad) {
-            const uint8_t* g = src + (row[i] >= 0 ? size_t(row[i]) * pitch + size_t(kb) * 128 + ch * 16 : 0);
-            cp_async_16_zfill(bt + uint32_t(c * 128 + ((ch ^ (c & 7)) << 4)), g, row[i] >= 0 ? 16u : 0u);
+          for (int i = 0; i < 8; ++i) {
+            const int c = cb + 16 * i;
+            if (c < npad) {
+              const uint8_t* g = src + (row[i] >= 0 ? size_t(row[i]) * pitch + kbyte + ch * 16 : 0);
+              cp_async_16_zfill(bt + uint32_t(c * 128 + ((ch ^ (c & 7)) << 4)), g, row[i] >= 0 ? 16u : 0u);
+            }
           }
         }
-        cp_async_arrive_noinc(&bready_bar[stage]);
+        cp_async_arrive_noinc(&full_bar[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
@@ -401,6 +441,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+int stages_for(int ksub, int bn_max) {
+  const int per_stage = ksub * (A_BYTES + bn_max * BK * 2);
+  return STAGE_SPACE / per_stage < MAX_STAGES ? STAGE_SPACE / per_stage : MAX_STAGES;
+}
+
+// K sub-tiles per stage: the widest of 4, 2, 1 that leaves a double-buffered
+// pipeline (measured on B200: 4 sub-tiles in 2 stages stream faster than 2 in
+// 4).  BIT_EXPERT_GEMM_DECODE_KSUB (1, 2 or 4) overrides it for tuning.
+int decode_ksub(int bn_max) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* s = getenv("BIT_EXPERT_GEMM_DECODE_KSUB");
+    const int e = s ? atoi(s) : 0;
+    forced = (e == 1 || e == 2 || e == 4) ? e : 0;
+  }
+  if (forced && stages_for(forced, bn_max) >= 2) return forced;
+  for (int k = 4; k > 1; k >>= 1)
+    if (stages_for(k, bn_max) >= 2) return k;
+  return 1;
+}
+
 template <int MODE>
 int launch_decode(const CUtensorMap& tw, const CUtensorMap& tws, const Args& a, cudaStream_t stream) {
   static bool attr_set[64] = {false};
@@ -410,8 +471,7 @@ int launch_decode(const CUtensorMap& tw, const CUtensorMap& tws, const Args& a, 
     MOE_CHECK_CUDA(cudaFuncSetAttribute(k_decode_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     if (dev < 64) attr_set[dev] = true;
   }
-  k_decode_gemm<MODE><<<num_sms(), kThreads, SMEM_BYTES, stream>>>(tw, tws, a);
-  MOE_CHECK_CUDA(cudaGetLastError());
+  MOE_CHECK_CUDA(launch_pdl(k_decode_gemm<MODE>, dim3(num_sms()), dim3(kThreads), SMEM_BYTES, stream, tw, tws, a));
   return MOE_OK;
 }
 
@@ -455,6 +515,12 @@ int decode_experts_16bit(const void* x, const int32_t* row_token, const int32_t*
   a.bf16 = dtype == MOE_DTYPE_BF16;
   a.status = device_status_ptr();
   a.limit_ns = wait_limit_ns();
+  // every group (routed: tokens that chose the expert; shared: all T) has at most T rows
+  a.bn_max = ((T < NMAX ? T : NMAX) + 15) & ~15;
+  a.ksub = decode_ksub(a.bn_max);
+  a.stages = stages_for(a.ksub, a.bn_max);
+  MOE_REQUIRE(a.stages >= 2, MOE_ERR_UNSUPPORTED, "decode experts: %d K sub-tiles per stage leave %d stages",
+              a.ksub, a.stages);
   // GEMM1 (+ SwiGLU): tokens gathered from x
   a.K = H;
   a.MB = I / 64;

@@ -1,49 +1,23 @@
 // Router logits, softmax over all experts, top-k and renormalised weights.
 //
 // Logits: for large T the tcgen05 grouped GEMM (one group, FP32 output with
-// the bias added in its epilogue); for small T a warp-per-expert GEMV that
-// streams each router row once.  Top-k: one warp per token, each lane holds
-// E/32 logits; k+extra rounds of a warp arg-max with ties to the lower index.
-// Because softmax is monotone and the selected weights are renormalised over
-// the selection, w_j = exp(l_j - l_max) / sum_S exp(l_i - l_max) equals
-// softmax(l)_j / sum_S softmax(l)_i, so only the selected logits are needed.
-#include <float.h>
-
+// the bias added in its epilogue); for small T a CUDA-core kernel in which
+// each block stages a few router rows in shared memory and its warps take the
+// tokens, so every router row is read from HBM once.  Top-k: one warp per
+// token (route.cuh).
 #include "common.cuh"
 #include "gemm_sm100.cuh"
+#include "route.cuh"
 
 namespace moe {
 
 template <typename T16>
-__global__ void __launch_bounds__(256) k_router_gemv(const T16* __restrict__ x, const T16* __restrict__ wr,
-                                                     const float* __restrict__ bias, int T, int H, int E,
-                                                     float* __restrict__ logits) {
-  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (e >= E) return;
-  const uint4* wrow = reinterpret_cast<const uint4*>(wr + size_t(e) * H);
-  const int nchunk = H / 8;
-  const float b = bias ? bias[e] : 0.0f;
-  for (int t = 0; t < T; ++t) {
-    const uint4* xrow = reinterpret_cast<const uint4*>(x + size_t(t) * H);
-    float acc = 0.0f;
-    for (int c = lane; c < nchunk; c += 32) {
-      uint4 wv = __ldg(wrow + c);
-      uint4 xv = __ldg(xrow + c);
-      const uint32_t* wp = reinterpret_cast<const uint32_t*>(&wv);
-      const uint32_t* xp = reinterpret_cast<const uint32_t*>(&xv);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float2 a = Pack2<T16>::unpack(wp[i]);
-        float2 bb = Pack2<T16>::unpack(xp[i]);
-        acc = fmaf(a.x, bb.x, acc);
-        acc = fmaf(a.y, bb.y, acc);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) logits[size_t(t) * E + e] = acc + b;
-  }
+__global__ void __launch_bounds__(256) k_router_small(const T16* __restrict__ x, const T16* __restrict__ wr,
+                                                      const float* __restrict__ bias, int T, int H, int E,
+                                                      float* __restrict__ logits) {
+  extern __shared__ __align__(16) uint8_t route_smem[];
+  router_block_logits<T16>(x, wr, bias, T, H, E, blockIdx.x * kRouterEB, reinterpret_cast<uint4*>(route_smem),
+                           logits);
 }
 
 // One warp per token.  NV = values per lane (E <= 32 * NV).
@@ -52,65 +26,9 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, 
                                               int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                                               float* __restrict__ topk_logit) {
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  const float* row = logits + size_t(t) * E;
-  float v[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int e = lane + 32 * i;
-    float x = e < E ? row[e] : -FLT_MAX;
-    v[i] = (x != x) ? -FLT_MAX : x;  // NaN never wins
-  }
-  uint32_t removed = 0;  // bit i: value i of this lane already selected (or absent)
-#pragma unroll
-  for (int i = 0; i < NV; ++i)
-    if (lane + 32 * i >= E) removed |= 1u << i;
-  float sel_v[16];
-  int sel_i[16];
-#pragma unroll 1
-  for (int r = 0; r < ks; ++r) {
-    float bv = -FLT_MAX;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int e = lane + 32 * i;
-      if (!(removed >> i & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
-        bv = v[i];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if ((bi & 31) == lane) removed |= 1u << (bi >> 5);
-    sel_v[r] = bv;
-    sel_i[r] = bi;
-  }
-  // renormalised softmax weights over the k selected experts
-  const float m = sel_v[0];
-  float z = 0.0f;
-  float p[16];
-#pragma unroll
-  for (int r = 0; r < 16; ++r) {
-    p[r] = r < k ? __expf(sel_v[r] - m) : 0.0f;
-    z += p[r];
-  }
-  const float inv = 1.0f / z;
-#pragma unroll
-  for (int r = 0; r < 16; ++r) {
-    if (r < ks && lane == r) {
-      topk_idx[size_t(t) * ks + r] = sel_i[r];
-      if (topk_logit) topk_logit[size_t(t) * ks + r] = sel_v[r];
-      if (r < k) topk_w[size_t(t) * k + r] = p[r] * inv;
-    }
-  }
+  topk_token<NV>(logits + size_t(t) * E, E, k, ks, threadIdx.x & 31, topk_idx + size_t(t) * ks,
+                 topk_w + size_t(t) * k, topk_logit ? topk_logit + size_t(t) * ks : nullptr);
 }
 
 size_t route_ws_bytes(int T, int E) {
@@ -148,14 +66,23 @@ int route_topk(const void* x, int T, int H, const void* w_router, const float* b
     int rc = launch_grouped_gemm(x, T, w_router, E, a, EPI_STORE, bn, stream);
     if (rc) return rc;
   } else {
-    const int blocks = (E * 32 + 255) / 256;
-    if (dtype == MOE_DTYPE_BF16)
-      k_router_gemv<__nv_bfloat16><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x),
-                                                                static_cast<const __nv_bfloat16*>(w_router), bias,
-                                                                T, H, E, logits);
-    else
-      k_router_gemv<__half><<<blocks, 256, 0, stream>>>(static_cast<const __half*>(x),
-                                                         static_cast<const __half*>(w_router), bias, T, H, E, logits);
+    const int blocks = (E + kRouterEB - 1) / kRouterEB;
+    const size_t smem = size_t(kRouterEB) * H * 2;
+    if (dtype == MOE_DTYPE_BF16) {
+      if (smem > 48 * 1024)
+        MOE_CHECK_CUDA(cudaFuncSetAttribute(k_router_small<__nv_bfloat16>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+      k_router_small<__nv_bfloat16><<<blocks, 256, smem, stream>>>(static_cast<const __nv_bfloat16*>(x),
+                                                                   static_cast<const __nv_bfloat16*>(w_router),
+                                                                   bias, T, H, E, logits);
+    } else {
+      if (smem > 48 * 1024)
+        MOE_CHECK_CUDA(cudaFuncSetAttribute(k_router_small<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            int(smem)));
+      k_router_small<__half><<<blocks, 256, smem, stream>>>(static_cast<const __half*>(x),
+                                                            static_cast<const __half*>(w_router), bias, T, H, E,
+                                                            logits);
+    }
     MOE_CHECK_CUDA(cudaGetLastError());
   }
   const int blocks = (T * 32 + 255) / 256;

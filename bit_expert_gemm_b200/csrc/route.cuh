@@ -1,0 +1,134 @@
+// Device pieces of routing shared by the standalone router / top-k kernels
+// and the fused small-batch route + permute kernel.
+//
+//   l[t, e] = x[t] . w_router[e] + bias[e]   (FP32 accumulate)
+//   S_t     = the k (+ extra) largest l[t, :], ties to the lower expert index
+//   w[t, j] = exp(l_j - l_max) / sum_{i in S_t, i < k} exp(l_i - l_max)
+//
+// softmax is monotone and the selected probabilities are renormalised over
+// the selection, so the renormalised softmax weights need only the selected
+// logits (the softmax denominator over all E experts cancels).
+#pragma once
+#include <float.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kRouterEB = 4;  // experts per block of the small-batch logits kernel
+
+// Logits of experts [e0, e0 + kRouterEB) for every token.  The block's weight
+// rows are staged in shared memory (w_sh: kRouterEB * H 16-bit values); warp
+// w then takes tokens w, w + nwarps, ...: its lanes stride over H in 8-value
+// chunks keeping one partial sum per expert, reduced across the warp at the
+// end.  Every thread of the block must call this.
+template <typename T16>
+__device__ void router_block_logits(const T16* __restrict__ x, const T16* __restrict__ wr,
+                                    const float* __restrict__ bias, int T, int H, int E, int e0, uint4* w_sh,
+                                    float* __restrict__ logits) {
+  const int nchunk = H / 8;
+  const int ne = min(kRouterEB, E - e0);
+  const uint4* src = reinterpret_cast<const uint4*>(wr + size_t(e0) * H);
+  for (int i = threadIdx.x; i < ne * nchunk; i += blockDim.x) w_sh[i] = __ldg(src + i);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int t = warp; t < T; t += nw) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + size_t(t) * H);
+    float acc[kRouterEB];
+#pragma unroll
+    for (int e = 0; e < kRouterEB; ++e) acc[e] = 0.0f;
+    for (int c = lane; c < nchunk; c += 32) {
+      const uint4 xv = __ldg(xr + c);
+      const uint32_t* xp = reinterpret_cast<const uint32_t*>(&xv);
+      float2 xf[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xf[i] = Pack2<T16>::unpack(xp[i]);
+#pragma unroll
+      for (int e = 0; e < kRouterEB; ++e) {
+        if (e < ne) {
+          const uint4 wv = w_sh[e * nchunk + c];
+          const uint32_t* wp = reinterpret_cast<const uint32_t*>(&wv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 wf = Pack2<T16>::unpack(wp[i]);
+            acc[e] = fmaf(wf.x, xf[i].x, acc[e]);
+            acc[e] = fmaf(wf.y, xf[i].y, acc[e]);
+          }
+        }
+      }
+    }
+    float mine = 0.0f;
+#pragma unroll
+    for (int e = 0; e < kRouterEB; ++e) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+      if (lane == e) mine = acc[e];
+    }
+    if (lane < ne) logits[size_t(t) * E + e0 + lane] = mine + (bias ? bias[e0 + lane] : 0.0f);
+  }
+  __syncthreads();  // w_sh is refilled by the caller's next block
+}
+
+// Top-(k + extra) of one token's logits by one warp: each lane holds E/32
+// values (NV per lane, E <= 32 * NV); ks rounds of a warp arg-max with ties
+// to the lower index; NaN never wins.  Lane r keeps the r-th selection and
+// writes idx_out[r], logit_out[r] (if not null) and, for r < k, the
+// renormalised weight w_out[r].  `row` is read through L2 (it may have been
+// written by other blocks of the same kernel).
+template <int NV>
+__device__ __forceinline__ void topk_token(const float* row, int E, int k, int ks, int lane, int32_t* idx_out,
+                                           float* w_out, float* logit_out) {
+  float v[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    const float x = e < E ? __ldcg(row + e) : -FLT_MAX;
+    v[i] = (x != x) ? -FLT_MAX : x;
+  }
+  uint32_t removed = 0;  // bit i: value i of this lane already selected (or absent)
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+    if (lane + 32 * i >= E) removed |= 1u << i;
+  float my_v = 0.0f, top = 0.0f;
+  int my_i = 0;
+#pragma unroll 1
+  for (int r = 0; r < ks; ++r) {
+    float bv = -FLT_MAX;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      if (!(removed >> i & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) removed |= 1u << (bi >> 5);
+    if (lane == r) {
+      my_v = bv;
+      my_i = bi;
+    }
+    if (r == 0) top = bv;
+  }
+  // renormalised softmax over the k selected experts (max-shifted)
+  const float p = lane < k ? __expf(my_v - top) : 0.0f;
+  float z = p;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  if (lane < ks) {
+    idx_out[lane] = my_i;
+    if (logit_out) logit_out[lane] = my_v;
+    if (lane < k) w_out[lane] = p * (1.0f / z);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,229 @@
+// Routing and permutation of a small batch (T <= 128 tokens, decode) in one
+// cooperative kernel, instead of the router, top-k and four permutation
+// launches that a large batch takes.  Three phases separated by grid-wide
+// barriers:
+//   1. logits: every block computes kRouterEB experts' logits for all tokens
+//      (router rows read from HBM once);
+//   2. top-k and renormalised weights: one warp per token;
+//   3. permutation, by block 0 alone: each expert's tokens as a bitmask in
+//      shared memory (T <= 128: at most four words per expert), counts by
+//      popcount, exclusive scan into expert_offsets, and every assignment's
+//      row = offset + popcount of the expert's bits below its token.  Same
+//      order as the standalone permutation: experts ascending, tokens
+//      ascending inside an expert.
+// Values written by other blocks of this launch are read with ld.global.cg
+// (through L2) after the grid barrier.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "route.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace moe {
+
+size_t route_ws_bytes(int T, int E);
+size_t permute_ws_bytes(int T, int E);
+int route_topk(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
+               int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, void* ws, size_t ws_bytes,
+               cudaStream_t stream);
+int permute(const int32_t* topk_idx, int T, int ks, int E, int32_t* offsets, int32_t* row_token, int32_t* slot_row,
+            void* ws, size_t ws_bytes, cudaStream_t stream);
+
+constexpr int kRouteSmallMaxT = 128;
+
+namespace {
+
+constexpr int kThreads = 256;
+
+struct RouteSmallArgs {
+  const void* x;
+  const void* wr;
+  const float* bias;
+  int T, H, E, k, ks;
+  float* logits;  // [T, E] scratch
+  int32_t* topk_idx;
+  float* topk_w;
+  float* topk_logit;
+  int32_t* offsets;
+  int32_t* row_token;
+  int32_t* slot_row;
+  int* status;
+};
+
+template <typename T16, int NV>
+__global__ void __launch_bounds__(kThreads) k_route_permute_small(const RouteSmallArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  cg::grid_group grid = cg::this_grid();
+  // launched after its inputs are complete: a programmatic dependent may start its prologue now
+  griddep_launch_dependents();
+  const int E = a.E, T = a.T, ks = a.ks;
+  // 1. logits
+  for (int eb = blockIdx.x; eb * kRouterEB < E; eb += gridDim.x)
+    router_block_logits<T16>(static_cast<const T16*>(a.x), static_cast<const T16*>(a.wr), a.bias, T, a.H, E,
+                             eb * kRouterEB, reinterpret_cast<uint4*>(smem), a.logits);
+  grid.sync();
+  // 2. top-k
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = blockIdx.x * (kThreads / 32) + warp; t < T; t += gridDim.x * (kThreads / 32))
+    topk_token<NV>(a.logits + size_t(t) * E, E, a.k, ks, lane, a.topk_idx + size_t(t) * ks,
+                   a.topk_w + size_t(t) * a.k, a.topk_logit ? a.topk_logit + size_t(t) * ks : nullptr);
+  grid.sync();
+  if (blockIdx.x != 0) return;
+  // 3. permutation (block 0)
+  const int W = (T + 31) / 32;
+  uint32_t* mask = reinterpret_cast<uint32_t*>(smem);  // [E, W]
+  int* off = reinterpret_cast<int*>(mask + E * W);     // [E + 1]
+  __shared__ int warp_tot[kThreads / 32];
+  for (int i = threadIdx.x; i < E * W; i += kThreads) mask[i] = 0;
+  __syncthreads();
+  const int n = T * ks;
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const int e = __ldcg(a.topk_idx + i);
+    const int t = i / ks;
+    if (e < 0 || e >= E) {
+      report(a.status, MOE_ERR_INVALID_ARG);
+      continue;
+    }
+    atomicOr(mask + e * W + (t >> 5), 1u << (t & 31));
+  }
+  __syncthreads();
+  // exclusive scan of the counts; thread i owns experts 4i .. 4i+3 (E <= 1024)
+  int cnt[4], local = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = threadIdx.x * 4 + j;
+    cnt[j] = 0;
+    if (e < E)
+      for (int w = 0; w < W; ++w) cnt[j] += __popc(mask[e * W + w]);
+    local += cnt[j];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int run = incl - local;
+  for (int w = 0; w < warp; ++w) run += warp_tot[w];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = threadIdx.x * 4 + j;
+    if (e < E) {
+      off[e] = run;
+      a.offsets[e] = run;
+    }
+    run += cnt[j];
+  }
+  if (threadIdx.x == kThreads - 1) {
+    off[E] = run;
+    a.offsets[E] = run;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const int e = __ldcg(a.topk_idx + i);
+    const int t = i / ks;
+    if (e < 0 || e >= E) {
+      a.slot_row[i] = -1;
+      continue;
+    }
+    const uint32_t* m = mask + e * W;
+    int rank = __popc(m[t >> 5] & ((1u << (t & 31)) - 1u));
+    for (int w = 0; w < (t >> 5); ++w) rank += __popc(m[w]);
+    const int pos = off[e] + rank;
+    a.row_token[pos] = t;
+    a.slot_row[i] = pos;
+  }
+}
+
+template <typename T16, int NV>
+int launch_small(const RouteSmallArgs& a, size_t smem, cudaStream_t stream) {
+  auto kern = k_route_permute_small<T16, NV>;
+  constexpr int kMaxDev = 64;
+  static int co_resident[kMaxDev] = {0};
+  static size_t smem_set[kMaxDev] = {0};
+  int dev = 0;
+  MOE_CHECK_CUDA(cudaGetDevice(&dev));
+  MOE_REQUIRE(dev < kMaxDev, MOE_ERR_UNSUPPORTED, "moe_route_permute: device %d >= %d", dev, kMaxDev);
+  if (smem > smem_set[dev] || co_resident[dev] == 0) {
+    if (smem > 48 * 1024)
+      MOE_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    int per_sm = 0;
+    MOE_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem));
+    MOE_REQUIRE(per_sm > 0, MOE_ERR_UNSUPPORTED, "moe_route_permute: kernel does not fit on an SM");
+    co_resident[dev] = per_sm * num_sms();
+    smem_set[dev] = smem;
+  }
+  const int want = (a.E + kRouterEB - 1) / kRouterEB;
+  const int grid = want < co_resident[dev] ? want : co_resident[dev];
+  void* params[] = {const_cast<RouteSmallArgs*>(&a)};
+  MOE_CHECK_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(kThreads), params,
+                                             smem, stream));
+  return MOE_OK;
+}
+
+template <typename T16>
+int dispatch_small(const RouteSmallArgs& a, size_t smem, cudaStream_t stream) {
+  const int nv = (a.E + 31) / 32;
+  if (nv <= 4) return launch_small<T16, 4>(a, smem, stream);
+  if (nv <= 8) return launch_small<T16, 8>(a, smem, stream);
+  if (nv <= 16) return launch_small<T16, 16>(a, smem, stream);
+  return launch_small<T16, 32>(a, smem, stream);
+}
+
+}  // namespace
+
+size_t route_permute_ws_bytes(int T, int E) {
+  if (T <= kRouteSmallMaxT) return route_ws_bytes(T, E);
+  WsCounter c;
+  c.take<uint8_t>(route_ws_bytes(T, E));
+  c.take<uint8_t>(permute_ws_bytes(T, E));
+  return c.used;
+}
+
+int route_permute(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
+                  int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, int32_t* offsets,
+                  int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const int ks = k + extra;
+  if (T > kRouteSmallMaxT) {
+    WsCarver carve(ws, ws_bytes);
+    void* ws_r = carve.take<uint8_t>(route_ws_bytes(T, E));
+    void* ws_p = carve.take<uint8_t>(permute_ws_bytes(T, E));
+    MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_route_permute: workspace of %zu bytes is too small", ws_bytes);
+    int rc = route_topk(x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w, topk_logit, ws_r,
+                        route_ws_bytes(T, E), stream);
+    if (rc) return rc;
+    return permute(topk_idx, T, ks, E, offsets, row_token, slot_row, ws_p, permute_ws_bytes(T, E), stream);
+  }
+  WsCarver carve(ws, ws_bytes);
+  float* logits = carve.take<float>(size_t(T) * E);
+  MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_route_permute: workspace of %zu bytes is too small", ws_bytes);
+  RouteSmallArgs a{};
+  a.x = x;
+  a.wr = w_router;
+  a.bias = bias;
+  a.T = T;
+  a.H = H;
+  a.E = E;
+  a.k = k;
+  a.ks = ks;
+  a.logits = logits;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.topk_logit = topk_logit;
+  a.offsets = offsets;
+  a.row_token = row_token;
+  a.slot_row = slot_row;
+  a.status = device_status_ptr();
+  const size_t w_bytes = size_t(kRouterEB) * H * 2;
+  const size_t p_bytes = (size_t(E) * ((T + 31) / 32) + E + 1) * 4;
+  const size_t smem = w_bytes > p_bytes ? w_bytes : p_bytes;
+  MOE_REQUIRE(smem <= 200 * 1024, MOE_ERR_UNSUPPORTED, "moe_route_permute: H=%d too large for the small-batch path",
+              H);
+  return dtype == MOE_DTYPE_BF16 ? dispatch_small<__nv_bfloat16>(a, smem, stream)
+                                 : dispatch_small<__half>(a, smem, stream);
+}
+
+}  // namespace moe

@@ -15,7 +15,8 @@ capture(x, fn)           records one pass (forward, or any callable over the
                          layer's buffers) into a CUDA graph bound to the
                          device buffer x; replaying the graph re-runs the
                          pass on whatever x then holds, without host work
-                         between the kernels
+                         between the kernels; graph_kernels then holds the
+                         number of kernel launches one replay makes
 """
 
 from __future__ import annotations
@@ -25,6 +26,21 @@ from typing import Dict, Optional
 import torch
 
 from . import abi
+
+
+def graph_kernel_nodes(g: "torch.cuda.CUDAGraph") -> int:
+    """Kernel nodes of a captured (not yet instantiated) graph: the launches
+    that one replay makes."""
+    from cuda.bindings import runtime as rt
+
+    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    err, nodes, n = rt.cudaGraphGetNodes(graph)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    if n and not nodes:
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes[:n]]
+    return sum(1 for t in kinds if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
 
 
 def prepare_nvfp4_weights(w: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
@@ -87,8 +103,8 @@ class MoELayer:
         self.y = torch.empty((T_max, H), dtype=self.adt, device=d)
         op = {"bf16": abi.MOE_OP_SWIGLU_BF16, "awq_g32": abi.MOE_OP_SWIGLU_AWQ_G32,
               "nvfp4": abi.MOE_OP_SWIGLU_NVFP4}[self.fmt]
-        self.ws_route = abi.workspace(abi.MOE_OP_ROUTE_TOPK, T_max, H, E, ks, 0, d)
-        self.ws_perm = abi.workspace(abi.MOE_OP_PERMUTE, T_max, H, E, ks, 0, d)
+        # route + permute in one call; the T_max workspace covers every T <= T_max
+        self.ws_route = abi.workspace(abi.MOE_OP_ROUTE_PERMUTE, T_max, H, E, ks, 0, d)
         self.ws_ffn = abi.workspace(op, T_max, H, E, ks, self.I, d)
         self.ws_sh = abi.workspace(abi.MOE_OP_SWIGLU_BF16, T_max, H, 1, 1, self.I_sh, d)
         if self.fmt == "bf16" and self.I_sh == self.I:
@@ -112,10 +128,9 @@ class MoELayer:
     def route(self, x: torch.Tensor):
         T = x.shape[0]
         ks = self.k + self.extra
-        abi.moe_route_topk(x, self.w["w_router"], self.w["bias"], self.k, self.extra, topk_idx=self.topk_idx[:T],
-                           topk_w=self.topk_w[:T], topk_logit=self.topk_logit[:T], ws=self.ws_route)
-        abi.moe_permute(self.topk_idx[:T], self.E, expert_offsets=self.offsets, row_token=self.row_token[:T * ks],
-                        slot_row=self.slot_row[:T], ws=self.ws_perm)
+        abi.moe_route_permute(x, self.w["w_router"], self.w["bias"], self.k, self.extra, topk_idx=self.topk_idx[:T],
+                              topk_w=self.topk_w[:T], topk_logit=self.topk_logit[:T], expert_offsets=self.offsets,
+                              row_token=self.row_token[:T * ks], slot_row=self.slot_row[:T], ws=self.ws_route)
 
     def experts(self, x: torch.Tensor) -> torch.Tensor:
         T = x.shape[0]
@@ -179,9 +194,11 @@ class MoELayer:
             for _ in range(warmup):
                 fn(x)
         torch.cuda.current_stream().wait_stream(s)
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(g):
             fn(x)
+        self.graph_kernels = graph_kernel_nodes(g)
+        g.instantiate()
         return g
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, x_dev: torch.Tensor) -> None:

@@ -82,7 +82,8 @@ enum {
   MOE_OP_SWIGLU_NVFP4 = 4,
   MOE_OP_REFILL = 5,
   MOE_OP_NVFP4_QUANTIZE = 6,
-  MOE_OP_EXPERTS_BF16 = 7
+  MOE_OP_EXPERTS_BF16 = 7,
+  MOE_OP_ROUTE_PERMUTE = 8
 };
 
 /* Version of this header's ABI. */
@@ -139,6 +140,21 @@ MOE_API int moe_route_topk(const void* x, int T, int H, const void* w_router, co
  * ------------------------------------------------------------------------- */
 MOE_API int moe_permute(const int32_t* topk_idx, int T, int k_slots, int E, int32_t* expert_offsets, int32_t* row_token,
                 int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_route_topk followed by moe_permute of its topk_idx (k_slots = k +
+ * extra), in one call, with the arguments and outputs of both.  For T <= 128
+ * (decode) everything runs in one cooperative kernel (grid-wide barriers
+ * between the logits, the top-k and the permutation); larger T takes the two
+ * calls' kernels in sequence.  Outputs equal those of the two calls, except
+ * that a near-tie among logits may resolve differently, as the logits are
+ * summed in another order.  Limits: those of both calls; for T <= 128 also
+ * 8 * H <= 204800 (the staged router rows).  Workspace: MOE_OP_ROUTE_PERMUTE.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_route_permute(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k,
+                              int extra, int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit,
+                              int32_t* expert_offsets, int32_t* row_token, int32_t* slot_row, void* ws,
+                              size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_permute without a workspace argument.  The pages have no counterpart:

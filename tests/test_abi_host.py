@@ -42,12 +42,20 @@ def test_route_rejects_bad_shapes(k, extra, E, H):
     rc = _code("moe_route_topk", None, 4, H, None, None, E, k, extra, 0, None, None, None, None, 0, None)
     assert rc in (abi.MOE_ERR_UNSUPPORTED, abi.MOE_ERR_INVALID_ARG)
     assert abi.load().moe_last_error().decode()
+    off = ctypes.c_void_p(256)  # never dereferenced: the shape check comes first
+    rc = _code("moe_route_permute", None, 4, H, None, None, E, k, extra, 0, None, None, None, off, None, None, None,
+               0, None)
+    assert rc in (abi.MOE_ERR_UNSUPPORTED, abi.MOE_ERR_INVALID_ARG)
 
 
 def test_calls_reject_null_pointers_and_bad_sizes():
     assert _code("moe_route_topk", None, 4, 256, None, None, 16, 2, 0, 0, None, None, None, None, 0, None) == \
         abi.MOE_ERR_INVALID_ARG
     assert _code("moe_permute", None, 4, 2, 2000, None, None, None, None, 0, None) == abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_route_permute", None, 4, 256, None, None, 16, 2, 0, 0, None, None, None, None, None, None, None,
+                 0, None) == abi.MOE_ERR_INVALID_ARG  # expert_offsets is null
+    assert _code("moe_route_permute", None, 4, 256, None, None, 16, 2, 0, 0, None, None, None, ctypes.c_void_p(256),
+                 None, None, None, 0, None) == abi.MOE_ERR_INVALID_ARG  # x is null
     assert _code("moe_permute", None, 4, 2, 16, None, None, None, None, 0, None) == abi.MOE_ERR_INVALID_ARG
     assert _code("moe_grouped_swiglu_bf16", None, None, None, 4, 8, 100, 64, 4, None, None, 0, 0, None, None, 0,
                  None) == abi.MOE_ERR_UNSUPPORTED

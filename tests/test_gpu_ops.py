@@ -180,3 +180,68 @@ def test_experts_routed_and_shared(T, H, I, E, k, out_fp32):
     sref, _ = moe.swiglu_expert(xs, sg[:I], sg[I:], f64(w["w_sh_down"]))
     err_sh = rel_err(f64(sh), sref)
     assert err_sh < 1e-2, err_sh
+
+
+ROUTE_PERMUTE_CASES = [
+    # T, H, E, k, extra, bias_std, act  (T <= 128: one cooperative kernel; T > 128: route then permute)
+    (1, 2048, 512, 10, 0, 1.5, "bf16"),
+    (7, 256, 16, 2, 0, 1.0, "bf16"),
+    (33, 512, 64, 4, 1, 1.0, "f16"),
+    (64, 2048, 512, 10, 1, 1.5, "bf16"),
+    (128, 2048, 512, 10, 0, 1.5, "bf16"),
+    (100, 256, 1000, 15, 1, 5.0, "bf16"),  # wide bias spread: 16 of 1000 still separates
+    (129, 512, 384, 10, 0, 1.5, "bf16"),
+    (300, 2048, 512, 10, 0, 1.5, "bf16"),
+]
+
+
+def _check_permutation_valid(gi, off, rt, sr, E):
+    """The permutation is a function of the selection: check it against the
+    selection it was built from (expert blocks ascending, tokens ascending
+    inside a block, every assignment's row pointing back at its token)."""
+    T, ks = gi.shape
+    counts = np.bincount(gi.ravel(), minlength=E) if T else np.zeros(E, np.int64)
+    assert np.array_equal(off, np.concatenate([[0], np.cumsum(counts)]))
+    for t in range(T):
+        for j in range(ks):
+            r = sr[t, j]
+            e = gi[t, j]
+            assert off[e] <= r < off[e + 1] and rt[r] == t
+    for e in range(E):
+        blk = rt[off[e]:off[e + 1]]
+        assert np.all(np.diff(blk) > 0)
+
+
+@pytest.mark.parametrize("T,H,E,k,extra,bstd,act", ROUTE_PERMUTE_CASES)
+def test_route_permute(T, H, E, k, extra, bstd, act):
+    wl = _wl(H=H, E=E, k=k, bias_std=bstd, act=act)
+    w = synth.make_weights(wl, seed=5, device=DEV)
+    x = synth.make_tokens(wl, T, seed=5, device=DEV)
+    idx, wt, lg, off, rt, sr = abi.moe_route_permute(x, w["w_router"], w["bias"], k, extra)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0
+    r = moe.route(f64(x), f64(w["w_router"]), f64(w["bias"]), k, extra)
+    ok = r["margin"] > 1e-3
+    gi = idx.cpu().numpy()
+    assert ok.mean() > 0.8
+    assert np.array_equal(gi[ok], r["idx"][ok])
+    assert np.allclose(wt.cpu().numpy()[ok], r["w"][ok], atol=2e-5, rtol=1e-4)
+    want_logit = np.take_along_axis(r["logits"], gi.astype(np.int64), 1)
+    assert np.allclose(lg.cpu().numpy(), want_logit, atol=2e-3, rtol=1e-4)
+    off_n, rt_n, sr_n = off.cpu().numpy(), rt.cpu().numpy(), sr.cpu().numpy()
+    _check_permutation_valid(gi, off_n, rt_n, sr_n, E)
+    if ok.all():  # the selection is unique: so is the permutation
+        want = moe.permute(r["idx"].astype(np.int64), E)
+        assert np.array_equal(off_n, want["offsets"])
+        assert np.array_equal(rt_n, want["row_token"])
+        assert np.array_equal(sr_n, want["slot_row"])
+
+
+def test_route_permute_empty_batch():
+    wl = _wl(H=256, E=16, k=2)
+    w = synth.make_weights(wl, seed=1, device=DEV)
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device=DEV)
+    off = torch.full((17,), -7, dtype=torch.int32, device=DEV)
+    abi.moe_route_permute(x, w["w_router"], w["bias"], 2, expert_offsets=off)
+    torch.cuda.synchronize()
+    assert off.cpu().tolist() == [0] * 17
