@@ -40,6 +40,10 @@ int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scale
                 cudaStream_t stream);
 size_t nvfp4_quant_ws_bytes(int batch, int rows, int K);
 size_t decode_ws_bytes(int rows, int T, int I);
+size_t decode_fused_ws_bytes(int rows, int T, int H, int I);
+int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
+                         int E, const void* w_gu, const void* w_d, const void* w_sh_gu, const void* w_sh_d, int dtype,
+                         int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, cudaStream_t stream);
 int decode_experts_16bit(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
                          int E, const void* w_gu, const void* w_d, const void* w_sh_gu, const void* w_sh_d, int dtype,
                          int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -206,9 +210,22 @@ static int dense_swiglu(const void* x, int T, int H, int I, const void* w_gu, co
 }
 
 static constexpr int kDecodeMaxT = 128;
+static constexpr int kFusedMaxT = 16;
+
+// The one-kernel split-K path for T <= 16; BIT_EXPERT_GEMM_DECODE_FUSED=0
+// selects the two-GEMM decode path instead (for comparisons).
+static bool fused_decode_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* s = getenv("BIT_EXPERT_GEMM_DECODE_FUSED");
+    on = (s && s[0] == '0') ? 0 : 1;
+  }
+  return on != 0;
+}
 
 static size_t experts_ws_bytes(int T, int rows, int H, int I) {
   (void)H;
+  if (T <= kFusedMaxT && fused_decode_enabled()) return decode_fused_ws_bytes(rows, T, H, I);
   if (T <= kDecodeMaxT) return decode_ws_bytes(rows, T, I);
   WsCounter c;
   c.take<uint16_t>(size_t(rows > T ? rows : T) * I);
@@ -348,6 +365,9 @@ int moe_experts_bf16(const void* x, const int32_t* row_token, const int32_t* exp
               "moe_experts_bf16: workspace of %zu bytes is too small (need %zu)", ws_bytes,
               experts_ws_bytes(T, rows, H, I));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T <= kFusedMaxT && fused_decode_enabled())
+    return decode_experts_fused(x, row_token, expert_offsets, T, rows, H, I, E, w_gate_up, w_down, w_sh_gate_up,
+                                w_sh_down, dtype, out_fp32, f, shared_out, ws, ws_bytes, st);
   if (T <= kDecodeMaxT)
     return decode_experts_16bit(x, row_token, expert_offsets, T, rows, H, I, E, w_gate_up, w_down, w_sh_gate_up,
                                 w_sh_down, dtype, out_fp32, f, shared_out, ws, ws_bytes, st);

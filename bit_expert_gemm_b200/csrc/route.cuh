@@ -18,9 +18,10 @@ namespace moe {
 constexpr int kRouterEB = 4;  // experts per block of the small-batch logits kernel
 
 // Logits of experts [e0, e0 + kRouterEB) for every token.  The block's weight
-// rows are staged in shared memory (w_sh: kRouterEB * H 16-bit values); warp
-// w then takes tokens w, w + nwarps, ...: its lanes stride over H in 8-value
-// chunks keeping one partial sum per expert, reduced across the warp at the
+// rows are staged in shared memory with cp.async (w_sh: kRouterEB * H 16-bit
+// values); warp w then takes tokens w, w + nwarps, ...: its lanes stride over
+// H in 8-value chunks, with up to 8 chunks of the token row in flight at
+// once, keeping one partial sum per expert, reduced across the warp at the
 // end.  Every thread of the block must call this.
 template <typename T16>
 __device__ void router_block_logits(const T16* __restrict__ x, const T16* __restrict__ wr,
@@ -29,30 +30,44 @@ __device__ void router_block_logits(const T16* __restrict__ x, const T16* __rest
   const int nchunk = H / 8;
   const int ne = min(kRouterEB, E - e0);
   const uint4* src = reinterpret_cast<const uint4*>(wr + size_t(e0) * H);
-  for (int i = threadIdx.x; i < ne * nchunk; i += blockDim.x) w_sh[i] = __ldg(src + i);
+  for (int i = threadIdx.x; i < ne * nchunk; i += blockDim.x)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(w_sh + i)), "l"(src + i) : "memory");
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  constexpr int U = 8;  // chunks of the token row per lane in flight
   for (int t = warp; t < T; t += nw) {
     const uint4* xr = reinterpret_cast<const uint4*>(x + size_t(t) * H);
     float acc[kRouterEB];
 #pragma unroll
     for (int e = 0; e < kRouterEB; ++e) acc[e] = 0.0f;
-    for (int c = lane; c < nchunk; c += 32) {
-      const uint4 xv = __ldg(xr + c);
-      const uint32_t* xp = reinterpret_cast<const uint32_t*>(&xv);
-      float2 xf[4];
+    for (int c0 = lane; c0 < nchunk; c0 += 32 * U) {
+      uint4 xv[U];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xf[i] = Pack2<T16>::unpack(xp[i]);
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        xv[u] = c < nchunk ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-      for (int e = 0; e < kRouterEB; ++e) {
-        if (e < ne) {
-          const uint4 wv = w_sh[e * nchunk + c];
-          const uint32_t* wp = reinterpret_cast<const uint32_t*>(&wv);
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < nchunk) {
+          const uint32_t* xp = reinterpret_cast<const uint32_t*>(&xv[u]);
+          float2 xf[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 wf = Pack2<T16>::unpack(wp[i]);
-            acc[e] = fmaf(wf.x, xf[i].x, acc[e]);
-            acc[e] = fmaf(wf.y, xf[i].y, acc[e]);
+          for (int i = 0; i < 4; ++i) xf[i] = Pack2<T16>::unpack(xp[i]);
+#pragma unroll
+          for (int e = 0; e < kRouterEB; ++e) {
+            if (e < ne) {
+              const uint4 wv = w_sh[e * nchunk + c];
+              const uint32_t* wp = reinterpret_cast<const uint32_t*>(&wv);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 wf = Pack2<T16>::unpack(wp[i]);
+                acc[e] = fmaf(wf.x, xf[i].x, acc[e]);
+                acc[e] = fmaf(wf.y, xf[i].y, acc[e]);
+              }
+            }
           }
         }
       }
@@ -69,56 +84,60 @@ __device__ void router_block_logits(const T16* __restrict__ x, const T16* __rest
   __syncthreads();  // w_sh is refilled by the caller's next block
 }
 
+// Order-preserving map of a float to an unsigned key (a < b <=> key(a) <
+// key(b) for non-NaN values; -0 is made +0 first so that it ties with +0).
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // Top-(k + extra) of one token's logits by one warp: each lane holds E/32
-// values (NV per lane, E <= 32 * NV); ks rounds of a warp arg-max with ties
-// to the lower index; NaN never wins.  Lane r keeps the r-th selection and
-// writes idx_out[r], logit_out[r] (if not null) and, for r < k, the
-// renormalised weight w_out[r].  `row` is read through L2 (it may have been
-// written by other blocks of the same kernel).
+// values (NV per lane, E <= 32 * NV) as order keys; each of the ks rounds
+// takes the lane's best remaining key, then a warp max of the keys and a warp
+// min of the indices holding that max (ties to the lower expert index), two
+// redux.sync instructions.  NaN counts as -FLT_MAX; absent and selected
+// values have key 0, below every real value.  Lane r keeps the r-th
+// selection and writes idx_out[r], logit_out[r] (if not null) and, for r < k,
+// the renormalised weight w_out[r].  `row` is read through L2 (it may have
+// been written by other blocks of the same kernel).
 template <int NV>
 __device__ __forceinline__ void topk_token(const float* row, int E, int k, int ks, int lane, int32_t* idx_out,
                                            float* w_out, float* logit_out) {
-  float v[NV];
+  uint32_t key[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int e = lane + 32 * i;
-    const float x = e < E ? __ldcg(row + e) : -FLT_MAX;
-    v[i] = (x != x) ? -FLT_MAX : x;
+    float x = e < E ? __ldcg(row + e) : -FLT_MAX;
+    x = (x != x) ? -FLT_MAX : x;
+    key[i] = e < E ? order_key(x) : 0u;
   }
-  uint32_t removed = 0;  // bit i: value i of this lane already selected (or absent)
-#pragma unroll
-  for (int i = 0; i < NV; ++i)
-    if (lane + 32 * i >= E) removed |= 1u << i;
-  float my_v = 0.0f, top = 0.0f;
+  uint32_t my_key = 0, top_key = 0;
   int my_i = 0;
 #pragma unroll 1
   for (int r = 0; r < ks; ++r) {
-    float bv = -FLT_MAX;
-    int bi = 0x7fffffff;
+    uint32_t bk = 0;
+    uint32_t bi = 0xffffffffu;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int e = lane + 32 * i;
-      if (!(removed >> i & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
-        bv = v[i];
-        bi = e;
+    for (int i = 0; i < NV; ++i)
+      if (key[i] > bk) {
+        bk = key[i];
+        bi = uint32_t(lane + 32 * i);
       }
-    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t win = __reduce_min_sync(0xffffffffu, bk == m ? bi : 0xffffffffu);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if ((bi & 31) == lane) removed |= 1u << (bi >> 5);
+    for (int i = 0; i < NV; ++i)
+      if (uint32_t(lane + 32 * i) == win) key[i] = 0;
     if (lane == r) {
-      my_v = bv;
-      my_i = bi;
+      my_key = m;
+      my_i = int(win);
     }
-    if (r == 0) top = bv;
+    if (r == 0) top_key = m;
   }
+  const float my_v = key_value(my_key), top = key_value(top_key);
   // renormalised softmax over the k selected experts (max-shifted)
   const float p = lane < k ? __expf(my_v - top) : 0.0f;
   float z = p;

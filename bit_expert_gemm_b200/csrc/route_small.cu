@@ -4,7 +4,8 @@
 // barriers:
 //   1. logits: every block computes kRouterEB experts' logits for all tokens
 //      (router rows read from HBM once);
-//   2. top-k and renormalised weights: one warp per token;
+//   2. top-k and renormalised weights: one warp per token (all in block 0
+//      when T <= 8, which then needs no second grid barrier);
 //   3. permutation, by block 0 alone: each expert's tokens as a bitmask in
 //      shared memory (T <= 128: at most four words per expert), counts by
 //      popcount, exclusive scan into expert_offsets, and every assignment's
@@ -63,13 +64,23 @@ __global__ void __launch_bounds__(kThreads) k_route_permute_small(const RouteSma
     router_block_logits<T16>(static_cast<const T16*>(a.x), static_cast<const T16*>(a.wr), a.bias, T, a.H, E,
                              eb * kRouterEB, reinterpret_cast<uint4*>(smem), a.logits);
   grid.sync();
-  // 2. top-k
+  // 2. top-k: by block 0 alone when every token has a warp of its own there
+  // (then the permutation follows after a block barrier), else by all blocks
+  // with a second grid barrier
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t = blockIdx.x * (kThreads / 32) + warp; t < T; t += gridDim.x * (kThreads / 32))
+  const bool solo = T <= kThreads / 32;
+  if (solo && blockIdx.x != 0) return;
+  const int t_first = solo ? warp : blockIdx.x * (kThreads / 32) + warp;
+  const int t_step = solo ? kThreads / 32 : gridDim.x * (kThreads / 32);
+  for (int t = t_first; t < T; t += t_step)
     topk_token<NV>(a.logits + size_t(t) * E, E, a.k, ks, lane, a.topk_idx + size_t(t) * ks,
                    a.topk_w + size_t(t) * a.k, a.topk_logit ? a.topk_logit + size_t(t) * ks : nullptr);
-  grid.sync();
-  if (blockIdx.x != 0) return;
+  if (solo) {
+    __syncthreads();
+  } else {
+    grid.sync();
+    if (blockIdx.x != 0) return;
+  }
   // 3. permutation (block 0)
   const int W = (T + 31) / 32;
   uint32_t* mask = reinterpret_cast<uint32_t*>(smem);  // [E, W]

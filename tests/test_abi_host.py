@@ -27,6 +27,8 @@ def test_workspace_sizes():
     # routed + shared experts: h [rows, I] for prefill, h [rows + T, I] (shared rows appended) for decode
     assert lib.moe_workspace_size(abi.MOE_OP_EXPERTS_BF16, 8192, 2048, 512, 10, 640) >= 81920 * 640 * 2
     assert lib.moe_workspace_size(abi.MOE_OP_EXPERTS_BF16, 64, 2048, 512, 10, 640) >= (640 + 64) * 640 * 2  # 16-bit h
+    # T <= 16: FP32 split-K partials [I/64][rows + T][H]
+    assert lib.moe_workspace_size(abi.MOE_OP_EXPERTS_BF16, 1, 2048, 512, 10, 640) >= 10 * 11 * 2048 * 4
     assert lib.moe_workspace_size(abi.MOE_OP_PERMUTE, 32768, 2048, 512, 11, 640) >= 512 * 1024 * 8
     assert lib.moe_workspace_size(99, 1, 1, 1, 1, 1) == 0
     assert lib.moe_workspace_size(abi.MOE_OP_ROUTE_TOPK, -1, 1, 1, 1, 1) == 0

@@ -155,14 +155,22 @@ def test_select_bit_exact(E):
             assert np.array_equal(kept.cpu().numpy(), k_ref)
 
 
-@pytest.mark.parametrize("T,H,I,E,k,out_fp32", [(1, 2048, 640, 512, 10, False), (8, 512, 128, 16, 4, False),
-                                                (64, 2048, 640, 64, 10, True), (128, 256, 64, 16, 2, False),
-                                                (300, 512, 128, 8, 3, False)])
-def test_experts_routed_and_shared(T, H, I, E, k, out_fp32):
-    """moe_experts_bf16: the decode path (T <= 128: weight-streaming GEMMs with
-    the shared expert as one more group) and the prefill path (T > 128)."""
-    wl = _wl(H=H, I=I, I_sh=I, E=E, k=k)
+@pytest.mark.parametrize("T,H,I,E,k,out_fp32,act", [
+    # T <= 16: one split-K kernel + partial sums
+    (1, 2048, 640, 512, 10, False, "bf16"), (8, 512, 128, 16, 4, False, "bf16"), (3, 256, 64, 16, 2, False, "bf16"),
+    (16, 1024, 192, 64, 6, True, "bf16"), (5, 384, 128, 32, 4, False, "f16"),
+    # 16 < T <= 128: two weight-streaming GEMMs
+    (17, 512, 128, 16, 3, False, "bf16"), (64, 2048, 640, 64, 10, True, "bf16"), (128, 256, 64, 16, 2, False, "bf16"),
+    # T > 128: the grouped prefill GEMMs
+    (300, 512, 128, 8, 3, False, "bf16")])
+def test_experts_routed_and_shared(T, H, I, E, k, out_fp32, act):
+    """moe_experts_bf16 on all three of its paths, routed rows and the shared
+    expert against the oracle."""
+    wl = _wl(H=H, I=I, I_sh=I, E=E, k=k, act=act)
     w = synth.make_weights(wl, seed=T + 7, device=DEV)
+    if act == "f16":
+        for key in ("w_gate_up", "w_down", "w_sh_gate_up", "w_sh_down"):
+            w[key] = w[key].to(torch.float16)
     x = synth.make_tokens(wl, T, seed=T + 7, device=DEV)
     idx = synth.make_routing(T, E, k, seed=T + 8)
     off, rt, sr = abi.moe_permute(idx.to(DEV), E)
