@@ -42,8 +42,8 @@ constexpr int KSUB = 2;                    // sub-tiles per pipeline stage
 constexpr int STAGE_BYTES = KSUB * SUB_BYTES;
 constexpr int STAGES = 5;
 constexpr int H_BYTES = NT * BK * 2;       // one h tile: 16 rows x 64 features
-constexpr int XS = NT + 1;                 // floats per row of the gate/up exchange (bank padding)
-constexpr int XCHG_BYTES = 64 * XS * 4;
+constexpr int XS = NT + 1;                 // floats per row of the accumulator exchange (bank padding)
+constexpr int XCHG_BYTES = BM * XS * 4;    // all 128 phase-A rows (64 gate, 64 up)
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * H_BYTES + XCHG_BYTES;
 constexpr int kThreads = 320;
 constexpr uint32_t TMEM_COLS = 512;
@@ -295,9 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 6) {
     // ---------------- epilogue ----------------
-    // TMEM lane quadrant q: in phase A q = 0, 1 hold gate features, q = 2, 3
-    // the up features of the same 64 intermediate features; in phase B lane
-    // = down-projection row (output feature) m*128 + q*32 + lane.
+    // TMEM lane quadrant q: in phase A lanes 0..63 hold the gate rows, 64..127
+    // the up rows of the same 64 intermediate features; in phase B lane =
+    // down-projection row (output feature) m*128 + q*32 + lane.
     const int q = warp & 3;
     const int R = args.rows + args.T;
     int n = 0;
@@ -319,20 +319,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld16(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(a * NT), v);
       tc_fence_before();
       mbar_arrive(&accA_empty[a]);
-      if (q >= 2) {
+      // rows 0..63 gate, 64..127 up pre-activations of the block's 64 features
 #pragma unroll
-        for (int c = 0; c < NT; ++c) xchg[((q - 2) * 32 + lane) * XS + c] = v[c];
-      }
+      for (int c = 0; c < NT; ++c) xchg[(q * 32 + lane) * XS + c] = v[c];
       epilogue_sync();
-      if (q < 2) {
-        // h[c][f] for feature f of the block, 16-bit, K-major 128-byte swizzled:
-        // row c at c*128 bytes, 16-byte chunk (f/8) xor (c%8), element f%8
-        const int f = q * 32 + lane;
+      {
+        // h[c][f] = silu(gate[f][c]) * up[f][c], 16-bit, K-major 128-byte
+        // swizzled: row c at c*128 bytes, 16-byte chunk (f/8) xor (c%8),
+        // element f%8.  1024 values over the 128 threads, in a rolled loop
+        // (this code runs once per item: compact code stays cached).
+        const int et = threadIdx.x - 64;
         uint8_t* ht = htile + a * H_BYTES;
-#pragma unroll
-        for (int c = 0; c < NT; ++c) {
-          const float h = silu_f(v[c]) * xchg[f * XS + c];
-          const uint32_t off = uint32_t(c * 128 + ((((f >> 3) ^ (c & 7))) << 4) + (f & 7) * 2);
+#pragma unroll 1
+        for (int idx = et; idx < 64 * NT; idx += 128) {
+          const int f = idx & 63, c = idx >> 6;
+          const float h = silu_f(xchg[f * XS + c]) * xchg[(64 + f) * XS + c];
+          const uint32_t off = uint32_t(c * 128 + (((f >> 3) ^ (c & 7)) << 4) + (f & 7) * 2);
           if (args.bf16)
             *reinterpret_cast<__nv_bfloat16*>(ht + off) = __float2bfloat16_rn(h);
           else
@@ -341,17 +343,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();  // the h tile is read by the tensor cores
       mbar_arrive(&h_full[a]);
-      epilogue_sync();           // the gate warps have read xchg before the next item overwrites it
+      epilogue_sync();           // every thread has read xchg before the next item overwrites it
       // phase B: FP32 partials of the group's rows
       if (!epilogue_all(mbar_wait(&accB_full, uint32_t(n & 1), &abort_flag, status, lim))) break;
       tc_fence_after();
       float* P = args.partial + (size_t(j) * R + r0) * args.H;
-      for (int m = 0; m < MB2; ++m) {
-        tmem_ld16(tmem_base + (uint32_t(q * 32) << 16) + ACCB_COL + uint32_t(m * NT), v);
-        const int feat = m * BM + q * 32 + lane;
+      // four blocks' accumulators (64 consecutive columns) per TMEM load wait
+      for (int m0 = 0; m0 < MB2; m0 += 4) {
+        float w0[32], w1[32];
+        const uint32_t ta = tmem_base + (uint32_t(q * 32) << 16) + ACCB_COL + uint32_t(m0 * NT);
+        tmem_ld32x2(ta, ta + 32, w0, w1);
 #pragma unroll
-        for (int c = 0; c < NT; ++c)
-          if (c < nn) P[size_t(c) * args.H + feat] = v[c];
+        for (int u = 0; u < 4; ++u) {
+          if (m0 + u < MB2) {
+            const int feat = (m0 + u) * BM + q * 32 + lane;
+#pragma unroll
+            for (int c = 0; c < NT; ++c) {
+              const float val = u < 2 ? w0[u * NT + c] : w1[(u - 2) * NT + c];
+              if (c < nn) P[size_t(c) * args.H + feat] = val;
+            }
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(&accB_empty);
