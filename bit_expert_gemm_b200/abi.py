@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 MOE_DTYPE_BF16, MOE_DTYPE_F16 = 0, 1
 (MOE_OP_ROUTE_TOPK, MOE_OP_PERMUTE, MOE_OP_SWIGLU_BF16, MOE_OP_SWIGLU_AWQ_G32, MOE_OP_SWIGLU_NVFP4, MOE_OP_REFILL,
- MOE_OP_NVFP4_QUANTIZE, MOE_OP_EXPERTS_BF16, MOE_OP_ROUTE_PERMUTE) = range(9)
+ MOE_OP_NVFP4_QUANTIZE, MOE_OP_EXPERTS_BF16, MOE_OP_ROUTE_PERMUTE, MOE_OP_EXPERTS_AWQ_G32) = range(10)
 
 
 class MoEError(RuntimeError):
@@ -50,6 +50,8 @@ _SIGS = {
     "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_grouped_swiglu_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _SZ, _P]),
     "moe_experts_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
+    "moe_experts_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P,
+                                 _SZ, _P]),
     "moe_grouped_swiglu_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "moe_awq_dequant_g32": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_nvfp4_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -251,6 +253,26 @@ def moe_experts_bf16(x, row_token, expert_offsets, rows: int, w_gate_up, w_down,
     _call("moe_experts_bf16", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E, _p(w_gate_up), _p(w_down),
           _p(w_sh_gate_up), _p(w_sh_down), _dtype_code(x), int(out_fp32), _p(f), _p(shared_out), _p(ws), ws.numel(),
           _stream(stream))
+    return f, shared_out
+
+
+def moe_experts_awq_g32(x, row_token, expert_offsets, rows: int, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d, w_sh_gate_up,
+                        w_sh_down, out_fp32: bool = False, f=None, shared_out=None, ws=None, stream=None):
+    """Routed AWQ experts (f [rows, H]) and the FP16 shared expert (shared_out [T, H]) in one call."""
+    T, H = x.shape
+    E = qw_gu.shape[0]
+    I = qw_gu.shape[2] * 8 // 2
+    dev = x.device
+    _need(x, torch.float16, "x")
+    if f is None:
+        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else torch.float16, device=dev)
+    if shared_out is None:
+        shared_out = torch.empty((T, H), dtype=torch.float16, device=dev)
+    if ws is None:
+        ws = workspace(MOE_OP_EXPERTS_AWQ_G32, T, H, E, max(1, rows // max(T, 1)), I, dev)
+    _call("moe_experts_awq_g32", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E, _p(qw_gu), _p(qz_gu),
+          _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), _p(w_sh_gate_up), _p(w_sh_down), int(out_fp32), _p(f),
+          _p(shared_out), _p(ws), ws.numel(), _stream(stream))
     return f, shared_out
 
 

@@ -41,6 +41,11 @@ int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scale
 size_t nvfp4_quant_ws_bytes(int batch, int rows, int K);
 size_t decode_ws_bytes(int rows, int T, int I);
 size_t decode_fused_ws_bytes(int rows, int T, int H, int I);
+int decode_experts_fused_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
+                             int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
+                             const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gu,
+                             const void* w_sh_d, int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
+                             cudaStream_t stream);
 int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
                          int E, const void* w_gu, const void* w_d, const void* w_sh_gu, const void* w_sh_d, int dtype,
                          int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -223,6 +228,15 @@ static bool fused_decode_enabled() {
   return on != 0;
 }
 
+// AWQ routed + 16-bit shared experts: the split-K partials for T <= 16, else
+// the grouped AWQ call's workspace, reused afterwards by the shared expert's h.
+static size_t experts_awq_ws_bytes(int T, int rows, int H, int I, int E) {
+  if (T <= kFusedMaxT && fused_decode_enabled()) return decode_fused_ws_bytes(rows, T, H, I);
+  const size_t a = awq_ws_bytes(rows, H, I, E);
+  const size_t b = size_t(T) * I * 2;
+  return a > b ? a : b;
+}
+
 static size_t experts_ws_bytes(int T, int rows, int H, int I) {
   (void)H;
   if (T <= kFusedMaxT && fused_decode_enabled()) return decode_fused_ws_bytes(rows, T, H, I);
@@ -267,6 +281,7 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k_slots, int I) {
     }
     case MOE_OP_SWIGLU_AWQ_G32: return awq_ws_bytes(rows, H, I, E);
     case MOE_OP_EXPERTS_BF16: return experts_ws_bytes(T, rows, H, I);
+    case MOE_OP_EXPERTS_AWQ_G32: return experts_awq_ws_bytes(T, rows, H, I, E);
     case MOE_OP_SWIGLU_NVFP4: return nvfp4_ws_bytes(rows, H, I, E);
     case MOE_OP_REFILL: return refill_ws_bytes(T, k_slots > 0 ? k_slots - 1 : 0);
     case MOE_OP_NVFP4_QUANTIZE: return nvfp4_quant_ws_bytes(1, T, H);
@@ -378,6 +393,39 @@ int moe_experts_bf16(const void* x, const int32_t* row_token, const int32_t* exp
     if (rc) return rc;
   }
   return dense_swiglu(x, T, H, I, w_sh_gate_up, w_sh_down, dtype, shared_out, static_cast<uint16_t*>(ws), st);
+}
+
+int moe_experts_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows, int H,
+                        int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
+                        const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gate_up,
+                        const void* w_sh_down, int out_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
+                        void* stream) {
+  MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG,
+              "moe_experts_awq_g32: bad sizes");
+  MOE_REQUIRE(H > 0 && I > 0 && H % 128 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_experts_awq_g32: need H %% 128 == 0 and I %% 64 == 0 (H=%d I=%d)", H, I);
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(x && row_token && expert_offsets && qw_gu && qz_gu && sc_gu && qw_d && qz_d && sc_d && w_sh_gate_up &&
+                  w_sh_down && f && shared_out,
+              MOE_ERR_INVALID_ARG, "moe_experts_awq_g32: null pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(qw_gu) && aligned16(qz_gu) && aligned16(sc_gu) && aligned16(qw_d) &&
+                  aligned16(qz_d) && aligned16(sc_d) && aligned16(w_sh_gate_up) && aligned16(w_sh_down) &&
+                  aligned16(f) && aligned16(shared_out),
+              MOE_ERR_INVALID_ARG, "moe_experts_awq_g32: operands must be 16-byte aligned");
+  MOE_REQUIRE(ws_bytes >= experts_awq_ws_bytes(T, rows, H, I, E), MOE_ERR_WORKSPACE,
+              "moe_experts_awq_g32: workspace of %zu bytes is too small (need %zu)", ws_bytes,
+              experts_awq_ws_bytes(T, rows, H, I, E));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T <= kFusedMaxT && fused_decode_enabled())
+    return decode_experts_fused_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d,
+                                    sc_d, w_sh_gate_up, w_sh_down, out_fp32, f, shared_out, ws, ws_bytes, st);
+  int rc = MOE_OK;
+  if (rows > 0) {
+    rc = grouped_swiglu_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
+                            out_fp32, f, ws, ws_bytes, st);
+    if (rc) return rc;
+  }
+  return dense_swiglu(x, T, H, I, w_sh_gate_up, w_sh_down, MOE_DTYPE_F16, shared_out, static_cast<uint16_t*>(ws), st);
 }
 
 int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,

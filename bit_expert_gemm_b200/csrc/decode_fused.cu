@@ -9,7 +9,7 @@
 //     of the group's rows written into a shared-memory tile in the operand
 //     layout of the next MMA.
 //   Phase B: that h slice times the matching 64 columns of the group's down
-//     projection (H x 64, as 16 blocks of 128 rows): a split-K slice of the
+//     projection (H x 64, as blocks of 128 rows): a split-K slice of the
 //     second GEMM, whose FP32 result is the partial P[j][row][0..H).
 // Phase B's weights do not depend on h, so they stream right behind phase
 // A's and the whole call is one stream of weights through every SM, with no
@@ -17,16 +17,30 @@
 // every row in a fixed order (deterministic) into f (routed rows) and
 // shared_out (shared rows).
 //
-// Warp roles: 0 TMA producer (weights), 1 UMMA issuer (TMEM owner), 2..5
-// epilogue, 6..9 token gather (cp.async, arriving on the stage's barrier).
-// TMEM: two 16-column phase-A accumulators (columns 0..31) and one phase-B
-// accumulator of H/128 blocks x 16 columns (from column 32).
+// Weight formats (template parameter WQ):
+//   WQ = 0: 16-bit routed and shared weights, output-major [N, K]; each
+//     64-wide K sub-tile of 128 weight rows arrives by TMA in the K-major
+//     128-byte swizzled layout the MMA reads.
+//   WQ = 1: routed experts in AWQ W4A16 g32 (input-major codes, zero points
+//     and FP16 scales, FP16 activations), the shared expert 16-bit as above.
+//     The producer stages each routed sub-tile's codes, scales and zero
+//     points (4.6 KB instead of 16 KB of FP16); four dequantisation warps
+//     expand it, exactly (fp16_rn((q - z) * s)), into an MN-major swizzled
+//     FP16 tile, and the MMA reads that.
+//
+// Warp roles: 0 TMA producer, 1 UMMA issuer (TMEM owner), 2..5 epilogue,
+// 6..9 token gather (cp.async, arriving on the stage's barrier), 10..13 AWQ
+// dequantisation (WQ = 1).  TMEM: two 16-column phase-A accumulators
+// (columns 0..31) and one phase-B accumulator of H/128 blocks x 16 columns
+// (from column 32).
 #include "common.cuh"
 #include "gemm_sm100.cuh"
 
 namespace moe {
 
 int make_tmap_16bit_sw128(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
+int make_tmap_2d(CUtensorMap* map, const void* base, int rows, int cols, int esize, int box_rows, int box_cols,
+                 CUtensorMapSwizzle swz);
 
 constexpr int kFusedMaxT = 16;
 
@@ -35,22 +49,42 @@ namespace {
 constexpr int BM = 128;                    // weight rows per MMA (M)
 constexpr int BK = 64;                     // K per sub-tile (one 128-byte swizzle row)
 constexpr int NT = 16;                     // token columns (N) of every MMA
-constexpr int A_BYTES = BM * BK * 2;       // 16 KB of weights per sub-tile
+constexpr int A_BYTES = BM * BK * 2;       // 16 KB of 16-bit weights per sub-tile
 constexpr int B_BYTES = NT * BK * 2;       // 2 KB of tokens per sub-tile
-constexpr int SUB_BYTES = A_BYTES + B_BYTES;
 constexpr int KSUB = 2;                    // sub-tiles per pipeline stage
-constexpr int STAGE_BYTES = KSUB * SUB_BYTES;
-constexpr int STAGES = 5;
 constexpr int H_BYTES = NT * BK * 2;       // one h tile: 16 rows x 64 features
 constexpr int XS = NT + 1;                 // floats per row of the accumulator exchange (bank padding)
 constexpr int XCHG_BYTES = BM * XS * 4;    // all 128 phase-A rows (64 gate, 64 up)
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * H_BYTES + XCHG_BYTES;
-constexpr int kThreads = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACCB_COL = 32;
 constexpr int FULL_ARRIVALS = 1 + 128;     // producer (with the TMA bytes) + one per gather thread
-static_assert(SUB_BYTES % 1024 == 0 && H_BYTES % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-static_assert(SMEM_BYTES <= 222 * 1024, "shared memory");
+// AWQ staging inside a sub-tile, after the FP16 weight tile and the token
+// tile: codes [64 K rows][16 words] (phase A: gate box [64][8] then up box
+// [64][8]; phase B: one box [64][16]), scales [2 groups][128] FP16 (phase A:
+// two boxes [2][64]), zero points [2 groups][16 words] (phase A: two boxes
+// [2][8], each in a 128-byte slot).  Every box starts on 128 bytes.
+constexpr int Q_CODES = A_BYTES + B_BYTES;
+constexpr int Q_SCALES = Q_CODES + 64 * 16 * 4;
+constexpr int Q_ZEROS = Q_SCALES + 2 * 128 * 2;
+constexpr int Q_END = Q_ZEROS + 2 * 128;
+constexpr uint32_t Q_TX = 64 * 16 * 4 + 2 * 128 * 2 + 2 * 16 * 4;  // bytes the TMA brings per AWQ sub-tile
+// MN-major FP16 weight tile (AWQ): 64-element atoms along M are LBO apart,
+// 8-row K groups SBO apart; one MMA (K = 16) spans two K groups
+constexpr uint32_t AQ_LBO = (BK / 8) * 1024;
+constexpr uint32_t AQ_SBO = 1024;
+constexpr int kDequantThreads = 128;
+
+template <int WQ>
+struct FusedCfg {
+  static constexpr int SUB_BYTES = WQ ? (Q_END + 1023) / 1024 * 1024 : A_BYTES + B_BYTES;
+  static constexpr int STAGE_BYTES = KSUB * SUB_BYTES;
+  static constexpr int STAGES = WQ ? 4 : 5;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * H_BYTES + XCHG_BYTES;
+  static constexpr int THREADS = 320 + (WQ ? kDequantThreads : 0);
+  static_assert(SUB_BYTES % 1024 == 0 && H_BYTES % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(SMEM_BYTES <= 222 * 1024, "shared memory");
+};
+static_assert(Q_CODES % 1024 == 0 && Q_SCALES % 128 == 0 && Q_ZEROS % 128 == 0, "TMA destinations");
 
 struct Args {
   const int* offsets;   // [E+1] routed expert offsets (device)
@@ -61,6 +95,14 @@ struct Args {
   int bf16;
   int* status;
   unsigned long long limit_ns;
+};
+
+// Tensor maps.  16-bit weights: gu (routed gate/up [E*2I, H], box 64 rows),
+// d (routed down [E*H, I], box 128 rows), and the shared expert's sgu, sd.
+// AWQ (WQ = 1) replaces gu and d by codes / scales / zero points.
+struct Maps {
+  CUtensorMap gu, d, sgu, sd;
+  CUtensorMap qc_gu, qs_gu, qz_gu, qc_d, qs_d, qz_d;
 };
 
 __device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -84,22 +126,24 @@ __device__ __forceinline__ bool epilogue_all(bool v) {
   return r != 0;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    k_decode_ffn(const __grid_constant__ CUtensorMap tmGU, const __grid_constant__ CUtensorMap tmGUs,
-                 const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmDs, const Args args) {
+template <int WQ>
+__global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
+    k_decode_ffn(const __grid_constant__ Maps maps, const Args args) {
+  using Cfg = FusedCfg<WQ>;
+  constexpr int STAGES = Cfg::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], accA_full[2], accA_empty[2], h_full[2],
-      h_empty[2], accB_full, accB_empty, drain_bar;
+  __shared__ __align__(8) uint64_t full_bar[STAGES], aready_bar[STAGES], empty_bar[STAGES], accA_full[2],
+      accA_empty[2], h_full[2], h_empty[2], accB_full, accB_empty, drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ int goff[kGemmMaxGroups + 2];
   __shared__ int item_start[kGemmMaxGroups + 2];
-  __shared__ int warp_sums[kThreads / 32];
+  __shared__ int warp_sums[Cfg::THREADS / 32];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // sub-tile u of stage s: weights at sub(s, u), tokens at sub(s, u) + A_BYTES
-  auto sub = [&](int s, int u) { return smem + s * STAGE_BYTES + u * SUB_BYTES; };
-  uint8_t* htile = smem + STAGES * STAGE_BYTES;  // two h tiles of H_BYTES
+  // sub-tile u of stage s: weights at sub(s, u), tokens at + A_BYTES, AWQ staging at + Q_CODES ...
+  auto sub = [&](int s, int u) { return smem + s * Cfg::STAGE_BYTES + u * Cfg::SUB_BYTES; };
+  uint8_t* htile = smem + STAGES * Cfg::STAGE_BYTES;  // two h tiles of H_BYTES
   float* xchg = reinterpret_cast<float*>(htile + 2 * H_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = args.E, G = E + 1;
@@ -112,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], FULL_ARRIVALS);
+      mbar_init(&aready_bar[s], kDequantThreads);
       mbar_init(&empty_bar[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -127,10 +172,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmGU);
-    tma_prefetch_desc(&tmGUs);
-    tma_prefetch_desc(&tmD);
-    tma_prefetch_desc(&tmDs);
+    tma_prefetch_desc(&maps.sgu);
+    tma_prefetch_desc(&maps.sd);
+    if (WQ) {
+      tma_prefetch_desc(&maps.qc_gu);
+      tma_prefetch_desc(&maps.qc_d);
+    } else {
+      tma_prefetch_desc(&maps.gu);
+      tma_prefetch_desc(&maps.d);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, TMEM_COLS);
@@ -197,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ---------------- TMA producer: phase-A then phase-B weights of every item ----------------
       const uint64_t pol = l2_policy_evict_first();  // read once per call
+      const int I = args.I, H = args.H;
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
@@ -204,25 +255,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
         const int g = group_of(L);
         const int j = L - item_start[g];
-        const CUtensorMap* gu = g < E ? &tmGU : &tmGUs;
-        const CUtensorMap* dn = g < E ? &tmD : &tmDs;
-        const int gu_base = g < E ? g * 2 * args.I : 0;
-        const int dn_base = g < E ? g * args.H : 0;
+        const bool q = WQ && g < E;  // AWQ routed expert
         for (int st = 0; st < NSA + NSB && ok; ++st) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
-          if (st < NSA) {
-            mbar_arrive_expect_tx(&full_bar[stage], uint32_t(KSUB * A_BYTES));
-            for (int u = 0; u < KSUB; ++u) {
+          const bool pa = st < NSA;
+          const int m0 = pa ? 0 : (st - NSA) * KSUB;
+          const int nsub = pa ? KSUB : min(KSUB, MB2 - m0);
+          mbar_arrive_expect_tx(&full_bar[stage], uint32_t(nsub) * (q ? Q_TX : uint32_t(A_BYTES)));
+          for (int u = 0; u < nsub; ++u) {
+            uint8_t* d = sub(stage, u);
+            uint64_t* fb = &full_bar[stage];
+            if (pa) {
               const int kx = (st * KSUB + u) * BK;
-              tma_load_2d_hint(sub(stage, u), gu, &full_bar[stage], kx, gu_base + j * 64, pol);
-              tma_load_2d_hint(sub(stage, u) + 64 * BK * 2, gu, &full_bar[stage], kx, gu_base + args.I + j * 64, pol);
+              if (q) {
+                // gate columns 64j.., up columns I + 64j.. of the input-major codes
+                const int crow = g * H + kx, grow = g * (H / 32) + kx / 32;
+                tma_load_2d_hint(d + Q_CODES, &maps.qc_gu, fb, j * 8, crow, pol);
+                tma_load_2d_hint(d + Q_CODES + 2048, &maps.qc_gu, fb, I / 8 + j * 8, crow, pol);
+                tma_load_2d_hint(d + Q_SCALES, &maps.qs_gu, fb, j * 64, grow, pol);
+                tma_load_2d_hint(d + Q_SCALES + 256, &maps.qs_gu, fb, I + j * 64, grow, pol);
+                tma_load_2d_hint(d + Q_ZEROS, &maps.qz_gu, fb, j * 8, grow, pol);
+                tma_load_2d_hint(d + Q_ZEROS + 128, &maps.qz_gu, fb, I / 8 + j * 8, grow, pol);
+              } else {
+                const CUtensorMap* gu = g < E ? &maps.gu : &maps.sgu;
+                const int base = g < E ? g * 2 * I : 0;
+                tma_load_2d_hint(d, gu, fb, kx, base + j * 64, pol);
+                tma_load_2d_hint(d + 64 * BK * 2, gu, fb, kx, base + I + j * 64, pol);
+              }
+            } else {
+              const int m = m0 + u;
+              if (q) {
+                const int crow = g * I + j * BK, grow = g * (I / 32) + j * 2;
+                tma_load_2d_hint(d + Q_CODES, &maps.qc_d, fb, m * 16, crow, pol);
+                tma_load_2d_hint(d + Q_SCALES, &maps.qs_d, fb, m * BM, grow, pol);
+                tma_load_2d_hint(d + Q_ZEROS, &maps.qz_d, fb, m * 16, grow, pol);
+              } else {
+                const CUtensorMap* dn = g < E ? &maps.d : &maps.sd;
+                tma_load_2d_hint(d, dn, fb, j * BK, (g < E ? g * H : 0) + m * BM, pol);
+              }
             }
-          } else {
-            const int m0 = (st - NSA) * KSUB;
-            const int nsub = min(KSUB, MB2 - m0);
-            mbar_arrive_expect_tx(&full_bar[stage], uint32_t(nsub * A_BYTES));
-            for (int u = 0; u < nsub; ++u)
-              tma_load_2d_hint(sub(stage, u), dn, &full_bar[stage], j * BK, dn_base + (m0 + u) * BM, pol);
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -237,12 +308,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- UMMA issuer ----------------
-      const uint32_t idesc = idesc_f16(args.bf16, BM, NT);
+      // 16-bit weights: K-major A; AWQ: the dequantised MN-major A (bit 15)
+      const uint32_t idesc_k = idesc_f16(args.bf16, BM, NT);
+      const uint32_t idesc_q = idesc_k | (1u << 15);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int n = 0;  // items of this CTA so far
+      // the stage's operands are complete: TMA + tokens (full), or after dequantisation (aready)
+      auto wait_operands = [&](int s) {
+        return mbar_wait(WQ ? &aready_bar[s] : &full_bar[s], phase, &abort_flag, status, lim);
+      };
+      auto adesc = [&](const uint8_t* tile, bool q, int kk) {
+        return q ? sdesc_mnmajor_sw128(smem_u32(tile), AQ_LBO, AQ_SBO) + uint64_t(kk * (2 * AQ_SBO >> 4))
+                 : sdesc_kmajor_sw128(smem_u32(tile)) + uint64_t(kk * 2);
+      };
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++n) {
+        const int g = group_of(L);
+        const bool q = WQ && g < E;
+        const uint32_t idesc = q ? idesc_q : idesc_k;
         const int a = n & 1;                     // phase-A accumulator and h tile of this item
         const uint32_t pa = uint32_t((n >> 1) & 1);  // their phase parity
         // phase A: D_A[weight row, token] over K = H
@@ -250,14 +334,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t dA = tmem_base + uint32_t(a * NT);
         for (int st = 0; st < NSA; ++st) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
+          if (!wait_operands(stage)) { ok = false; break; }
           tc_fence_after();
           for (int u = 0; u < KSUB; ++u) {
-            const uint64_t ad = sdesc_kmajor_sw128(smem_u32(sub(stage, u)));
             const uint64_t bd = sdesc_kmajor_sw128(smem_u32(sub(stage, u) + A_BYTES));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              umma_f16(dA, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (st | u | kk) != 0);
+              umma_f16(dA, adesc(sub(stage, u), q, kk), bd + uint64_t(kk * 2), idesc, (st | u | kk) != 0);
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -273,14 +356,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int st = 0; st < NSB; ++st) {
           const int m0 = st * KSUB;
           const int nsub = min(KSUB, MB2 - m0);
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
+          if (!wait_operands(stage)) { ok = false; break; }
           tc_fence_after();
           for (int u = 0; u < nsub; ++u) {
-            const uint64_t ad = sdesc_kmajor_sw128(smem_u32(sub(stage, u)));
             const uint32_t dB = tmem_base + ACCB_COL + uint32_t((m0 + u) * NT);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              umma_f16(dB, ad + uint64_t(kk * 2), hd + uint64_t(kk * 2), idesc, kk != 0);
+              umma_f16(dB, adesc(sub(stage, u), q, kk), hd + uint64_t(kk * 2), idesc, kk != 0);
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -368,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&accB_empty);
     }
-  } else {
+  } else if (warp < 10) {
     // ---------------- token gather: warps 6..9 ----------------
     // Thread gt copies 16-byte chunk (gt % 8) of token row gt / 8 of every
     // phase-A sub-tile into the K-major swizzled token tile; rows past the
@@ -406,6 +488,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");  // every copy has landed before the block exits
+  } else if (WQ) {
+    // ---------------- AWQ dequantisation: warps 10..13 ----------------
+    // Thread (wc, r0): code word column wc (output columns 8wc..8wc+7 of the
+    // tile: phase A wc < 8 gate, wc >= 8 up; phase B the 128 down rows of the
+    // block) of K rows r0, r0 + 8, ..., r0 + 56 -> one 16-byte chunk of the
+    // MN-major FP16 tile per row.  Shared-expert stages (16-bit) need nothing:
+    // the threads only arrive.
+    const int dt = threadIdx.x - 320;
+    const int wc = dt & 15;
+    const int r0 = dt >> 4;  // 0..7
+    const uint32_t atom_off = uint32_t(wc >> 3) * AQ_LBO;
+    const uint32_t chunk = uint32_t(wc & 7);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+      const int g = group_of(L);
+      const bool q = g < E;
+      for (int st = 0; st < NSA + NSB; ++st) {
+        if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
+        const bool pa = st < NSA;
+        const int nsub = pa ? KSUB : min(KSUB, MB2 - (st - NSA) * KSUB);
+        if (q) {
+          for (int u = 0; u < nsub; ++u) {
+            uint8_t* d = sub(stage, u);
+            // phase A: box (wc / 8) of width 8 words; phase B: one box of 16
+            const int half = pa ? (wc >> 3) : 0;
+            const int wl = pa ? (wc & 7) : wc;
+            const int cw = pa ? 8 : 16;  // code words per K row in the box
+            const uint32_t* codes = reinterpret_cast<const uint32_t*>(d + Q_CODES + half * 2048) + wl;
+            const uint16_t* sc = reinterpret_cast<const uint16_t*>(d + Q_SCALES + half * 256) + wl * 8;
+            const uint32_t* zr = reinterpret_cast<const uint32_t*>(d + Q_ZEROS + half * 128) + wl;
+            const uint4 s0 = *reinterpret_cast<const uint4*>(sc);
+            const uint4 s1 = *reinterpret_cast<const uint4*>(sc + cw * 8);
+            const uint32_t z0 = zr[0], z1 = zr[cw];
+            uint8_t* at = d + atom_off;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = r0 + 8 * i;
+              const uint4 v = r < 32 ? awq_dequant8(codes[r * cw], z0, s0) : awq_dequant8(codes[r * cw], z1, s1);
+              const uint32_t off = uint32_t(r >> 3) * AQ_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
+              *reinterpret_cast<uint4*>(at + off) = v;
+            }
+          }
+          fence_proxy_async_smem();  // the FP16 tile is read by the tensor cores
+        }
+        mbar_arrive(&aready_bar[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
   }
 
   tc_fence_before();
@@ -446,20 +578,32 @@ __global__ void __launch_bounds__(256) k_sum_partials(const float* __restrict__ 
   *reinterpret_cast<uint2*>(out) = v;
 }
 
-}  // namespace
-
-size_t decode_fused_ws_bytes(int rows, int T, int H, int I) {
-  WsCounter c;
-  c.take<float>(size_t(I / BK) * (rows + T) * H);
-  return c.used;
+template <int WQ>
+int launch_fused(const Maps& maps, const Args& a, int f_fp32, void* f, void* shared_out, cudaStream_t stream) {
+  using Cfg = FusedCfg<WQ>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  MOE_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev >= 64 || !attr_set[dev]) {
+    MOE_CHECK_CUDA(cudaFuncSetAttribute(k_decode_ffn<WQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+    if (dev < 64) attr_set[dev] = true;
+  }
+  MOE_CHECK_CUDA(launch_pdl(k_decode_ffn<WQ>, dim3(num_sms()), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, stream, maps, a));
+  const int R = a.rows + a.T;
+  if (R == 0) return MOE_OK;
+  const dim3 grid(R, (a.H / 4 + 255) / 256);
+  if (a.bf16)
+    MOE_CHECK_CUDA(launch_pdl(k_sum_partials<__nv_bfloat16>, grid, dim3(256), 0, stream,
+                              static_cast<const float*>(a.partial), a.I / BK, R, a.rows, a.H, f, f_fp32,
+                              static_cast<__nv_bfloat16*>(shared_out)));
+  else
+    MOE_CHECK_CUDA(launch_pdl(k_sum_partials<__half>, grid, dim3(256), 0, stream, static_cast<const float*>(a.partial),
+                              a.I / BK, R, a.rows, a.H, f, f_fp32, static_cast<__half*>(shared_out)));
+  return MOE_OK;
 }
 
-// Routed experts (rows in permuted order, f [rows, H]) and the shared expert
-// (shared_out [T, H]) for T <= 16 with weights of width I: k_decode_ffn then
-// k_sum_partials.  The FP32 partials [I/64][rows + T][H] live in ws.
-int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
-                         int E, const void* w_gu, const void* w_d, const void* w_sh_gu, const void* w_sh_d, int dtype,
-                         int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+int fill_args(Args& a, const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
+              int E, int dtype, void* ws, size_t ws_bytes) {
   MOE_REQUIRE(T <= kFusedMaxT, MOE_ERR_UNSUPPORTED, "fused decode experts: T=%d > %d", T, kFusedMaxT);
   MOE_REQUIRE(H % BM == 0 && I % BK == 0, MOE_ERR_UNSUPPORTED,
               "fused decode experts: need H %% 128 == 0 and I %% 64 == 0 (H=%d I=%d)", H, I);
@@ -467,13 +611,7 @@ int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t*
   WsCarver carve(ws, ws_bytes);
   float* P = carve.take<float>(size_t(I / BK) * (rows + T) * H);
   MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "fused decode experts: workspace of %zu bytes is too small", ws_bytes);
-  CUtensorMap tgu, tgus, td, tds;
-  int rc = make_tmap_16bit_sw128(&tgu, w_gu, E * 2 * I, H, 64);
-  if (!rc) rc = make_tmap_16bit_sw128(&tgus, w_sh_gu, 2 * I, H, 64);
-  if (!rc) rc = make_tmap_16bit_sw128(&td, w_d, E * H, I, BM);
-  if (!rc) rc = make_tmap_16bit_sw128(&tds, w_sh_d, H, I, BM);
-  if (rc) return rc;
-  Args a{};
+  a = Args{};
   a.offsets = offsets;
   a.E = E;
   a.rows = rows;
@@ -486,24 +624,62 @@ int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t*
   a.bf16 = dtype == MOE_DTYPE_BF16;
   a.status = device_status_ptr();
   a.limit_ns = wait_limit_ns();
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  MOE_CHECK_CUDA(cudaGetDevice(&dev));
-  if (dev >= 64 || !attr_set[dev]) {
-    MOE_CHECK_CUDA(cudaFuncSetAttribute(k_decode_ffn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    if (dev < 64) attr_set[dev] = true;
-  }
-  MOE_CHECK_CUDA(launch_pdl(k_decode_ffn, dim3(num_sms()), dim3(kThreads), SMEM_BYTES, stream, tgu, tgus, td, tds, a));
-  const int R = rows + T;
-  if (R == 0) return MOE_OK;
-  const dim3 grid(R, (H / 4 + 255) / 256);
-  if (a.bf16)
-    MOE_CHECK_CUDA(launch_pdl(k_sum_partials<__nv_bfloat16>, grid, dim3(256), 0, stream, static_cast<const float*>(P),
-                              I / BK, R, rows, H, f, f_fp32, static_cast<__nv_bfloat16*>(shared_out)));
-  else
-    MOE_CHECK_CUDA(launch_pdl(k_sum_partials<__half>, grid, dim3(256), 0, stream, static_cast<const float*>(P), I / BK,
-                              R, rows, H, f, f_fp32, static_cast<__half*>(shared_out)));
   return MOE_OK;
+}
+
+}  // namespace
+
+size_t decode_fused_ws_bytes(int rows, int T, int H, int I) {
+  WsCounter c;
+  c.take<float>(size_t(I / BK) * (rows + T) * H);
+  return c.used;
+}
+
+// Routed experts (rows in permuted order, f [rows, H]) and the shared expert
+// (shared_out [T, H]) for T <= 16 with 16-bit weights of width I:
+// k_decode_ffn then k_sum_partials.  The FP32 partials [I/64][rows + T][H]
+// live in ws.
+int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
+                         int E, const void* w_gu, const void* w_d, const void* w_sh_gu, const void* w_sh_d, int dtype,
+                         int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Args a;
+  int rc = fill_args(a, x, row_token, offsets, T, rows, H, I, E, dtype, ws, ws_bytes);
+  if (rc) return rc;
+  Maps m;
+  memset(&m, 0, sizeof(m));
+  rc = make_tmap_16bit_sw128(&m.gu, w_gu, E * 2 * I, H, 64);
+  if (!rc) rc = make_tmap_16bit_sw128(&m.sgu, w_sh_gu, 2 * I, H, 64);
+  if (!rc) rc = make_tmap_16bit_sw128(&m.d, w_d, E * H, I, BM);
+  if (!rc) rc = make_tmap_16bit_sw128(&m.sd, w_sh_d, H, I, BM);
+  if (rc) return rc;
+  return launch_fused<0>(m, a, f_fp32, f, shared_out, stream);
+}
+
+// The same with the routed experts in AWQ W4A16 g32 (qw_* input-major codes,
+// qz_* zero points, sc_* FP16 scales; FP16 activations) and the shared
+// expert in FP16.
+int decode_experts_fused_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
+                             int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
+                             const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gu,
+                             const void* w_sh_d, int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
+                             cudaStream_t stream) {
+  Args a;
+  int rc = fill_args(a, x, row_token, offsets, T, rows, H, I, E, MOE_DTYPE_F16, ws, ws_bytes);
+  if (rc) return rc;
+  Maps m;
+  memset(&m, 0, sizeof(m));
+  const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  rc = make_tmap_16bit_sw128(&m.sgu, w_sh_gu, 2 * I, H, 64);
+  if (!rc) rc = make_tmap_16bit_sw128(&m.sd, w_sh_d, H, I, BM);
+  // gate/up: input dim H, output dim 2I; down: input dim I, output dim H
+  if (!rc) rc = make_tmap_2d(&m.qc_gu, qw_gu, E * H, 2 * I / 8, 4, BK, 8, none);
+  if (!rc) rc = make_tmap_2d(&m.qs_gu, sc_gu, E * (H / 32), 2 * I, 2, 2, 64, none);
+  if (!rc) rc = make_tmap_2d(&m.qz_gu, qz_gu, E * (H / 32), 2 * I / 8, 4, 2, 8, none);
+  if (!rc) rc = make_tmap_2d(&m.qc_d, qw_d, E * I, H / 8, 4, BK, 16, none);
+  if (!rc) rc = make_tmap_2d(&m.qs_d, sc_d, E * (I / 32), H, 2, 2, BM, none);
+  if (!rc) rc = make_tmap_2d(&m.qz_d, qz_d, E * (I / 32), H / 8, 4, 2, 16, none);
+  if (rc) return rc;
+  return launch_fused<1>(m, a, f_fp32, f, shared_out, stream);
 }
 
 }  // namespace moe

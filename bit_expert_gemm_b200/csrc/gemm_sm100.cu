@@ -474,6 +474,8 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // 2-D tensor map of a row-major [rows, cols] matrix of `esize`-byte elements,
 // box [box_rows, box_cols].
 int make_tmap_2d(CUtensorMap* map, const void* base, int rows, int cols, int esize, int box_rows, int box_cols,
@@ -496,7 +498,6 @@ int make_tmap_2d(CUtensorMap* map, const void* base, int rows, int cols, int esi
   return MOE_OK;
 }
 
-}  // namespace
 
 // 2-D tensor map of a row-major [rows, cols] 16-bit matrix, box [box_rows, 64]
 // with the 128-byte swizzle (the K-major UMMA operand layout).

@@ -107,11 +107,12 @@ class MoELayer:
         self.ws_route = abi.workspace(abi.MOE_OP_ROUTE_PERMUTE, T_max, H, E, ks, 0, d)
         self.ws_ffn = abi.workspace(op, T_max, H, E, ks, self.I, d)
         self.ws_sh = abi.workspace(abi.MOE_OP_SWIGLU_BF16, T_max, H, 1, 1, self.I_sh, d)
-        if self.fmt == "bf16" and self.I_sh == self.I:
-            # routed + shared experts in one call: big enough for the decode path
-            # (T <= 128) and the prefill path
-            need = max(abi.moe_workspace_size(abi.MOE_OP_EXPERTS_BF16, t, H, E, ks, self.I)
-                       for t in {T_max, min(T_max, 128)})
+        if self.fmt in ("bf16", "awq_g32") and self.I_sh == self.I:
+            # routed + shared experts in one call: big enough for every path it
+            # takes for T <= T_max (T <= 16, T <= 128, larger)
+            op_exp = abi.MOE_OP_EXPERTS_BF16 if self.fmt == "bf16" else abi.MOE_OP_EXPERTS_AWQ_G32
+            need = max(abi.moe_workspace_size(op_exp, t, H, E, ks, self.I)
+                       for t in {T_max, min(T_max, 128), min(T_max, 16)})
             self.ws_exp = torch.empty(max(256, need), dtype=torch.uint8, device=d)
         else:
             self.ws_exp = None
@@ -159,7 +160,7 @@ class MoELayer:
 
     def experts_and_shared(self, x: torch.Tensor):
         """Routed expert rows f and the shared expert's output; one C-ABI call
-        (moe_experts_bf16) for 16-bit weights."""
+        (moe_experts_bf16 / moe_experts_awq_g32) for 16-bit and AWQ weights."""
         if self.ws_exp is None:
             return self.experts(x), self.shared_expert(x)
         T = x.shape[0]
@@ -167,9 +168,14 @@ class MoELayer:
         f = self.f[:rows]
         sh = self.shared[:T]
         w = self.w
-        abi.moe_experts_bf16(x, self.row_token[:rows], self.offsets, rows, w["w_gate_up"], w["w_down"],
-                             w["w_sh_gate_up"], w["w_sh_down"], out_fp32=f.dtype == torch.float32, f=f,
-                             shared_out=sh, ws=self.ws_exp)
+        if self.fmt == "bf16":
+            abi.moe_experts_bf16(x, self.row_token[:rows], self.offsets, rows, w["w_gate_up"], w["w_down"],
+                                 w["w_sh_gate_up"], w["w_sh_down"], out_fp32=f.dtype == torch.float32, f=f,
+                                 shared_out=sh, ws=self.ws_exp)
+        else:
+            abi.moe_experts_awq_g32(x, self.row_token[:rows], self.offsets, rows, w["qw_gu"], w["qz_gu"], w["sc_gu"],
+                                    w["qw_d"], w["qz_d"], w["sc_d"], w["w_sh_gate_up"], w["w_sh_down"],
+                                    out_fp32=f.dtype == torch.float32, f=f, shared_out=sh, ws=self.ws_exp)
         return f, sh
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:

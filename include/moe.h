@@ -83,7 +83,8 @@ enum {
   MOE_OP_REFILL = 5,
   MOE_OP_NVFP4_QUANTIZE = 6,
   MOE_OP_EXPERTS_BF16 = 7,
-  MOE_OP_ROUTE_PERMUTE = 8
+  MOE_OP_ROUTE_PERMUTE = 8,
+  MOE_OP_EXPERTS_AWQ_G32 = 9
 };
 
 /* Version of this header's ABI. */
@@ -201,12 +202,15 @@ MOE_API int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, con
  * routed part is moe_grouped_swiglu_bf16 (f [rows, H]), the shared part the
  * same SwiGLU on every token with w_sh_gate_up [2I, H] and w_sh_down [H, I]
  * (shared_out [T, H] dtype; the shared expert has the routed experts' width
- * I).  For T <= 128 (decode) both run as weight-streaming tensor-core GEMMs
- * with the weights as the M operand and the few tokens as N, routed and
- * shared work items in the same two launches: the first applies SwiGLU in its
- * epilogue and writes h [rows + T, I] (dtype) to the workspace, the second
- * reads it back.  Larger T uses the grouped prefill GEMMs.  row_token is
- * required.
+ * I).  Decode-sized batches run as weight-streaming tensor-core GEMMs with
+ * the weights as the M operand and the few tokens as N, routed and shared
+ * work items in the same launches: for T <= 16 one kernel computes, per
+ * block of 64 intermediate features, gate/up, SwiGLU and that block's slice
+ * of the down projection, FP32 partials that a second kernel sums in a fixed
+ * order (no wait between the two GEMMs); for 16 < T <= 128 the first GEMM
+ * applies SwiGLU in its epilogue and writes h [rows + T, I] (dtype) to the
+ * workspace, the second reads it back.  Larger T uses the grouped prefill
+ * GEMMs.  row_token is required.
  * Limits: H % 128 == 0, I % 64 == 0.  Workspace: MOE_OP_EXPERTS_BF16.
  * ------------------------------------------------------------------------- */
 MOE_API int moe_experts_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows,
@@ -236,6 +240,25 @@ MOE_API int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, 
                                int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
                                const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
                                int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Routed AWQ experts and the FP16 shared expert of one layer in one call
+ * [AWQ] [ARCH]: the routed part is moe_grouped_swiglu_awq_g32 (f [rows, H]),
+ * the shared part the SwiGLU of every token with w_sh_gate_up [2I, H] and
+ * w_sh_down [H, I] FP16 (shared_out [T, H] FP16).  For T <= 16 (decode) both
+ * run in one weight-streaming kernel: the routed weights stream as packed
+ * codes, zero points and scales and are dequantised in shared memory, the
+ * second GEMM is split along I into FP32 partials in the workspace that a
+ * second kernel sums in a fixed order.  Larger T uses the grouped AWQ GEMMs
+ * and then the dense shared expert.  Layouts, exact dequantisation and x as
+ * in moe_grouped_swiglu_awq_g32; row_token is required.  Limits: H % 128 ==
+ * 0, I % 64 == 0.  Workspace: MOE_OP_EXPERTS_AWQ_G32.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_experts_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
+                                int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
+                                const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
+                                const void* w_sh_gate_up, const void* w_sh_down, int out_fp32, void* f,
+                                void* shared_out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * AWQ dequantisation [AWQ], the same device code the grouped GEMM runs on

@@ -48,6 +48,33 @@ def _awq_expert_fn(w, I):
     return ew
 
 
+@pytest.mark.parametrize("T,H,I,E,k,out_fp32", [(1, 2048, 640, 512, 10, False), (8, 512, 128, 16, 4, True),
+                                                (16, 1024, 192, 64, 6, False), (3, 256, 64, 16, 2, True),
+                                                (40, 512, 128, 16, 4, False)])
+def test_experts_awq_routed_and_shared(T, H, I, E, k, out_fp32):
+    """moe_experts_awq_g32: routed AWQ experts (T <= 16: dequantised in the
+    split-K weight-streaming kernel; larger T: the grouped AWQ GEMMs) and the
+    FP16 shared expert, against the oracle."""
+    wl = dataclasses.replace(synth.WORKLOADS["awq_g32"], H=H, I=I, I_sh=I, E=E, k=k)
+    w = synth.make_weights(wl, seed=T + I + 3, device=DEV)
+    x = synth.make_tokens(wl, T, seed=T + 3, device=DEV)
+    idx = synth.make_routing(T, E, k, seed=T + 4)
+    off, rt, sr = abi.moe_permute(idx.to(DEV), E)
+    f, sh = abi.moe_experts_awq_g32(x, rt, off, T * k, w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"], w["qz_d"],
+                                    w["sc_d"], w["w_sh_gate_up"], w["w_sh_down"], out_fp32=out_fp32)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0
+    perm = moe.permute(idx.numpy().astype(np.int64), E)
+    xs = f64(x)
+    ref, _ = moe.routed_outputs(xs, perm, _awq_expert_fn(w, I))
+    err = rel_err(f64(f)[sr.cpu().numpy().ravel()], ref[perm["slot_row"].ravel()])
+    assert err < 1e-2, err  # FP16 h and output rounding only
+    sg = f64(w["w_sh_gate_up"])
+    sref, _ = moe.swiglu_expert(xs, sg[:I], sg[I:], f64(w["w_sh_down"]))
+    err_sh = rel_err(f64(sh), sref)
+    assert err_sh < 1e-2, err_sh
+
+
 FFN_CASES = [
     # T, H, I, E, k
     (37, 256, 64, 16, 2),
