@@ -144,16 +144,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended (it issues nothing) until the phase completes or about 1 ms
+// passes, so waiting roles leave the issue slots to the working ones.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase of `bar` with the given parity has completed.  The
 // wait is bounded: after `limit_ns` (or as soon as another role of the CTA
 // raised *abort) it records MOE_ERR_TIMEOUT, raises *abort and returns false.
+// The deadline and the abort flag are checked every 64 suspended tries, so the
+// wait ends at most about 64 ms after either.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
                                           unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer_ns();
   uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity)) return true;
     if (((++spins) & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
@@ -352,21 +369,38 @@ struct Pack2<__half> {
 // pairs (j = 2m low half, 2m+1 high half).  0x6400 | q is the FP16 value
 // 1024 + q, so one subtraction of two such values gives q - z exactly; the
 // single FP16 multiplication then rounds once, to nearest even.
-__device__ __forceinline__ uint32_t awq_pair_1024(uint32_t w, int m) {
-  return ((w >> (8 * m)) & 0xFu) | (((w >> (8 * m + 4)) & 0xFu) << 16) | 0x64006400u;
+//
+// (W >> 4m) & 0x000F000F | 0x64006400 yields the pair (1024 + q_m,
+// 1024 + q_{m+4}) in one logic operation, so the arithmetic runs on the pairs
+// (m, m+4) and four byte permutations restore the column order.  The zero
+// points and scales of a group (AwqGroup) are prepared once for its 32 rows.
+struct AwqGroup {
+  uint32_t z[4];  // FP16 pairs (1024 + z_m, 1024 + z_{m+4})
+  uint32_t s[4];  // FP16 pairs (s_m, s_{m+4})
+};
+__device__ __forceinline__ AwqGroup awq_group(uint32_t Z, uint4 S) {
+  AwqGroup g;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) g.z[m] = ((Z >> (4 * m)) & 0x000F000Fu) | 0x64006400u;
+  g.s[0] = __byte_perm(S.x, S.z, 0x5410);
+  g.s[1] = __byte_perm(S.x, S.z, 0x7632);
+  g.s[2] = __byte_perm(S.y, S.w, 0x5410);
+  g.s[3] = __byte_perm(S.y, S.w, 0x7632);
+  return g;
 }
-__device__ __forceinline__ uint4 awq_dequant8(uint32_t W, uint32_t Z, uint4 S) {
-  const uint32_t sp[4] = {S.x, S.y, S.z, S.w};
-  uint32_t r[4];
+__device__ __forceinline__ uint4 awq_dequant8(uint32_t W, const AwqGroup& g) {
+  uint32_t d[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    uint32_t q = awq_pair_1024(W, m), z = awq_pair_1024(Z, m);
-    __half2 d = __hsub2(*reinterpret_cast<__half2*>(&q), *reinterpret_cast<__half2*>(&z));
-    __half2 v = __hmul2(d, *reinterpret_cast<const __half2*>(&sp[m]));
-    r[m] = *reinterpret_cast<uint32_t*>(&v);
+    uint32_t q = ((W >> (4 * m)) & 0x000F000Fu) | 0x64006400u;
+    __half2 t = __hsub2(*reinterpret_cast<__half2*>(&q), *reinterpret_cast<const __half2*>(&g.z[m]));
+    __half2 v = __hmul2(t, *reinterpret_cast<const __half2*>(&g.s[m]));
+    d[m] = *reinterpret_cast<uint32_t*>(&v);  // (c_m, c_{m+4})
   }
-  return make_uint4(r[0], r[1], r[2], r[3]);
+  return make_uint4(__byte_perm(d[0], d[1], 0x5410), __byte_perm(d[2], d[3], 0x5410), __byte_perm(d[0], d[1], 0x7632),
+                    __byte_perm(d[2], d[3], 0x7632));
 }
+__device__ __forceinline__ uint4 awq_dequant8(uint32_t W, uint32_t Z, uint4 S) { return awq_dequant8(W, awq_group(Z, S)); }
 
 // Shared-memory matrix descriptor of an MN-major operand in the 128-byte
 // swizzled layout: atoms of 64 16-bit elements along MN by 8 rows along K

@@ -29,7 +29,7 @@
 //     FP16 tile, and the MMA reads that.
 //
 // Warp roles: 0 TMA producer, 1 UMMA issuer (TMEM owner), 2..5 epilogue,
-// 6..9 token gather (cp.async, arriving on the stage's barrier), 10..13 AWQ
+// 6..9 token gather (cp.async, arriving on the stage's barrier), 10..17 AWQ
 // dequantisation (WQ = 1).  TMEM: two 16-column phase-A accumulators
 // (columns 0..31) and one phase-B accumulator of H/128 blocks x 16 columns
 // (from column 32).
@@ -72,7 +72,7 @@ constexpr uint32_t Q_TX = 64 * 16 * 4 + 2 * 128 * 2 + 2 * 16 * 4;  // bytes the 
 // 8-row K groups SBO apart; one MMA (K = 16) spans two K groups
 constexpr uint32_t AQ_LBO = (BK / 8) * 1024;
 constexpr uint32_t AQ_SBO = 1024;
-constexpr int kDequantThreads = 128;
+constexpr int kDequantThreads = 256;  // two dequantisation warps per SM sub-partition
 
 template <int WQ>
 struct FusedCfg {
@@ -176,7 +176,11 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
     tma_prefetch_desc(&maps.sd);
     if (WQ) {
       tma_prefetch_desc(&maps.qc_gu);
+      tma_prefetch_desc(&maps.qs_gu);
+      tma_prefetch_desc(&maps.qz_gu);
       tma_prefetch_desc(&maps.qc_d);
+      tma_prefetch_desc(&maps.qs_d);
+      tma_prefetch_desc(&maps.qz_d);
     } else {
       tma_prefetch_desc(&maps.gu);
       tma_prefetch_desc(&maps.d);
@@ -244,66 +248,74 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
   };
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer: phase-A then phase-B weights of every item ----------------
-      const uint64_t pol = l2_policy_evict_first();  // read once per call
-      const int I = args.I, H = args.H;
-      int stage = 0;
-      uint32_t phase = 0;
-      long issued = 0;
-      bool ok = true;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-        const int g = group_of(L);
-        const int j = L - item_start[g];
-        const bool q = WQ && g < E;  // AWQ routed expert
-        for (int st = 0; st < NSA + NSB && ok; ++st) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
-          const bool pa = st < NSA;
-          const int m0 = pa ? 0 : (st - NSA) * KSUB;
-          const int nsub = pa ? KSUB : min(KSUB, MB2 - m0);
+    // ---------------- TMA producer: phase-A then phase-B weights of every item ----------------
+    // Lane 0 owns the stage barriers; the copies of a stage (up to 12) are
+    // issued together, one per lane, in the same instructions: a copy costs
+    // its issuing thread on the order of a hundred cycles.
+    const uint64_t pol = l2_policy_evict_first();  // read once per call
+    const int I = args.I, H = args.H;
+    int stage = 0;
+    uint32_t phase = 0;
+    long issued = 0;
+    bool ok = true;
+    for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+      const int g = group_of(L);
+      const int j = L - item_start[g];
+      const bool q = WQ && g < E;  // AWQ routed expert
+      for (int st = 0; st < NSA + NSB; ++st) {
+        if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const bool pa = st < NSA;
+        const int m0 = pa ? 0 : (st - NSA) * KSUB;
+        const int nsub = pa ? KSUB : min(KSUB, MB2 - m0);
+        if (lane == 0)
           mbar_arrive_expect_tx(&full_bar[stage], uint32_t(nsub) * (q ? Q_TX : uint32_t(A_BYTES)));
-          for (int u = 0; u < nsub; ++u) {
-            uint8_t* d = sub(stage, u);
-            uint64_t* fb = &full_bar[stage];
-            if (pa) {
-              const int kx = (st * KSUB + u) * BK;
-              if (q) {
-                // gate columns 64j.., up columns I + 64j.. of the input-major codes
-                const int crow = g * H + kx, grow = g * (H / 32) + kx / 32;
-                tma_load_2d_hint(d + Q_CODES, &maps.qc_gu, fb, j * 8, crow, pol);
-                tma_load_2d_hint(d + Q_CODES + 2048, &maps.qc_gu, fb, I / 8 + j * 8, crow, pol);
-                tma_load_2d_hint(d + Q_SCALES, &maps.qs_gu, fb, j * 64, grow, pol);
-                tma_load_2d_hint(d + Q_SCALES + 256, &maps.qs_gu, fb, I + j * 64, grow, pol);
-                tma_load_2d_hint(d + Q_ZEROS, &maps.qz_gu, fb, j * 8, grow, pol);
-                tma_load_2d_hint(d + Q_ZEROS + 128, &maps.qz_gu, fb, I / 8 + j * 8, grow, pol);
-              } else {
-                const CUtensorMap* gu = g < E ? &maps.gu : &maps.sgu;
-                const int base = g < E ? g * 2 * I : 0;
-                tma_load_2d_hint(d, gu, fb, kx, base + j * 64, pol);
-                tma_load_2d_hint(d + 64 * BK * 2, gu, fb, kx, base + I + j * 64, pol);
-              }
+        __syncwarp();
+        // copy `lane` of the stage: per sub-tile 6 (AWQ phase A), 3 (AWQ
+        // phase B), 2 (16-bit phase A) or 1 (16-bit phase B)
+        const int per = q ? (pa ? 6 : 3) : (pa ? 2 : 1);
+        const int u = lane / per, which = lane - u * per;
+        if (u < nsub) {
+          uint8_t* d = sub(stage, u);
+          uint64_t* fb = &full_bar[stage];
+          if (pa) {
+            const int kx = (st * KSUB + u) * BK;
+            if (q) {
+              // gate columns 64j.., up columns I + 64j.. of the input-major codes
+              const int crow = g * H + kx, grow = g * (H / 32) + kx / 32;
+              const int half = which & 1, kind = which >> 1;  // kind 0 codes, 1 scales, 2 zeros
+              const int c8 = half ? I / 8 + j * 8 : j * 8;
+              if (kind == 0) tma_load_2d_hint(d + Q_CODES + half * 2048, &maps.qc_gu, fb, c8, crow, pol);
+              else if (kind == 1) tma_load_2d_hint(d + Q_SCALES + half * 256, &maps.qs_gu, fb, c8 * 8, grow, pol);
+              else tma_load_2d_hint(d + Q_ZEROS + half * 128, &maps.qz_gu, fb, c8, grow, pol);
             } else {
-              const int m = m0 + u;
-              if (q) {
-                const int crow = g * I + j * BK, grow = g * (I / 32) + j * 2;
-                tma_load_2d_hint(d + Q_CODES, &maps.qc_d, fb, m * 16, crow, pol);
-                tma_load_2d_hint(d + Q_SCALES, &maps.qs_d, fb, m * BM, grow, pol);
-                tma_load_2d_hint(d + Q_ZEROS, &maps.qz_d, fb, m * 16, grow, pol);
-              } else {
-                const CUtensorMap* dn = g < E ? &maps.d : &maps.sd;
-                tma_load_2d_hint(d, dn, fb, j * BK, (g < E ? g * H : 0) + m * BM, pol);
-              }
+              const CUtensorMap* gu = g < E ? &maps.gu : &maps.sgu;
+              const int base = g < E ? g * 2 * I : 0;
+              tma_load_2d_hint(d + which * 64 * BK * 2, gu, fb, kx, base + which * I + j * 64, pol);
+            }
+          } else {
+            const int m = m0 + u;
+            if (q) {
+              const int crow = g * I + j * BK, grow = g * (I / 32) + j * 2;
+              if (which == 0) tma_load_2d_hint(d + Q_CODES, &maps.qc_d, fb, m * 16, crow, pol);
+              else if (which == 1) tma_load_2d_hint(d + Q_SCALES, &maps.qs_d, fb, m * BM, grow, pol);
+              else tma_load_2d_hint(d + Q_ZEROS, &maps.qz_d, fb, m * 16, grow, pol);
+            } else {
+              const CUtensorMap* dn = g < E ? &maps.d : &maps.sd;
+              tma_load_2d_hint(d, dn, fb, j * BK, (g < E ? g * H : 0) + m * BM, pol);
             }
           }
-          ++issued;
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
+        __syncwarp();
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
-      if (!ok) {  // let the loads in flight land before the block exits
-        volatile int never = 0;
-        for (long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-          mbar_wait(&full_bar[i % STAGES], uint32_t((i / STAGES) & 1), &never, nullptr, lim);
-      }
+    }
+    if (!ok && lane == 0) {  // let the loads in flight land before the block exits
+      volatile int never = 0;
+      for (long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+        mbar_wait(&full_bar[i % STAGES], uint32_t((i / STAGES) & 1), &never, nullptr, lim);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -430,20 +442,17 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
       if (!epilogue_all(mbar_wait(&accB_full, uint32_t(n & 1), &abort_flag, status, lim))) break;
       tc_fence_after();
       float* P = args.partial + (size_t(j) * R + r0) * args.H;
-      // four blocks' accumulators (64 consecutive columns) per TMEM load wait
-      for (int m0 = 0; m0 < MB2; m0 += 4) {
-        float w0[32], w1[32];
-        const uint32_t ta = tmem_base + (uint32_t(q * 32) << 16) + ACCB_COL + uint32_t(m0 * NT);
-        tmem_ld32x2(ta, ta + 32, w0, w1);
+      // two blocks' accumulators (32 consecutive columns) per TMEM load wait
+      for (int m0 = 0; m0 < MB2; m0 += 2) {
+        float w0[32];
+        tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + ACCB_COL + uint32_t(m0 * NT), w0);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 2; ++u) {
           if (m0 + u < MB2) {
             const int feat = (m0 + u) * BM + q * 32 + lane;
 #pragma unroll
-            for (int c = 0; c < NT; ++c) {
-              const float val = u < 2 ? w0[u * NT + c] : w1[(u - 2) * NT + c];
-              if (c < nn) P[size_t(c) * args.H + feat] = val;
-            }
+            for (int c = 0; c < NT; ++c)
+              if (c < nn) P[size_t(c) * args.H + feat] = w0[u * NT + c];
           }
         }
       }
@@ -489,15 +498,16 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
     }
     asm volatile("cp.async.wait_all;" ::: "memory");  // every copy has landed before the block exits
   } else if (WQ) {
-    // ---------------- AWQ dequantisation: warps 10..13 ----------------
+    // ---------------- AWQ dequantisation: warps 10..17 ----------------
     // Thread (wc, r0): code word column wc (output columns 8wc..8wc+7 of the
     // tile: phase A wc < 8 gate, wc >= 8 up; phase B the 128 down rows of the
-    // block) of K rows r0, r0 + 8, ..., r0 + 56 -> one 16-byte chunk of the
-    // MN-major FP16 tile per row.  Shared-expert stages (16-bit) need nothing:
-    // the threads only arrive.
+    // block) of K rows r0, r0 + 16, r0 + 32, r0 + 48 -> one 16-byte chunk of
+    // the MN-major FP16 tile per row.  Shared-expert stages (16-bit) need
+    // nothing: the threads only arrive.
+    constexpr int NRW = 64 / (kDequantThreads / 16);  // rows per thread per sub-tile
     const int dt = threadIdx.x - 320;
     const int wc = dt & 15;
-    const int r0 = dt >> 4;  // 0..7
+    const int r0 = dt >> 4;  // 0..15
     const uint32_t atom_off = uint32_t(wc >> 3) * AQ_LBO;
     const uint32_t chunk = uint32_t(wc & 7);
     int stage = 0;
@@ -511,25 +521,41 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
         const bool pa = st < NSA;
         const int nsub = pa ? KSUB : min(KSUB, MB2 - (st - NSA) * KSUB);
         if (q) {
-          for (int u = 0; u < nsub; ++u) {
-            uint8_t* d = sub(stage, u);
-            // phase A: box (wc / 8) of width 8 words; phase B: one box of 16
-            const int half = pa ? (wc >> 3) : 0;
-            const int wl = pa ? (wc & 7) : wc;
-            const int cw = pa ? 8 : 16;  // code words per K row in the box
-            const uint32_t* codes = reinterpret_cast<const uint32_t*>(d + Q_CODES + half * 2048) + wl;
-            const uint16_t* sc = reinterpret_cast<const uint16_t*>(d + Q_SCALES + half * 256) + wl * 8;
-            const uint32_t* zr = reinterpret_cast<const uint32_t*>(d + Q_ZEROS + half * 128) + wl;
-            const uint4 s0 = *reinterpret_cast<const uint4*>(sc);
-            const uint4 s1 = *reinterpret_cast<const uint4*>(sc + cw * 8);
-            const uint32_t z0 = zr[0], z1 = zr[cw];
-            uint8_t* at = d + atom_off;
+          // phase A: box (wc / 8) of width 8 words; phase B: one box of 16
+          const int half = pa ? (wc >> 3) : 0;
+          const int wl = pa ? (wc & 7) : wc;
+          const int cw = pa ? 8 : 16;  // code words per K row in the box
+          // every staged input of the stage first (loads before any store, so
+          // that the rows' conversions overlap), then convert and store
+          uint32_t cv[KSUB][NRW], z[KSUB][2];
+          uint4 sv[KSUB][2];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int r = r0 + 8 * i;
-              const uint4 v = r < 32 ? awq_dequant8(codes[r * cw], z0, s0) : awq_dequant8(codes[r * cw], z1, s1);
-              const uint32_t off = uint32_t(r >> 3) * AQ_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
-              *reinterpret_cast<uint4*>(at + off) = v;
+          for (int u = 0; u < KSUB; ++u) {
+            if (u < nsub) {
+              const uint8_t* d = sub(stage, u);
+              const uint32_t* codes = reinterpret_cast<const uint32_t*>(d + Q_CODES + half * 2048) + wl;
+              const uint16_t* sc = reinterpret_cast<const uint16_t*>(d + Q_SCALES + half * 256) + wl * 8;
+              const uint32_t* zr = reinterpret_cast<const uint32_t*>(d + Q_ZEROS + half * 128) + wl;
+#pragma unroll
+              for (int i = 0; i < NRW; ++i) cv[u][i] = codes[(r0 + 16 * i) * cw];
+              sv[u][0] = *reinterpret_cast<const uint4*>(sc);
+              sv[u][1] = *reinterpret_cast<const uint4*>(sc + cw * 8);
+              z[u][0] = zr[0];
+              z[u][1] = zr[cw];
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < KSUB; ++u) {
+            if (u < nsub) {
+              uint8_t* at = sub(stage, u) + atom_off;
+              const AwqGroup g0 = awq_group(z[u][0], sv[u][0]), g1 = awq_group(z[u][1], sv[u][1]);
+#pragma unroll
+              for (int i = 0; i < NRW; ++i) {
+                const int r = r0 + 16 * i;  // rows 0..31 use group 0, 32..63 group 1
+                const uint4 v = awq_dequant8(cv[u][i], i < NRW / 2 ? g0 : g1);
+                const uint32_t off = uint32_t(r >> 3) * AQ_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
+                *reinterpret_cast<uint4*>(at + off) = v;
+              }
             }
           }
           fence_proxy_async_smem();  // the FP16 tile is read by the tensor cores

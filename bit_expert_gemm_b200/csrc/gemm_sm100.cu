@@ -432,10 +432,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ, AG>::THREADS, 1)
         const uint4 s1 = *reinterpret_cast<const uint4*>(sc + W2 * 8);
         const uint32_t z0 = zr[0], z1 = zr[W2];
         uint8_t* btile = smB(stage) + atom_off;
-#pragma unroll 4
-        for (int r = r0; r < BK; r += RP) {
-          const uint32_t w = codes[r * W2];
-          const uint4 v = r < 32 ? awq_dequant8(w, z0, s0) : awq_dequant8(w, z1, s1);
+        // the thread's code words first (loads before any store, so that the
+        // rows' conversions overlap), then convert and store
+        constexpr int NR = BK / RP;
+        uint32_t cw[NR];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) cw[i] = codes[(r0 + i * RP) * W2];
+        const AwqGroup g0 = awq_group(z0, s0), g1 = awq_group(z1, s1);
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const int r = r0 + i * RP;
+          const uint4 v = awq_dequant8(cw[i], r < 32 ? g0 : g1);
           const uint32_t off = uint32_t(r >> 3) * Cfg::B_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
           *reinterpret_cast<uint4*>(btile + off) = v;
         }
