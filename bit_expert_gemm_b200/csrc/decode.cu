@@ -51,7 +51,6 @@ constexpr int SMEM_BYTES = 217 * 1024;  // dynamic; + ~9 KB static stays under t
 constexpr int STAGE_SPACE = SMEM_BYTES - 1024 - XCHG_BYTES;
 static_assert(STAGE_SPACE >= 6 * (A_BYTES + NMAX * BK * 2), "six full stages must fit");
 constexpr int kThreads = 320;
-constexpr int kGatherThreads = 128;
 constexpr uint32_t TMEM_COLS = 2 * NMAX;  // two accumulators of 128 x NMAX
 enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
 

@@ -8,10 +8,11 @@
 // tensor in the epilogue.  Tiles: 128 rows of A x 128 rows of B, K stepped by
 // 256 elements (one 128-byte swizzle row of packed FP4), four MMAs of K = 64
 // per step.  The block scales are stored row-major ([rows, K/16] bytes) in
-// global memory; four scale-factor warps load each step's scales and write
-// them in the 32x128-bit atom layout the tensor cores read (rows r, r+32,
-// r+64, r+96 interleaved per 16-byte row), from where the UMMA warp copies
-// them into TMEM (tcgen05.cp) right before the MMAs that use them.
+// global memory; four scale-factor warps copy each step's scales (cp.async,
+// 4 bytes per row and MMA) straight into the 32x128-bit atom layout the
+// tensor cores read (rows r, r+32, r+64, r+96 interleaved per 16-byte row),
+// from where the UMMA warp copies them into TMEM (tcgen05.cp) right before
+// the MMAs that use them.
 //
 // Warp roles: 0 TMA producer, 1 UMMA issuer (TMEM owner), 2..5 epilogue,
 // 6..9 scale-factor staging.
@@ -140,20 +141,6 @@ __device__ __forceinline__ TileMap decode_tile(int L, int nt, const int* tile_st
   return t;
 }
 
-// 16 bytes of scales of row `row` for K step kt (scales 16kt .. 16kt+15),
-// zero past the row end or for rows outside the matrix.
-__device__ __forceinline__ uint4 load_sf16(const uint8_t* sf, int row, int nrows, int nsf, int kt) {
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
-  if (row >= 0 && row < nrows) {
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(sf + size_t(row) * nsf + 16 * kt);
-    const int valid = (nsf - 16 * kt) / 4;  // nsf % 4 == 0
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (j < valid) w[j] = __ldg(p + j);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_nvfp4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Args args) {
@@ -174,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&sfready_bar[s], 4);
+      mbar_init(&sfready_bar[s], 128);  // one cp.async arrival per scale-factor thread
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
@@ -291,12 +278,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_g = goff[t.g + 1] - goff[t.g];
       const size_t out_row = size_t(goff[t.g]) + size_t(t.m) * BM + row_in_tile;
       const bool valid = t.m * BM + row_in_tile < n_g && out_row < size_t(args.rows);
+      // the tile's weight global scales, loaded while the MMAs still run
+      const float gw0 = __ldg(args.gs_w + t.g * args.gs_w_stride);
+      const float gw1 = args.swiglu ? __ldg(args.gs_w + t.g * args.gs_w_stride + 1) : 0.0f;
       if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag, status, lim)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
       if (args.swiglu) {
-        const float sg = gsa * args.gs_w[t.g * args.gs_w_stride];
-        const float su = gsa * args.gs_w[t.g * args.gs_w_stride + 1];
+        const float sg = gsa * gw0;
+        const float su = gsa * gw1;
 #pragma unroll 1
         for (int c = 0; c < BN / 2 / 32; ++c) {
           float gv[32], uv[32];
@@ -305,8 +295,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f(gv[2 * i] * sg) * (uv[2 * i] * su);
-              const float h1 = silu_f(gv[2 * i + 1] * sg) * (uv[2 * i + 1] * su);
+              // h is quantised to FP4 next: the fast division is ample here
+              const float g0 = gv[2 * i] * sg, g1 = gv[2 * i + 1] * sg;
+              const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * (uv[2 * i] * su);
+              const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * (uv[2 * i + 1] * su);
               pk[i] = Pack2<__nv_bfloat16>::pack(h0, h1);
               // the amax is taken on the stored BF16 values, the ones that get quantised
               const float2 r = Pack2<__nv_bfloat16>::unpack(pk[i]);
@@ -318,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        const float sw = gsa * args.gs_w[t.g * args.gs_w_stride];
+        const float sw = gsa * gw0;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
@@ -357,8 +349,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- scale-factor staging: warps 6..9 ----------------
     // Thread st owns row st of the A tile and row st of the B tile; for each
-    // of the step's four MMAs it writes that row's 4 scales (one 32-bit word)
-    // to word (st % 32) * 4 + st / 32 of the MMA's 512-byte atom.
+    // of the step's four MMAs it copies that row's 4 scales (one 32-bit word)
+    // with cp.async straight to word (st % 32) * 4 + st / 32 of the MMA's
+    // 512-byte atom (zero for rows outside the matrix or past K), and arrives
+    // on the stage's barrier when its copies land: the loads of several
+    // stages are in flight at once.
     const int st = threadIdx.x - 192;
     const uint32_t word_off = uint32_t(((st & 31) * 4 + (st >> 5)) * 4);
     int stage = 0;
@@ -371,24 +366,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         b_row = t.g * args.b_rows_per_group + t.n * BNH + (st < BNH ? st : args.up_offset + st - BNH);
       else
         b_row = t.g * args.b_rows_per_group + t.n * BNH + st;
+      const bool a_ok = a_row >= 0 && a_row < args.a_rows, b_ok = b_row >= 0 && b_row < args.b_rows_total;
+      const uint8_t* a_src = args.sfa + (a_ok ? size_t(a_row) * nsf : 0);
+      const uint8_t* b_src = args.sfb + (b_ok ? size_t(b_row) * nsf : 0);
+      bool ok = true;
       for (int kt = 0; kt < KT; ++kt) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { L = total; break; }
-        const uint4 fa = load_sf16(args.sfa, a_row, args.a_rows, nsf, kt);
-        const uint4 fb = load_sf16(args.sfb, b_row, args.b_rows_total, nsf, kt);
-        uint8_t* s = stg(stage);
-        const uint32_t wa[4] = {fa.x, fa.y, fa.z, fa.w};
-        const uint32_t wb[4] = {fb.x, fb.y, fb.z, fb.w};
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
+        const uint32_t s = smem_u32(stg(stage));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          *reinterpret_cast<uint32_t*>(s + SFA_OFF + j * SF_ATOM + word_off) = wa[j];
-          *reinterpret_cast<uint32_t*>(s + SFB_OFF + j * SF_ATOM + word_off) = wb[j];
+          const int c = 16 * kt + 4 * j;     // first scale of this MMA's word
+          const bool in_k = c < nsf;          // nsf % 4 == 0: a word is all in or all out
+          const uint32_t na = (a_ok && in_k) ? 4u : 0u, nb = (b_ok && in_k) ? 4u : 0u;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(s + SFA_OFF + j * SF_ATOM + word_off),
+                       "l"(a_src + (na ? c : 0)), "r"(na)
+                       : "memory");
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(s + SFB_OFF + j * SF_ATOM + word_off),
+                       "l"(b_src + (nb ? c : 0)), "r"(nb)
+                       : "memory");
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sfready_bar[stage]);
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sfready_bar[stage]))
+                     : "memory");
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
+      if (!ok) break;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // every copy has landed before the CTA exits
   }
 
   tc_fence_before();

@@ -23,13 +23,20 @@ __global__ void __launch_bounds__(256) k_amax(const T16* __restrict__ v, long n,
   const uint4* p = reinterpret_cast<const uint4*>(v + b * n);
   const long nv = n / 8;
   float m = 0.0f;
-  for (long i = long(blockIdx.x) * blockDim.x + threadIdx.x; i < nv; i += long(gridDim.x) * blockDim.x) {
-    uint4 q = __ldg(p + i);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  const long step = long(gridDim.x) * blockDim.x;
+  // four independent 16-byte loads in flight per thread
+  for (long i0 = long(blockIdx.x) * blockDim.x + threadIdx.x; i0 < nv; i0 += 4 * step) {
+    uint4 q[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float2 f = Pack2<T16>::unpack(w[j]);
-      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    for (int u = 0; u < 4; ++u) q[u] = i0 + u * step < nv ? __ldg(p + i0 + u * step) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float2 f = Pack2<T16>::unpack(w[j]);
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
     }
   }
 #pragma unroll
@@ -73,6 +80,26 @@ __global__ void __launch_bounds__(256) k_nvfp4_quant(const T16* __restrict__ v, 
   const long out_row = long(b) * rows + r;
   *reinterpret_cast<uint2*>(codes + out_row * (K / 2) + blk * 8) = make_uint2(c[0], c[1]);
   sf[out_row * nb + blk] = uint8_t(s);
+}
+
+// Gathers NVFP4 rows: out row r = row row_token[r] of the codes [*, K/2] and
+// scales [*, K/16]; one warp per row (K % 64 == 0).
+__global__ void __launch_bounds__(256) k_gather_fp4_rows(const uint8_t* __restrict__ codes,
+                                                         const uint8_t* __restrict__ sf,
+                                                         const int32_t* __restrict__ row_token, int rows, int K,
+                                                         uint8_t* __restrict__ codes_out, uint8_t* __restrict__ sf_out) {
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const size_t t = size_t(row_token[r]);
+  const int nc = K / 32;  // 16-byte chunks of codes per row
+  const uint4* cs = reinterpret_cast<const uint4*>(codes + t * (K / 2));
+  uint4* cd = reinterpret_cast<uint4*>(codes_out + size_t(r) * (K / 2));
+  for (int c = lane; c < nc; c += 32) cd[c] = __ldg(cs + c);
+  const int ns = K / 64;  // 4-byte words of scales per row
+  const uint32_t* ss = reinterpret_cast<const uint32_t*>(sf + t * (K / 16));
+  uint32_t* sd = reinterpret_cast<uint32_t*>(sf_out + size_t(r) * (K / 16));
+  for (int c = lane; c < ns; c += 32) sd[c] = __ldg(ss + c);
 }
 
 // amax_n > 0: reduce amax over the first amax_n values of each tensor
@@ -131,7 +158,7 @@ int nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const f
 //   -> quantise h -> GEMM2.
 // ---------------------------------------------------------------------------
 struct Nvfp4Ws {
-  uint8_t *xq, *xsf, *hq, *hsf;
+  uint8_t *xq, *xsf, *xq_tok, *xsf_tok, *hq, *hsf;
   uint16_t* h;
   unsigned* amax;  // [2]: x, h
   float* gs;       // [2]: x, h
@@ -139,6 +166,9 @@ struct Nvfp4Ws {
 
 template <typename C>
 static void carve_nvfp4(C& c, int rows, int H, int I) {
+  c.template take<uint8_t>(size_t(rows) * H / 2);
+  c.template take<uint8_t>(size_t(rows) * H / 16);
+  // per-token codes and scales of x: T <= rows tokens
   c.template take<uint8_t>(size_t(rows) * H / 2);
   c.template take<uint8_t>(size_t(rows) * H / 16);
   c.template take<uint8_t>(size_t(rows) * I / 2);
@@ -163,6 +193,8 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
   Nvfp4Ws w;
   w.xq = carve.take<uint8_t>(size_t(rows) * H / 2);
   w.xsf = carve.take<uint8_t>(size_t(rows) * H / 16);
+  w.xq_tok = carve.take<uint8_t>(size_t(T) * H / 2);
+  w.xsf_tok = carve.take<uint8_t>(size_t(T) * H / 16);
   w.hq = carve.take<uint8_t>(size_t(rows) * I / 2);
   w.hsf = carve.take<uint8_t>(size_t(rows) * I / 16);
   w.h = carve.take<uint16_t>(size_t(rows) * I);
@@ -170,10 +202,18 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
   w.gs = carve.take<float>(2);
   MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_grouped_swiglu_nvfp4: workspace of %zu bytes is too small", ws_bytes);
   if (rows == 0) return MOE_OK;
-  // x: amax over the whole [T, H] input, quantise the gathered rows
-  int rc = quantize_rows(x, MOE_DTYPE_BF16, row_token, 1, rows, H, 0, long(T) * H, act_gs_in, w.amax, w.xq, w.xsf,
-                         w.gs, stream);
+  // x: amax over the whole [T, H] input, each token quantised once, then the
+  // FP4 rows gathered in permuted order (identical to quantising the gathered
+  // rows: the quantisation is per row with the one global scale of x)
+  // (identity rows, row_token == NULL: quantised in place, no gather)
+  int rc = quantize_rows(x, MOE_DTYPE_BF16, nullptr, 1, T, H, 0, long(T) * H, act_gs_in, w.amax,
+                         row_token ? w.xq_tok : w.xq, row_token ? w.xsf_tok : w.xsf, w.gs, stream);
   if (rc) return rc;
+  if (row_token) {
+    k_gather_fp4_rows<<<(rows * 32 + 255) / 256, 256, 0, stream>>>(w.xq_tok, w.xsf_tok, row_token, rows, H, w.xq,
+                                                                    w.xsf);
+    MOE_CHECK_CUDA(cudaGetLastError());
+  }
   MOE_CHECK_CUDA(cudaMemsetAsync(w.amax + 1, 0, sizeof(unsigned), stream));
   rc = launch_grouped_gemm_nvfp4(w.xq, w.xsf, rows, w_gu, sf_gu, E * 2 * I, offsets, E, rows, H, I, 2 * I, I, 1, w.gs,
                                  gs_gu, 2, w.h, I, 0, reinterpret_cast<float*>(w.amax + 1), stream);
