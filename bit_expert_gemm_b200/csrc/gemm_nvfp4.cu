@@ -7,15 +7,14 @@
 // then scaled by the FP32 global scales of the activation and of the weight
 // tensor in the epilogue.  Tiles: 128 rows of A x 128 rows of B, K stepped by
 // 256 elements (one 128-byte swizzle row of packed FP4), four MMAs of K = 64
-// per step.  The block scales are stored row-major ([rows, K/16] bytes) in
-// global memory; four scale-factor warps copy each step's scales (cp.async,
-// 4 bytes per row and MMA) straight into the 32x128-bit atom layout the
-// tensor cores read (rows r, r+32, r+64, r+96 interleaved per 16-byte row),
-// from where the UMMA warp copies them into TMEM (tcgen05.cp) right before
-// the MMAs that use them.
+// per step.  The block scales arrive already in operand-tile order (nvfp4.cu
+// k_pack_sf_a / k_pack_sf_b): per 128-row tile and K step, four 512-byte
+// atoms in the 32x128-bit layout the tensor cores read (rows r, r+32, r+64,
+// r+96 interleaved per 16-byte row), fetched with one 2 KB bulk copy per
+// operand on the stage's barrier; the UMMA warp copies them into TMEM
+// (tcgen05.cp) right before the MMAs that use them.
 //
-// Warp roles: 0 TMA producer, 1 UMMA issuer (TMEM owner), 2..5 epilogue,
-// 6..9 scale-factor staging.
+// Warp roles: 0 TMA producer, 1 UMMA issuer (TMEM owner), 2..5 epilogue.
 #include <cstring>
 
 #include "common.cuh"
@@ -39,7 +38,8 @@ constexpr int SFB_OFF = SFA_OFF + 4 * SF_ATOM;
 constexpr int STAGE_BYTES = SFB_OFF + 4 * SF_ATOM;  // 36 KB
 constexpr int STAGES = 5;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-constexpr int kThreads = 320;
+constexpr int kThreads = 192;
+constexpr int SF_TILE = 4 * SF_ATOM;     // scales of one operand tile for one K step
 constexpr uint32_t TMEM_COLS = 512;      // 2 x 128 accumulator + scale factors
 constexpr uint32_t SFA_COL = 2 * BN;     // 4 MMAs x 4 columns
 constexpr uint32_t SFB_COL = SFA_COL + 16;
@@ -48,8 +48,8 @@ static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
 struct Args {
   const int* group_offsets;
   int G, rows, K, n_out, b_rows_per_group, up_offset, swiglu;
-  const uint8_t* sfa;  // [a_rows, K/16]
-  const uint8_t* sfb;  // [b_rows_total, K/16]
+  const uint8_t* sfa;  // A tiles (tile_start[g] + m) x K steps x SF_TILE
+  const uint8_t* sfb;  // B tiles (g * n_tiles + n) x K steps x SF_TILE
   int a_rows, b_rows_total;
   const float* gs_act;  // device scalar
   const float* gs_w;    // [G * gs_w_stride]
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_nvfp4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Args args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], sfready_bar[STAGES], tfull_bar[2],
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[2],
       tempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
@@ -161,7 +161,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&sfready_bar[s], 128);  // one cp.async arrival per scale-factor thread
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
@@ -190,7 +189,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nt = args.n_out / BNH;
   const int total = tile_start[G] * nt;
   const int KT = (args.K + BKE - 1) / BKE;
-  const int nsf = args.K / 16;
   int* status = args.status;
   const unsigned long long lim = args.limit_ns;
 
@@ -207,8 +205,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b_row = t.g * args.b_rows_per_group + t.n * BNH;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], A_BYTES + B_BYTES);
+          mbar_arrive_expect_tx(&full_bar[stage], A_BYTES + B_BYTES + 2 * SF_TILE);
           tma_load_2d(stg(stage), &tmA, &full_bar[stage], kt * BKB, a_row);
+          bulk_load(stg(stage) + SFA_OFF, args.sfa + (size_t(tile_start[t.g] + t.m) * KT + kt) * SF_TILE, SF_TILE,
+                    &full_bar[stage]);
+          bulk_load(stg(stage) + SFB_OFF, args.sfb + (size_t(t.g * nt + t.n) * KT + kt) * SF_TILE, SF_TILE,
+                    &full_bar[stage]);
           if (args.swiglu) {
             tma_load_2d(stg(stage) + A_BYTES, &tmB, &full_bar[stage], kt * BKB, b_row);
             tma_load_2d(stg(stage) + A_BYTES + BNH * BKB, &tmB, &full_bar[stage], kt * BKB, b_row + args.up_offset);
@@ -239,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem_base + uint32_t(acc * BN);
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
-          if (!mbar_wait(&sfready_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sbase = smem_u32(stg(stage));
 #pragma unroll
@@ -346,52 +347,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
       if (lane == 0) atomicMax(reinterpret_cast<unsigned*>(args.amax_out), __float_as_uint(hmax));
     }
-  } else {
-    // ---------------- scale-factor staging: warps 6..9 ----------------
-    // Thread st owns row st of the A tile and row st of the B tile; for each
-    // of the step's four MMAs it copies that row's 4 scales (one 32-bit word)
-    // with cp.async straight to word (st % 32) * 4 + st / 32 of the MMA's
-    // 512-byte atom (zero for rows outside the matrix or past K), and arrives
-    // on the stage's barrier when its copies land: the loads of several
-    // stages are in flight at once.
-    const int st = threadIdx.x - 192;
-    const uint32_t word_off = uint32_t(((st & 31) * 4 + (st >> 5)) * 4);
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
-      TileMap t = decode_tile(L, nt, tile_start, G);
-      const int a_row = goff[t.g] + t.m * BM + st;
-      int b_row;
-      if (args.swiglu)
-        b_row = t.g * args.b_rows_per_group + t.n * BNH + (st < BNH ? st : args.up_offset + st - BNH);
-      else
-        b_row = t.g * args.b_rows_per_group + t.n * BNH + st;
-      const bool a_ok = a_row >= 0 && a_row < args.a_rows, b_ok = b_row >= 0 && b_row < args.b_rows_total;
-      const uint8_t* a_src = args.sfa + (a_ok ? size_t(a_row) * nsf : 0);
-      const uint8_t* b_src = args.sfb + (b_ok ? size_t(b_row) * nsf : 0);
-      bool ok = true;
-      for (int kt = 0; kt < KT; ++kt) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
-        const uint32_t s = smem_u32(stg(stage));
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = 16 * kt + 4 * j;     // first scale of this MMA's word
-          const bool in_k = c < nsf;          // nsf % 4 == 0: a word is all in or all out
-          const uint32_t na = (a_ok && in_k) ? 4u : 0u, nb = (b_ok && in_k) ? 4u : 0u;
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(s + SFA_OFF + j * SF_ATOM + word_off),
-                       "l"(a_src + (na ? c : 0)), "r"(na)
-                       : "memory");
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(s + SFB_OFF + j * SF_ATOM + word_off),
-                       "l"(b_src + (nb ? c : 0)), "r"(nb)
-                       : "memory");
-        }
-        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sfready_bar[stage]))
-                     : "memory");
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
-      }
-      if (!ok) break;
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");  // every copy has landed before the CTA exits
   }
 
   tc_fence_before();

@@ -102,6 +102,84 @@ __global__ void __launch_bounds__(256) k_gather_fp4_rows(const uint8_t* __restri
   for (int c = lane; c < ns; c += 32) sd[c] = __ldg(ss + c);
 }
 
+// ---------------------------------------------------------------------------
+// Scale factors in the block-scaled GEMM's operand-tile order.  For operand
+// tile t (128 rows) and K step kt (256 elements = 16 scales per row): four
+// 512-byte atoms, one per MMA of K = 64; in atom j, 16-byte row i holds the
+// scales 16kt + 4j .. 16kt + 4j + 3 of tile rows i, i + 32, i + 64, i + 96
+// (one 32-bit word each), the layout tcgen05.cp copies into TMEM.  Rows
+// outside the operand and scales past K are zero.  The GEMM then fetches a
+// stage's scales with one 2 KB bulk copy per operand.
+// ---------------------------------------------------------------------------
+constexpr int kSfTileBytes = 2048;
+
+__device__ __forceinline__ void pack_sf_row(const uint8_t* sf, int nsf, bool valid, size_t row, int kt, int i,
+                                            uint8_t* tile) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = 16 * kt + 4 * j;
+    const uint32_t w = (valid && c < nsf) ? __ldg(reinterpret_cast<const uint32_t*>(sf + row * nsf + c)) : 0u;
+    *reinterpret_cast<uint32_t*>(tile + j * 512 + (i & 31) * 16 + (i >> 5) * 4) = w;
+  }
+}
+
+// tile_start[g] = 128-row tiles of groups 0..g-1 (groups from offsets [G+1]); one block
+__global__ void __launch_bounds__(1024) k_tile_starts(const int32_t* __restrict__ offsets, int G,
+                                                      int32_t* __restrict__ tile_start) {
+  __shared__ int warp_tot[32];
+  const int per = (G + 1023) / 1024;
+  const int g0 = threadIdx.x * per;
+  int local = 0;
+  for (int g = g0; g < g0 + per && g < G; ++g) local += (offsets[g + 1] - offsets[g] + 127) / 128;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int run = incl - local;
+  for (int w = 0; w < warp; ++w) run += warp_tot[w];
+  for (int g = g0; g < g0 + per && g < G; ++g) {
+    tile_start[g] = run;
+    run += (offsets[g + 1] - offsets[g] + 127) / 128;
+  }
+  if (threadIdx.x == 1023) tile_start[G] = run;
+}
+
+// A operand (activations in permuted row order): tile t is rows
+// offsets[g] + 128 m .. of group g, t = tile_start[g] + m.  Grid (max tiles,
+// KT), 128 threads (one per tile row).
+__global__ void __launch_bounds__(128) k_pack_sf_a(const uint8_t* __restrict__ sf, int K,
+                                                   const int32_t* __restrict__ offsets, int G,
+                                                   const int32_t* __restrict__ tile_start, uint8_t* __restrict__ out) {
+  const int t = blockIdx.x, kt = blockIdx.y, i = threadIdx.x;
+  if (t >= tile_start[G]) return;
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  const int m = t - tile_start[lo];
+  const long row = long(offsets[lo]) + long(m) * 128 + i;
+  pack_sf_row(sf, K / 16, row < offsets[lo + 1], size_t(row), kt, i,
+              out + (size_t(t) * gridDim.y + kt) * kSfTileBytes);
+}
+
+// B operand (weights): tile (g, n) is, for SwiGLU, the 64 gate rows n*64.. and
+// the 64 up rows up_offset + n*64.. of group g, else the 128 rows n*128...
+// Grid (G * nt, KT), 128 threads.
+__global__ void __launch_bounds__(128) k_pack_sf_b(const uint8_t* __restrict__ sf, int K, int nt, int rows_per_group,
+                                                   int swiglu, int up_offset, uint8_t* __restrict__ out) {
+  const int tile = blockIdx.x, kt = blockIdx.y, i = threadIdx.x;
+  const int g = tile / nt, n = tile - g * nt;
+  const int r = swiglu ? (i < 64 ? n * 64 + i : up_offset + n * 64 + i - 64) : n * 128 + i;
+  pack_sf_row(sf, K / 16, r < rows_per_group, size_t(g) * rows_per_group + r, kt, i,
+              out + (size_t(tile) * gridDim.y + kt) * kSfTileBytes);
+}
+
 // amax_n > 0: reduce amax over the first amax_n values of each tensor
 // first; amax_n == 0: amax already holds it (or gs_in is given).
 template <typename T16>
@@ -154,11 +232,14 @@ int nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const f
 
 // ---------------------------------------------------------------------------
 // Grouped SwiGLU with NVFP4 weights and on-the-fly NVFP4 activations:
-//   amax(x) -> quantise gathered rows -> GEMM1 (+SwiGLU, h in BF16, amax(h))
-//   -> quantise h -> GEMM2.
+//   amax(x) -> quantise each token -> gather the FP4 rows -> scales in tile
+//   order -> GEMM1 (+SwiGLU, h in BF16, amax(h)) -> quantise h -> scales in
+//   tile order -> GEMM2.
 // ---------------------------------------------------------------------------
 struct Nvfp4Ws {
   uint8_t *xq, *xsf, *xq_tok, *xsf_tok, *hq, *hsf;
+  int32_t* tile_start;                 // [E+1] 128-row tiles before each group
+  uint8_t *xsf_p, *hsf_p, *w1sf_p, *w2sf_p;  // scales in GEMM tile order
   uint16_t* h;
   unsigned* amax;  // [2]: x, h
   float* gs;       // [2]: x, h
@@ -178,10 +259,23 @@ static void carve_nvfp4(C& c, int rows, int H, int I) {
   c.template take<float>(2);
 }
 
+// Tile-ordered scale factors: A tiles of the permuted rows (at most
+// ceil(rows/128) + E), B tiles of every expert's weights.
+template <typename C>
+static void carve_nvfp4_packed(C& c, int rows, int H, int I, int E) {
+  const size_t tiles = size_t(rows + 127) / 128 + E;
+  const size_t kt1 = (H + 255) / 256, kt2 = (I + 255) / 256;
+  c.template take<int32_t>(size_t(E) + 1);
+  c.template take<uint8_t>(tiles * kt1 * kSfTileBytes);
+  c.template take<uint8_t>(tiles * kt2 * kSfTileBytes);
+  c.template take<uint8_t>(size_t(E) * (I / 64) * kt1 * kSfTileBytes);
+  c.template take<uint8_t>(size_t(E) * (H / 128) * kt2 * kSfTileBytes);
+}
+
 size_t nvfp4_ws_bytes(int rows, int H, int I, int E) {
-  (void)E;
   WsCounter c;
   carve_nvfp4(c, rows, H, I);
+  carve_nvfp4_packed(c, rows, H, I, E);
   return c.used;
 }
 
@@ -200,6 +294,15 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
   w.h = carve.take<uint16_t>(size_t(rows) * I);
   w.amax = carve.take<unsigned>(2);
   w.gs = carve.take<float>(2);
+  {
+    const size_t tiles = size_t(rows + 127) / 128 + E;
+    const size_t kt1 = (H + 255) / 256, kt2 = (I + 255) / 256;
+    w.tile_start = carve.take<int32_t>(size_t(E) + 1);
+    w.xsf_p = carve.take<uint8_t>(tiles * kt1 * kSfTileBytes);
+    w.hsf_p = carve.take<uint8_t>(tiles * kt2 * kSfTileBytes);
+    w.w1sf_p = carve.take<uint8_t>(size_t(E) * (I / 64) * kt1 * kSfTileBytes);
+    w.w2sf_p = carve.take<uint8_t>(size_t(E) * (H / 128) * kt2 * kSfTileBytes);
+  }
   MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_grouped_swiglu_nvfp4: workspace of %zu bytes is too small", ws_bytes);
   if (rows == 0) return MOE_OK;
   // x: amax over the whole [T, H] input, each token quantised once, then the
@@ -214,15 +317,25 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
                                                                     w.xsf);
     MOE_CHECK_CUDA(cudaGetLastError());
   }
+  // scale factors in GEMM tile order: A tiles of the permuted rows, B tiles of the weights
+  const int tiles = (rows + 127) / 128 + E;
+  const int kt1 = (H + 255) / 256, kt2 = (I + 255) / 256;
+  k_tile_starts<<<1, 1024, 0, stream>>>(offsets, E, w.tile_start);
+  k_pack_sf_a<<<dim3(tiles, kt1), 128, 0, stream>>>(w.xsf, H, offsets, E, w.tile_start, w.xsf_p);
+  k_pack_sf_b<<<dim3(E * (I / 64), kt1), 128, 0, stream>>>(sf_gu, H, I / 64, 2 * I, 1, I, w.w1sf_p);
+  MOE_CHECK_CUDA(cudaGetLastError());
   MOE_CHECK_CUDA(cudaMemsetAsync(w.amax + 1, 0, sizeof(unsigned), stream));
-  rc = launch_grouped_gemm_nvfp4(w.xq, w.xsf, rows, w_gu, sf_gu, E * 2 * I, offsets, E, rows, H, I, 2 * I, I, 1, w.gs,
-                                 gs_gu, 2, w.h, I, 0, reinterpret_cast<float*>(w.amax + 1), stream);
+  rc = launch_grouped_gemm_nvfp4(w.xq, w.xsf_p, rows, w_gu, w.w1sf_p, E * 2 * I, offsets, E, rows, H, I, 2 * I, I, 1,
+                                 w.gs, gs_gu, 2, w.h, I, 0, reinterpret_cast<float*>(w.amax + 1), stream);
   if (rc) return rc;
   rc = quantize_rows(w.h, MOE_DTYPE_BF16, nullptr, 1, rows, I, 0, 0, act_gs_in ? act_gs_in + 1 : nullptr, w.amax + 1,
                      w.hq, w.hsf, w.gs + 1, stream);
   if (rc) return rc;
-  rc = launch_grouped_gemm_nvfp4(w.hq, w.hsf, rows, w_d, sf_d, E * H, offsets, E, rows, I, H, H, 0, 0, w.gs + 1, gs_d,
-                                 1, f, H, out_fp32, nullptr, stream);
+  k_pack_sf_a<<<dim3(tiles, kt2), 128, 0, stream>>>(w.hsf, I, offsets, E, w.tile_start, w.hsf_p);
+  k_pack_sf_b<<<dim3(E * (H / 128), kt2), 128, 0, stream>>>(sf_d, I, H / 128, H, 0, 0, w.w2sf_p);
+  MOE_CHECK_CUDA(cudaGetLastError());
+  rc = launch_grouped_gemm_nvfp4(w.hq, w.hsf_p, rows, w_d, w.w2sf_p, E * H, offsets, E, rows, I, H, H, 0, 0, w.gs + 1,
+                                 gs_d, 1, f, H, out_fp32, nullptr, stream);
   if (rc) return rc;
   if (act_gs_out) MOE_CHECK_CUDA(cudaMemcpyAsync(act_gs_out, w.gs, 2 * sizeof(float), cudaMemcpyDeviceToDevice, stream));
   return MOE_OK;
