@@ -57,6 +57,10 @@ _SIGS = {
     "moe_nvfp4_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_grouped_swiglu_nvfp4": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ,
                                       _P]),
+    "moe_nvfp4_packed_sf_bytes": (_SZ, [_I, _I, _I, _I]),
+    "moe_nvfp4_prepack_sf": (_I, [_P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "moe_grouped_swiglu_nvfp4_prepacked": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I,
+                                                _P, _P, _SZ, _P]),
     "moe_combine": (_I, [_P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "razor_refill_rms_accumulate": (_I, [_P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "razor_select": (_I, [_P, _P, _I, _I, _P, _P, _P, _P]),
@@ -346,6 +350,36 @@ def moe_grouped_swiglu_nvfp4(x, row_token, expert_offsets, rows: int, w_gu, sf_g
     _call("moe_grouped_swiglu_nvfp4", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E, _p(w_gu),
           _p(sf_gu), _p(gs_gu), _p(w_d), _p(sf_d), _p(gs_d), _p(act_gs_in), _p(act_gs_out), int(out_fp32), _p(f),
           _p(ws), ws.numel(), _stream(stream))
+    return f
+
+
+def moe_nvfp4_prepack_sf(sf, swiglu: bool, out=None, stream=None):
+    """Rearrange one projection's weight scales sf [E, rows, K/16] into the FP4 GEMM's tile order."""
+    E, R, K16 = sf.shape
+    K = K16 * 16
+    nbytes = int(load().moe_nvfp4_packed_sf_bytes(E, R, K, int(swiglu)))
+    if nbytes == 0:
+        raise ValueError(f"moe_nvfp4_prepack_sf: unsupported sizes E={E} rows={R} K={K}")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=sf.device)
+    _call("moe_nvfp4_prepack_sf", _p(sf), E, R, K, int(swiglu), _p(out), out.numel(), _stream(stream))
+    return out
+
+
+def moe_grouped_swiglu_nvfp4_prepacked(x, row_token, expert_offsets, rows: int, w_gu, sf_gu_packed, gs_gu, w_d,
+                                       sf_d_packed, gs_d, act_gs_in=None, act_gs_out=None, out_fp32: bool = False,
+                                       f=None, ws=None, stream=None):
+    T, H = x.shape
+    E = w_gu.shape[0]
+    I = w_gu.shape[1] // 2
+    dev = x.device
+    if f is None:
+        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=dev)
+    if ws is None:
+        ws = workspace(MOE_OP_SWIGLU_NVFP4, rows, H, E, 1, I, dev)
+    _call("moe_grouped_swiglu_nvfp4_prepacked", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E,
+          _p(w_gu), _p(sf_gu_packed), _p(gs_gu), _p(w_d), _p(sf_d_packed), _p(gs_d), _p(act_gs_in),
+          _p(act_gs_out), int(out_fp32), _p(f), _p(ws), ws.numel(), _stream(stream))
     return f
 
 

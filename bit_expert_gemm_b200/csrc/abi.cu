@@ -58,7 +58,11 @@ size_t nvfp4_ws_bytes(int rows, int H, int I, int E);
 int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
                          int I, int E, const uint8_t* w_gu, const uint8_t* sf_gu, const float* gs_gu,
                          const uint8_t* w_d, const uint8_t* sf_d, const float* gs_d, const float* act_gs_in,
-                         float* act_gs_out, int out_fp32, void* f, void* ws, size_t ws_bytes, cudaStream_t stream);
+                         float* act_gs_out, int out_fp32, void* f, void* ws, size_t ws_bytes, cudaStream_t stream,
+                         const uint8_t* w1sf_packed, const uint8_t* w2sf_packed);
+size_t nvfp4_packed_sf_bytes(int E, int rows_per_expert, int K, int swiglu);
+int nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, int K, int swiglu, uint8_t* out,
+                     cudaStream_t stream);
 
 namespace {
 thread_local char g_err[1024] = "";
@@ -480,7 +484,46 @@ int moe_grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int3
   MOE_REQUIRE(x && expert_offsets && w_gu && sf_gu && gs_gu && w_d && sf_d && gs_d && f, MOE_ERR_INVALID_ARG,
               "moe_grouped_swiglu_nvfp4: null pointer");
   return grouped_swiglu_nvfp4(x, row_token, expert_offsets, T, rows, H, I, E, w_gu, sf_gu, gs_gu, w_d, sf_d, gs_d,
-                              act_gs_in, act_gs_out, out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+                              act_gs_in, act_gs_out, out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                              nullptr, nullptr);
+}
+
+size_t moe_nvfp4_packed_sf_bytes(int E, int rows_per_expert, int K, int swiglu) {
+  if (E < 1 || rows_per_expert <= 0 || K <= 0 || rows_per_expert % 128 || K % 128) return 0;
+  return nvfp4_packed_sf_bytes(E, rows_per_expert, K, swiglu);
+}
+
+int moe_nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, int K, int swiglu, uint8_t* out,
+                         size_t out_bytes, void* stream) {
+  MOE_REQUIRE(E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG, "moe_nvfp4_prepack_sf: E=%d", E);
+  MOE_REQUIRE(rows_per_expert > 0 && K > 0 && rows_per_expert % 128 == 0 && K % 128 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_nvfp4_prepack_sf: rows_per_expert=%d and K=%d must be positive multiples of 128",
+              rows_per_expert, K);
+  MOE_REQUIRE(swiglu == 0 || swiglu == 1, MOE_ERR_INVALID_ARG, "moe_nvfp4_prepack_sf: swiglu=%d", swiglu);
+  MOE_REQUIRE(sf && out, MOE_ERR_INVALID_ARG, "moe_nvfp4_prepack_sf: null pointer");
+  const size_t need = nvfp4_packed_sf_bytes(E, rows_per_expert, K, swiglu);
+  MOE_REQUIRE(out_bytes >= need, MOE_ERR_WORKSPACE, "moe_nvfp4_prepack_sf: out holds %zu bytes, need %zu",
+              out_bytes, need);
+  return nvfp4_prepack_sf(sf, E, rows_per_expert, K, swiglu, out, static_cast<cudaStream_t>(stream));
+}
+
+int moe_grouped_swiglu_nvfp4_prepacked(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
+                                       int rows, int H, int I, int E, const uint8_t* w_gu, const uint8_t* sf_gu_packed,
+                                       const float* gs_gu, const uint8_t* w_d, const uint8_t* sf_d_packed,
+                                       const float* gs_d, const float* act_gs_in, float* act_gs_out, int out_fp32,
+                                       void* f, void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_nvfp4_prepacked: bad sizes");
+  MOE_REQUIRE(H > 0 && I > 0 && H % 128 == 0 && I % 128 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_grouped_swiglu_nvfp4_prepacked: H=%d and I=%d must be positive multiples of 128", H, I);
+  MOE_REQUIRE(row_token || rows == T, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_nvfp4_prepacked: without row_token rows must equal T");
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(x && expert_offsets && w_gu && sf_gu_packed && gs_gu && w_d && sf_d_packed && gs_d && f,
+              MOE_ERR_INVALID_ARG, "moe_grouped_swiglu_nvfp4_prepacked: null pointer");
+  return grouped_swiglu_nvfp4(x, row_token, expert_offsets, T, rows, H, I, E, w_gu, nullptr, gs_gu, w_d, nullptr, gs_d,
+                              act_gs_in, act_gs_out, out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                              sf_gu_packed, sf_d_packed);
 }
 
 int moe_combine(const void* f, int f_fp32, const int32_t* slot_row, int k_slots, const float* topk_w,

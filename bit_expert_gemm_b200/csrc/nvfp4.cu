@@ -282,7 +282,8 @@ size_t nvfp4_ws_bytes(int rows, int H, int I, int E) {
 int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
                          int I, int E, const uint8_t* w_gu, const uint8_t* sf_gu, const float* gs_gu,
                          const uint8_t* w_d, const uint8_t* sf_d, const float* gs_d, const float* act_gs_in,
-                         float* act_gs_out, int out_fp32, void* f, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                         float* act_gs_out, int out_fp32, void* f, void* ws, size_t ws_bytes, cudaStream_t stream,
+                         const uint8_t* w1sf_packed, const uint8_t* w2sf_packed) {
   WsCarver carve(ws, ws_bytes);
   Nvfp4Ws w;
   w.xq = carve.take<uint8_t>(size_t(rows) * H / 2);
@@ -322,22 +323,48 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
   const int kt1 = (H + 255) / 256, kt2 = (I + 255) / 256;
   k_tile_starts<<<1, 1024, 0, stream>>>(offsets, E, w.tile_start);
   k_pack_sf_a<<<dim3(tiles, kt1), 128, 0, stream>>>(w.xsf, H, offsets, E, w.tile_start, w.xsf_p);
-  k_pack_sf_b<<<dim3(E * (I / 64), kt1), 128, 0, stream>>>(sf_gu, H, I / 64, 2 * I, 1, I, w.w1sf_p);
+  const uint8_t* w1sf = w1sf_packed;
+  if (!w1sf) {  // weight scales not packed by the caller: pack them for this call
+    k_pack_sf_b<<<dim3(E * (I / 64), kt1), 128, 0, stream>>>(sf_gu, H, I / 64, 2 * I, 1, I, w.w1sf_p);
+    w1sf = w.w1sf_p;
+  }
   MOE_CHECK_CUDA(cudaGetLastError());
   MOE_CHECK_CUDA(cudaMemsetAsync(w.amax + 1, 0, sizeof(unsigned), stream));
-  rc = launch_grouped_gemm_nvfp4(w.xq, w.xsf_p, rows, w_gu, w.w1sf_p, E * 2 * I, offsets, E, rows, H, I, 2 * I, I, 1,
+  rc = launch_grouped_gemm_nvfp4(w.xq, w.xsf_p, rows, w_gu, w1sf, E * 2 * I, offsets, E, rows, H, I, 2 * I, I, 1,
                                  w.gs, gs_gu, 2, w.h, I, 0, reinterpret_cast<float*>(w.amax + 1), stream);
   if (rc) return rc;
   rc = quantize_rows(w.h, MOE_DTYPE_BF16, nullptr, 1, rows, I, 0, 0, act_gs_in ? act_gs_in + 1 : nullptr, w.amax + 1,
                      w.hq, w.hsf, w.gs + 1, stream);
   if (rc) return rc;
   k_pack_sf_a<<<dim3(tiles, kt2), 128, 0, stream>>>(w.hsf, I, offsets, E, w.tile_start, w.hsf_p);
-  k_pack_sf_b<<<dim3(E * (H / 128), kt2), 128, 0, stream>>>(sf_d, I, H / 128, H, 0, 0, w.w2sf_p);
+  const uint8_t* w2sf = w2sf_packed;
+  if (!w2sf) {
+    k_pack_sf_b<<<dim3(E * (H / 128), kt2), 128, 0, stream>>>(sf_d, I, H / 128, H, 0, 0, w.w2sf_p);
+    w2sf = w.w2sf_p;
+  }
   MOE_CHECK_CUDA(cudaGetLastError());
-  rc = launch_grouped_gemm_nvfp4(w.hq, w.hsf_p, rows, w_d, w.w2sf_p, E * H, offsets, E, rows, I, H, H, 0, 0, w.gs + 1,
+  rc = launch_grouped_gemm_nvfp4(w.hq, w.hsf_p, rows, w_d, w2sf, E * H, offsets, E, rows, I, H, H, 0, 0, w.gs + 1,
                                  gs_d, 1, f, H, out_fp32, nullptr, stream);
   if (rc) return rc;
   if (act_gs_out) MOE_CHECK_CUDA(cudaMemcpyAsync(act_gs_out, w.gs, 2 * sizeof(float), cudaMemcpyDeviceToDevice, stream));
+  return MOE_OK;
+}
+
+// Weight scales [E, rows_per_expert, K/16] in the FP4 GEMM's B-tile order:
+// SwiGLU (gate/up) projections pair 64 gate rows n*64.. with the 64 up rows
+// up_offset + n*64..; other projections take 128 rows per tile.
+size_t nvfp4_packed_sf_bytes(int E, int rows_per_expert, int K, int swiglu) {
+  (void)swiglu;  // both orders put 128 rows in a tile
+  const size_t nt = size_t(rows_per_expert) / 128;
+  return size_t(E) * nt * ((K + 255) / 256) * kSfTileBytes;
+}
+
+int nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, int K, int swiglu, uint8_t* out,
+                     cudaStream_t stream) {
+  const int kt = (K + 255) / 256;
+  const int nt = rows_per_expert / 128;  // SwiGLU: I/64 tiles of 64 gate + 64 up rows (rows_per_expert = 2I)
+  k_pack_sf_b<<<dim3(E * nt, kt), 128, 0, stream>>>(sf, K, nt, rows_per_expert, swiglu, rows_per_expert / 2, out);
+  MOE_CHECK_CUDA(cudaGetLastError());
   return MOE_OK;
 }
 

@@ -48,7 +48,9 @@ def prepare_nvfp4_weights(w: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]
     library (moe_nvfp4_quantize): gate, up and down of every expert are
     separate tensors with their own global scale.
     w_gu [E, 2I, H/2], sf_gu [E, 2I, H/16], gs_gu [E, 2]; w_d [E, H, I/2],
-    sf_d [E, H, I/16], gs_d [E]."""
+    sf_d [E, H, I/16], gs_d [E].  The weight scales are also rearranged once
+    into the FP4 GEMM's tile order (sfp_gu, sfp_d: moe_nvfp4_prepack_sf), so the
+    layer's calls do not redo it every step."""
     gu, wd = w["w_gate_up"], w["w_down"]
     E, I2, H = gu.shape
     I = I2 // 2
@@ -57,6 +59,8 @@ def prepare_nvfp4_weights(w: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]
     out["w_gu"], out["sf_gu"], out["gs_gu"] = c.reshape(E, I2, H // 2), sf.reshape(E, I2, H // 16), gs.reshape(E, 2)
     c, sf, gs = abi.moe_nvfp4_quantize(wd)
     out["w_d"], out["sf_d"], out["gs_d"] = c, sf, gs
+    out["sfp_gu"] = abi.moe_nvfp4_prepack_sf(out["sf_gu"], swiglu=True)
+    out["sfp_d"] = abi.moe_nvfp4_prepack_sf(out["sf_d"], swiglu=False)
     return out
 
 
@@ -146,9 +150,10 @@ class MoELayer:
                                            w["sc_gu"], w["qw_d"], w["qz_d"], w["sc_d"],
                                            out_fp32=f.dtype == torch.float32, f=f, ws=self.ws_ffn)
         else:
-            abi.moe_grouped_swiglu_nvfp4(x, self.row_token[:rows], self.offsets, rows, w["w_gu"], w["sf_gu"],
-                                         w["gs_gu"], w["w_d"], w["sf_d"], w["gs_d"], act_gs_in=w.get("act_gs"),
-                                         out_fp32=f.dtype == torch.float32, f=f, ws=self.ws_ffn)
+            abi.moe_grouped_swiglu_nvfp4_prepacked(x, self.row_token[:rows], self.offsets, rows, w["w_gu"],
+                                                   w["sfp_gu"], w["gs_gu"], w["w_d"], w["sfp_d"], w["gs_d"],
+                                                   act_gs_in=w.get("act_gs"), out_fp32=f.dtype == torch.float32,
+                                                   f=f, ws=self.ws_ffn)
         return f
 
     def shared_expert(self, x: torch.Tensor) -> torch.Tensor:

@@ -307,6 +307,41 @@ MOE_API int moe_grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, co
                              size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Weight block scales of one NVFP4 projection, rearranged once into the order
+ * in which the FP4 GEMM's B tiles read them, so that moe_grouped_swiglu_nvfp4
+ * need not rearrange static scales on every call [NVFP4] (the scale values
+ * are unchanged: this is layout only).
+ * sf [E, rows_per_expert, K/16] uint8 E4M3 (moe_nvfp4_quantize's layout);
+ * swiglu = 1 for a gate/up projection whose rows are [gate I | up I]
+ * (rows_per_expert = 2I, each tile pairs 64 gate with the matching 64 up
+ * rows), 0 for a plain projection (128 consecutive rows per tile).
+ * out: device buffer of moe_nvfp4_packed_sf_bytes(...) bytes, owned by the
+ * caller; the layout is opaque and is only read by
+ * moe_grouped_swiglu_nvfp4_prepacked.  moe_nvfp4_packed_sf_bytes returns 0
+ * for unsupported sizes.
+ * Limits: rows_per_expert % 128 == 0, K % 128 == 0, out_bytes large enough
+ * (MOE_ERR_WORKSPACE otherwise).
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_nvfp4_packed_sf_bytes(int E, int rows_per_expert, int K, int swiglu);
+MOE_API int moe_nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, int K, int swiglu, uint8_t* out,
+                                 size_t out_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_grouped_swiglu_nvfp4 with the weight scales given already rearranged
+ * by moe_nvfp4_prepack_sf (sf_gu_packed from sf_gu with swiglu = 1,
+ * rows_per_expert = 2I, K = H; sf_d_packed from sf_d with swiglu = 0,
+ * rows_per_expert = H, K = I).  Results are identical to
+ * moe_grouped_swiglu_nvfp4's; all other arguments, limits and the workspace
+ * are the same.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_grouped_swiglu_nvfp4_prepacked(const void* x, const int32_t* row_token, const int32_t* expert_offsets,
+                                               int T, int rows, int H, int I, int E, const uint8_t* w_gu,
+                                               const uint8_t* sf_gu_packed, const float* gs_gu, const uint8_t* w_d,
+                                               const uint8_t* sf_d_packed, const float* gs_d,
+                                               const float* act_gs_in, float* act_gs_out, int out_fp32, void* f,
+                                               void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Weighted combine [ARCH]:
  *   y[t] = sum_{j<k} topk_w[t, j] * f[slot_row[t, j]]  (+ gate[t] * shared[t])
  * summed in FP32 in slot order, rounded once to dtype.

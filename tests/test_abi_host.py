@@ -77,3 +77,22 @@ def test_zero_sized_calls_are_no_ops():
     assert _code("moe_grouped_swiglu_bf16", None, ctypes.c_void_p(16), None, 0, 0, 256, 64, 4, None, None, 0, 0, None,
                  None, 0, None) == abi.MOE_OK
     assert _code("moe_combine", None, 0, None, 2, None, None, None, 0, 2, 256, 0, None, None) == abi.MOE_OK
+
+
+def test_nvfp4_prepack_sizes_and_checks():
+    lib = abi.load()
+    # one 2 KB scale tile per 128 rows and 256 K per expert
+    assert lib.moe_nvfp4_packed_sf_bytes(512, 1280, 2048, 1) == 512 * 10 * 8 * 2048
+    assert lib.moe_nvfp4_packed_sf_bytes(512, 2048, 640, 0) == 512 * 16 * 3 * 2048
+    assert lib.moe_nvfp4_packed_sf_bytes(4, 100, 256, 0) == 0
+    buf = ctypes.c_void_p(256)  # never dereferenced: the checks come first
+    assert _code("moe_nvfp4_prepack_sf", buf, 4, 100, 256, 0, buf, 1 << 20, None) == abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_nvfp4_prepack_sf", buf, 4, 128, 256, 2, buf, 1 << 20, None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("moe_nvfp4_prepack_sf", None, 4, 128, 256, 0, buf, 1 << 20, None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("moe_nvfp4_prepack_sf", buf, 4, 128, 256, 0, buf, 4 * 2048 - 1, None) == abi.MOE_ERR_WORKSPACE
+    assert _code("moe_grouped_swiglu_nvfp4_prepacked", None, None, None, 4, 8, 256, 100, 4, None, None, None, None,
+                 None, None, None, None, 0, None, None, 0, None) == abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_grouped_swiglu_nvfp4_prepacked", buf, None, buf, 4, 4, 256, 128, 4, buf, None, buf, buf, buf,
+                 buf, None, None, 0, buf, None, 0, None) == abi.MOE_ERR_INVALID_ARG  # packed gate/up scales missing
+    assert _code("moe_grouped_swiglu_nvfp4_prepacked", None, None, None, 0, 0, 256, 128, 4, None, None, None, None,
+                 None, None, None, None, 0, None, None, 0, None) == abi.MOE_OK

@@ -77,6 +77,11 @@ def test_grouped_swiglu_nvfp4(T, H, I, E, k):
     assert abs(_np(gs_out)[1] / s_h - 1) < 1e-2
     err = rel_err(f64(f)[sr.cpu().numpy().ravel()], ref[perm["slot_row"].ravel()])
     assert err <= TOL_4BIT, err
+    # weight scales rearranged once up front give the same result, bit for bit
+    fp = abi.moe_grouped_swiglu_nvfp4_prepacked(x, rt, off, T * k, w["w_gu"], w["sfp_gu"], w["gs_gu"], w["w_d"],
+                                                w["sfp_d"], w["gs_d"], out_fp32=True)
+    torch.cuda.synchronize()
+    assert torch.equal(fp, f)
 
 
 def _layer_ref(wl, w, x, deq, act_gs=None):
