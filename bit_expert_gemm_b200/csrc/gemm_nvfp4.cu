@@ -11,10 +11,18 @@
 // k_pack_sf_a / k_pack_sf_b): per 128-row tile and K step, four 512-byte
 // atoms in the 32x128-bit layout the tensor cores read (rows r, r+32, r+64,
 // r+96 interleaved per 16-byte row), fetched with one 2 KB bulk copy per
-// operand on the stage's barrier; the UMMA warp copies them into TMEM
-// (tcgen05.cp) right before the MMAs that use them.
+// operand on the stage's barrier.  Two copy warps move them into a TMEM slot
+// of their own per pipeline stage (tcgen05.cp, one for A and one for B, each
+// committing to the stage's scales-ready barrier), so that the copies neither
+// queue behind the MMA issue nor overwrite columns an MMA in flight still
+// reads: copies issued by the MMA thread itself into one shared slot held
+// the MMA pipe to about a third of its rate.
 //
-// Warp roles: 0 TMA producer, 1 UMMA issuer (TMEM owner), 2..5 epilogue.
+// Warp roles: 0 and 8 TMA producers (A with its scales, B with its scales:
+// one thread issuing every copy of a stage held the loads to about 86 GB/s
+// per SM, since copy instructions block while the TMA unit is busy),
+// 1 UMMA issuer (TMEM owner), 2..5 epilogue, 6 and 7 scale-factor copies
+// (A and B).
 #include <cstring>
 
 #include "common.cuh"
@@ -36,13 +44,17 @@ constexpr int SF_ATOM = 512;             // 128 rows x 4 scales
 constexpr int SFA_OFF = A_BYTES + B_BYTES;
 constexpr int SFB_OFF = SFA_OFF + 4 * SF_ATOM;
 constexpr int STAGE_BYTES = SFB_OFF + 4 * SF_ATOM;  // 36 KB
-constexpr int STAGES = 5;
+#ifndef NVFP4_STAGES
+#define NVFP4_STAGES 5
+#endif
+constexpr int STAGES = NVFP4_STAGES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-constexpr int kThreads = 192;
+constexpr int kThreads = 288;
 constexpr int SF_TILE = 4 * SF_ATOM;     // scales of one operand tile for one K step
-constexpr uint32_t TMEM_COLS = 512;      // 2 x 128 accumulator + scale factors
-constexpr uint32_t SFA_COL = 2 * BN;     // 4 MMAs x 4 columns
-constexpr uint32_t SFB_COL = SFA_COL + 16;
+constexpr uint32_t TMEM_COLS = 512;      // 2 x 128 accumulator + a scale slot per stage
+constexpr uint32_t SF_COL = 2 * BN;      // slot s at SF_COL + 32 s: A (4 MMAs x 4 columns), then B
+constexpr uint32_t SF_SLOT = 32;
+static_assert(SF_COL + STAGES * SF_SLOT <= TMEM_COLS, "scale slots must fit in TMEM");
 static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
 
 struct Args {
@@ -145,8 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_nvfp4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Args args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[2],
-      tempty_bar[2], drain_bar;
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], sfready_bar[STAGES], tfull_bar[2],
+      tempty_bar[2], drain_bar, cdrain_bar[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ int goff[kGemmMaxGroups + 1];
@@ -159,18 +171,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], 2);  // one expect_tx arrival from each producer
       mbar_init(&empty_bar[s], 1);
+      mbar_init(&sfready_bar[s], 2);  // one tcgen05.commit from each copy warp
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
       mbar_init(&tempty_bar[i], 128);
     }
     mbar_init(&drain_bar, 1);
+    mbar_init(&cdrain_bar[0], 1);
+    mbar_init(&cdrain_bar[1], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if ((warp == 0 || warp == 8) && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
@@ -192,9 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* status = args.status;
   const unsigned long long lim = args.limit_ns;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 8) {
     if (lane == 0) {
-      // ---------------- TMA producer: packed FP4 codes of A and B ----------------
+      // ---------------- TMA producers: warp 0 A, warp 8 B (codes + scales) ----------------
+      const bool pa = warp == 0;
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
@@ -205,17 +221,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b_row = t.g * args.b_rows_per_group + t.n * BNH;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], A_BYTES + B_BYTES + 2 * SF_TILE);
-          tma_load_2d(stg(stage), &tmA, &full_bar[stage], kt * BKB, a_row);
-          bulk_load(stg(stage) + SFA_OFF, args.sfa + (size_t(tile_start[t.g] + t.m) * KT + kt) * SF_TILE, SF_TILE,
-                    &full_bar[stage]);
-          bulk_load(stg(stage) + SFB_OFF, args.sfb + (size_t(t.g * nt + t.n) * KT + kt) * SF_TILE, SF_TILE,
-                    &full_bar[stage]);
-          if (args.swiglu) {
-            tma_load_2d(stg(stage) + A_BYTES, &tmB, &full_bar[stage], kt * BKB, b_row);
-            tma_load_2d(stg(stage) + A_BYTES + BNH * BKB, &tmB, &full_bar[stage], kt * BKB, b_row + args.up_offset);
+          if (pa) {
+            mbar_arrive_expect_tx(&full_bar[stage], A_BYTES + SF_TILE);
+            tma_load_2d(stg(stage), &tmA, &full_bar[stage], kt * BKB, a_row);
+            bulk_load(stg(stage) + SFA_OFF, args.sfa + (size_t(tile_start[t.g] + t.m) * KT + kt) * SF_TILE, SF_TILE,
+                      &full_bar[stage]);
           } else {
-            tma_load_2d(stg(stage) + A_BYTES, &tmB, &full_bar[stage], kt * BKB, b_row);
+            mbar_arrive_expect_tx(&full_bar[stage], B_BYTES + SF_TILE);
+            bulk_load(stg(stage) + SFB_OFF, args.sfb + (size_t(t.g * nt + t.n) * KT + kt) * SF_TILE, SF_TILE,
+                      &full_bar[stage]);
+            if (args.swiglu) {
+              tma_load_2d(stg(stage) + A_BYTES, &tmB, &full_bar[stage], kt * BKB, b_row);
+              tma_load_2d(stg(stage) + A_BYTES + BNH * BKB, &tmB, &full_bar[stage], kt * BKB, b_row + args.up_offset);
+            } else {
+              tma_load_2d(stg(stage) + A_BYTES, &tmB, &full_bar[stage], kt * BKB, b_row);
+            }
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -240,20 +260,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(acc * BN);
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
+          // the stage's scales are in TMEM (the copy warps saw its operands land first)
+          if (!mbar_wait(&sfready_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sbase = smem_u32(stg(stage));
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_cp_32x128b_x4(tmem_base + SFA_COL + 4 * j, sdesc_sf_atom(sbase + SFA_OFF + j * SF_ATOM));
-            tmem_cp_32x128b_x4(tmem_base + SFB_COL + 4 * j, sdesc_sf_atom(sbase + SFB_OFF + j * SF_ATOM));
-          }
+          const uint32_t sf = tmem_base + SF_COL + uint32_t(stage) * SF_SLOT;
           const uint64_t ad = sdesc_kmajor_sw128(sbase);
           const uint64_t bd = sdesc_kmajor_sw128(sbase + A_BYTES);
 #pragma unroll
           for (int j = 0; j < 4; ++j)  // K = 64 per MMA: 32 bytes along the swizzled row
-            umma_mxf4nvf4(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), kIdescMxf4, tmem_base + SFA_COL + 4 * j,
-                          tmem_base + SFB_COL + 4 * j, (kt | j) != 0);
+            umma_mxf4nvf4(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), kIdescMxf4, sf + 4 * j, sf + 16 + 4 * j,
+                          (kt | j) != 0);
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -266,7 +283,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(&drain_bar, 0, &never, nullptr, lim);
     }
-  } else if (warp < 6) {
+  } else if (warp == 6 || warp == 7) {
+    if (lane == 0) {
+      // ---------------- scale-factor copies: warp 6 A, warp 7 B ----------------
+      // Slot `stage` is free again once the stage has been refilled: the
+      // producer refills only after the MMAs that read the slot completed.
+      const int which = warp - 6;
+      const uint32_t src_off = which ? SFB_OFF : SFA_OFF;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t src = smem_u32(stg(stage)) + src_off;
+          const uint32_t dst = tmem_base + SF_COL + uint32_t(stage) * SF_SLOT + uint32_t(which * 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tmem_cp_32x128b_x4(dst + 4 * j, sdesc_sf_atom(src + j * SF_ATOM));
+          umma_commit(&sfready_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // this warp's copies have landed before TMEM is released
+      umma_commit(&cdrain_bar[which]);
+      volatile int never = 0;
+      mbar_wait(&cdrain_bar[which], 0, &never, nullptr, lim);
+    }
+  } else {
     // ---------------- epilogue: warps 2..5 ----------------
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
