@@ -25,8 +25,11 @@ sample of the same workload on this machine's host cores.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -248,6 +251,31 @@ KERNEL_NAMES = {"bf16": "moe_experts_bf16 (routed + shared experts: GEMM1/SwiGLU
                          "tcgen05 kind::mxf4nvf4)"}
 
 
+def measured_traffic(workload: str):
+    """DRAM bytes per expert call from the committed ncu summaries under
+    profiles/: a line `traffic: workload=W bytes_per_launch=N sources=a,b
+    sha256=H`.  The hash is over the listed kernel sources as they were when
+    the counters were taken; if the sources have changed since, the figure no
+    longer belongs to the kernel that runs and None is returned."""
+    pat = re.compile(r"traffic: workload=(\S+) bytes_per_launch=(\d+) sources=(\S+) sha256=([0-9a-f]+)")
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(path):
+            m = pat.search(line)
+            if not m or m.group(1) != workload:
+                continue
+            h = hashlib.sha256()
+            try:
+                for f in m.group(3).split(","):
+                    with open(os.path.join(ROOT, "bit_expert_gemm_b200", "csrc", f), "rb") as fh:
+                        h.update(fh.read())
+            except OSError:
+                return None, None
+            if h.hexdigest()[:len(m.group(4))] != m.group(4):
+                return None, os.path.relpath(path, ROOT) + " (kernel sources changed since the capture)"
+            return int(m.group(2)), os.path.relpath(path, ROOT)
+    return None, None
+
+
 def _count_step_kernels(layer, x, step) -> int:
     layer.capture(x, step, warmup=0)
     return layer.graph_kernels
@@ -418,6 +446,10 @@ def run_native(args, dist: Dist) -> None:
     value = tokens / (ms / 1e3)
     peaks = measured_peaks()
     roofline = expert_roofline(wl, [u[0] for u in units], T, rows, ffn_ms, peaks)
+    roofline["traffic"], src = measured_traffic(args.workload)
+    if src:
+        roofline["traffic_source"] = (src + ": dram__bytes_read.sum + dram__bytes_write.sum of the expert call's "
+                                      "launches, bytes per call, cold-cache ncu capture")
 
     # end-to-end through the public API: pinned host x -> y in pinned host memory
     e2e = None
