@@ -3,6 +3,8 @@
 // streaming kernels: every byte of f is read once with 16-byte vector loads.
 #include <float.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -20,6 +22,27 @@ __device__ __forceinline__ void load4(const void* f, size_t r, int H, int c, flo
   }
 }
 
+// Loads 8 consecutive values of row `r` starting at column c as FP32 (one or
+// two 16-byte loads).
+template <typename T16, bool F32>
+__device__ __forceinline__ void load8(const void* f, size_t r, int H, int c, float (&v)[8]) {
+  if (F32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(f) + r * H + c);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(static_cast<const T16*>(f) + r * H + c));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 u = Pack2<T16>::unpack(w[i]);
+      v[2 * i] = u.x;
+      v[2 * i + 1] = u.y;
+    }
+  }
+}
+
 template <typename T16>
 __device__ __forceinline__ void store4(T16* y, size_t r, int H, int c, const float (&v)[4]) {
   uint2 q;
@@ -28,64 +51,110 @@ __device__ __forceinline__ void store4(T16* y, size_t r, int H, int c, const flo
   *reinterpret_cast<uint2*>(y + r * H + c) = q;
 }
 
-// y[t] = sum_j w[t,j] f[slot_row[t,j]] (+ gate[t] * shared[t]); grid (T, ceil(H/4/256)).
-template <typename T16, bool F32>
+// y[t] = sum_j w[t,j] f[slot_row[t,j]] (+ gate[t] * shared[t]).  Each thread
+// owns 8 consecutive columns (16-byte loads of 16-bit f); a block of 256
+// threads covers 2048 columns of a row and walks tokens t = blockIdx.x,
+// blockIdx.x + gridDim.x, ... (grid (min(T, 8 x SMs), ceil(H/2048))).  The
+// KM (>= k) row loads of a token are all issued before the first is used, so
+// that they are in flight together; the sum then runs in slot order.
+template <typename T16, bool F32, int KM>
 __global__ void __launch_bounds__(256) k_combine(const void* __restrict__ f, const int32_t* __restrict__ slot_row,
                                                  int ks, const float* __restrict__ w, const T16* __restrict__ shared,
-                                                 const float* __restrict__ gate, int k, int H, T16* __restrict__ y) {
+                                                 const float* __restrict__ gate, int k, int H, int T,
+                                                 T16* __restrict__ y) {
+  constexpr int NV = F32 ? 2 : 1;  // 16-byte vectors per row and thread
   griddep_wait();  // f comes from the kernel just before (programmatic dependent launch)
   griddep_launch_dependents();
-  const int t = blockIdx.x;
-  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
   if (c >= H) return;
-  // all slots' rows and weights first, so that the k row loads are in flight together
-  int r[16];
-  float wj[16];
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    int r[KM];
+    float wj[KM];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    r[j] = j < k ? __ldg(slot_row + size_t(t) * ks + j) : 0;
-    wj[j] = j < k ? __ldg(w + size_t(t) * k + j) : 0.0f;
-  }
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    if (j < k && r[j] >= 0) {  // -1: an assignment the permutation rejected
-      float v[4];
-      load4<T16, F32>(f, size_t(r[j]), H, c, v);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = fmaf(wj[j], v[i], acc[i]);
+    for (int j = 0; j < KM; ++j) {
+      r[j] = j < k ? __ldg(slot_row + size_t(t) * ks + j) : -1;
+      wj[j] = j < k ? __ldg(w + size_t(t) * k + j) : 0.0f;
     }
-  }
-  if (shared) {
-    const float g = gate ? gate[t] : 1.0f;
-    float v[4];
-    load4<T16, false>(shared, size_t(t), H, c, v);
+    uint4 raw[KM][NV];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = fmaf(g, v[i], acc[i]);
+    for (int j = 0; j < KM; ++j) {  // -1: past k, or an assignment the permutation rejected
+      const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(f) +
+                                                      (size_t(r[j] < 0 ? 0 : r[j]) * H + c) * (F32 ? 4 : 2));
+#pragma unroll
+      for (int v = 0; v < NV; ++v) raw[j][v] = r[j] >= 0 ? __ldg(p + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint4 sraw = make_uint4(0u, 0u, 0u, 0u);
+    if (shared) sraw = __ldg(reinterpret_cast<const uint4*>(shared + size_t(t) * H + c));
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      if (r[j] >= 0) {
+        float v[8];
+        if (F32) {
+#pragma unroll
+          for (int q = 0; q < NV; ++q) {
+            v[4 * q] = __uint_as_float(raw[j][q].x);
+            v[4 * q + 1] = __uint_as_float(raw[j][q].y);
+            v[4 * q + 2] = __uint_as_float(raw[j][q].z);
+            v[4 * q + 3] = __uint_as_float(raw[j][q].w);
+          }
+        } else {
+          const uint32_t u[4] = {raw[j][0].x, raw[j][0].y, raw[j][0].z, raw[j][0].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 h = Pack2<T16>::unpack(u[i]);
+            v[2 * i] = h.x;
+            v[2 * i + 1] = h.y;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj[j], v[i], acc[i]);
+      }
+    }
+    if (shared) {
+      const float g = gate ? gate[t] : 1.0f;
+      const uint32_t u[4] = {sraw.x, sraw.y, sraw.z, sraw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 h = Pack2<T16>::unpack(u[i]);
+        acc[2 * i] = fmaf(g, h.x, acc[2 * i]);
+        acc[2 * i + 1] = fmaf(g, h.y, acc[2 * i + 1]);
+      }
+    }
+    uint4 q;
+    q.x = Pack2<T16>::pack(acc[0], acc[1]);
+    q.y = Pack2<T16>::pack(acc[2], acc[3]);
+    q.z = Pack2<T16>::pack(acc[4], acc[5]);
+    q.w = Pack2<T16>::pack(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(y + size_t(t) * H + c) = q;
   }
-  store4<T16>(y, size_t(t), H, c, acc);
+}
+
+template <typename T16, bool F32>
+static cudaError_t launch_combine(dim3 grid, cudaStream_t stream, const void* f, const int32_t* slot_row, int ks,
+                                  const float* w, const void* shared, const float* gate, int k, int H, int T,
+                                  void* y) {
+  const T16* sh = static_cast<const T16*>(shared);
+  T16* yy = static_cast<T16*>(y);
+  if (k <= 8) return launch_pdl(k_combine<T16, F32, 8>, grid, dim3(256), 0, stream, f, slot_row, ks, w, sh, gate, k, H, T, yy);
+  if (k <= 12) return launch_pdl(k_combine<T16, F32, 12>, grid, dim3(256), 0, stream, f, slot_row, ks, w, sh, gate, k, H, T, yy);
+  return launch_pdl(k_combine<T16, F32, 16>, grid, dim3(256), 0, stream, f, slot_row, ks, w, sh, gate, k, H, T, yy);
 }
 
 int combine(const void* f, int f_fp32, const int32_t* slot_row, int ks, const float* w, const void* shared,
             const float* gate, int T, int k, int H, int dtype, void* y, cudaStream_t stream) {
   if (T == 0) return MOE_OK;
-  dim3 grid(T, (H / 4 + 255) / 256);
+  dim3 grid(std::min(T, 8 * num_sms()), (H / 8 + 255) / 256);
   if (dtype == MOE_DTYPE_BF16) {
-    using T16 = __nv_bfloat16;
     if (f_fp32)
-      MOE_CHECK_CUDA(launch_pdl(k_combine<T16, true>, grid, dim3(256), 0, stream, f, slot_row, ks, w,
-                                static_cast<const T16*>(shared), gate, k, H, static_cast<T16*>(y)));
+      MOE_CHECK_CUDA((launch_combine<__nv_bfloat16, true>(grid, stream, f, slot_row, ks, w, shared, gate, k, H, T, y)));
     else
-      MOE_CHECK_CUDA(launch_pdl(k_combine<T16, false>, grid, dim3(256), 0, stream, f, slot_row, ks, w,
-                                static_cast<const T16*>(shared), gate, k, H, static_cast<T16*>(y)));
+      MOE_CHECK_CUDA((launch_combine<__nv_bfloat16, false>(grid, stream, f, slot_row, ks, w, shared, gate, k, H, T, y)));
   } else {
-    using T16 = __half;
     if (f_fp32)
-      MOE_CHECK_CUDA(launch_pdl(k_combine<T16, true>, grid, dim3(256), 0, stream, f, slot_row, ks, w,
-                                static_cast<const T16*>(shared), gate, k, H, static_cast<T16*>(y)));
+      MOE_CHECK_CUDA((launch_combine<__half, true>(grid, stream, f, slot_row, ks, w, shared, gate, k, H, T, y)));
     else
-      MOE_CHECK_CUDA(launch_pdl(k_combine<T16, false>, grid, dim3(256), 0, stream, f, slot_row, ks, w,
-                                static_cast<const T16*>(shared), gate, k, H, static_cast<T16*>(y)));
+      MOE_CHECK_CUDA((launch_combine<__half, false>(grid, stream, f, slot_row, ks, w, shared, gate, k, H, T, y)));
   }
   MOE_CHECK_CUDA(cudaGetLastError());
   return MOE_OK;
