@@ -425,7 +425,10 @@ __device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t smem_addr, uint
   return d;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g).  Its callers round the product silu(g) * u to a
+// 16-bit type right after, so the fast division (a couple of FP32 ulp) is
+// invisible there; IEEE division made the SwiGLU epilogues ALU-heavy.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
