@@ -42,6 +42,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from bit_expert_gemm_b200 import MoELayer, abi, synth  # noqa: E402
+from bit_expert_gemm_b200.layer import HostPipeline  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at E=512,k=10 (prefill TFLOP/s & decode HBM GB/s vs roofline)"
 L2_BYTES = 126 * 1024 * 1024
@@ -451,41 +452,47 @@ def run_native(args, dist: Dist) -> None:
         roofline["traffic_source"] = (src + ": dram__bytes_read.sum + dram__bytes_write.sum of the expert call's "
                                       "launches, bytes per call, cold-cache ncu capture")
 
-    # end-to-end through the public API: pinned host x -> y in pinned host memory
+    # end-to-end through the public API: pinned host x -> y in pinned host memory, every step's upload and
+    # download inside the timed region, overlapped with the neighbouring steps' forwards (HostPipeline)
     e2e = None
     if not args.no_e2e and kind == "forward":
         xh = [x.cpu().pin_memory() for _, x in units]
-        yh = torch.empty((T, wl.H), dtype=layer.y.dtype).pin_memory()
-        xd = torch.empty_like(xs[0])
-        g_e2e = None if args.no_graph else [lay.capture(xd) for lay, _ in units]
+        yh = [torch.empty((T, wl.H), dtype=layer.y.dtype).pin_memory() for _ in range(2)]
+        pipes = {}
+        for lay, _ in units:
+            if id(lay) not in pipes:
+                pipes[id(lay)] = HostPipeline(lay, T, use_graphs=not args.no_graph)
 
         def e2e_step(i):
             u = i % n_units
-            lay = units[u][0]
-            xd.copy_(xh[u], non_blocking=True)
-            if g_e2e is not None:
-                g_e2e[u].replay()
-            else:
-                lay.forward(xd)
-            yh.copy_(lay.y[:T], non_blocking=True)
+            pipes[id(units[u][0])].step(xh[u], yh[i & 1])
+
+        def e2e_finish():
+            for p in pipes.values():
+                p.finish()
 
         for i in range(max(2, args.warmup, n_units)):
             e2e_step(i)
+        e2e_finish()
         dist.barrier()
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
+        for p in pipes.values():
+            p.begin()
         for i in range(args.steps):
             e2e_step(i)
+        e2e_finish()
         b.record(stream)
         torch.cuda.synchronize()
         dist.barrier()
         e2e_ms = dist.max(a.elapsed_time(b) / args.steps)
         e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
                "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
-               "d2h_bytes_per_step": int(yh.numel() * yh.element_size()),
-               "path": "pinned host x -> H2D copy -> layer (CUDA graph of the C-ABI calls) -> D2H copy of y"}
+               "d2h_bytes_per_step": int(yh[0].numel() * yh[0].element_size()),
+               "path": "pinned host x -> H2D copy -> layer (CUDA graph of the C-ABI calls) -> D2H copy of y, "
+                       "with HostPipeline overlapping step i+1's upload and step i-1's download with step i"}
 
     if launches_per_step is None:  # eager: count one pass's launches from a throw-away capture
         launches_per_step = _count_step_kernels(layer, xs[0], lambda xx: step(layer, xx))

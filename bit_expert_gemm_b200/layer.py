@@ -183,12 +183,14 @@ class MoELayer:
                                     out_fp32=f.dtype == torch.float32, f=f, shared_out=sh, ws=self.ws_exp)
         return f, sh
 
-    def forward(self, x: torch.Tensor) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """y [T, H] = the layer applied to x [T, H]; into `y` if given, else
+        into the layer's own output buffer (overwritten by the next pass)."""
         T = x.shape[0]
         assert T <= self.T_max and self.extra == 0
         self.route(x)
         f, sh = self.experts_and_shared(x)
-        y = self.y[:T]
+        y = self.y[:T] if y is None else y
         abi.moe_combine(f, self.slot_row[:T], self.topk_w[:T], shared_out=sh, y=y)
         return y
 
@@ -230,3 +232,73 @@ class MoELayer:
         abi.razor_refill_rms_accumulate(f, self.slot_row[:T], self.topk_idx[:T], self.topk_logit[:T], self.offsets,
                                         sum_sq, count, shared_out=sh, y_out=y, ws=self.ws_refill)
         return y
+
+
+class HostPipeline:
+    """Streams token batches from pinned host memory through one layer and
+    back, overlapping the upload of batch i+1 and the download of batch i-1
+    with the forward of batch i: uploads and downloads run on two copy
+    streams, the forward (one CUDA graph per device buffer) on the caller's
+    current stream, with two device buffers each for x and y and events
+    between them, so a buffer is only refilled once the pass that reads it
+    is done.
+
+        pipe = HostPipeline(layer, T)
+        for i, (xh, yh) in enumerate(batches):   # pinned host tensors [T, H]
+            pipe.step(xh, yh)
+        pipe.finish()                            # the current stream waits for the last download
+
+    A host output buffer is complete once finish() (or a later wait on the
+    current stream) has returned; a host input buffer may be reused once the
+    step after next has been enqueued.
+    """
+
+    def __init__(self, layer: MoELayer, T: int, use_graphs: bool = True):
+        assert T <= layer.T_max and layer.extra == 0
+        H = layer.w["w_router"].shape[1]
+        dev = layer.dev
+        self.layer, self.T = layer, T
+        self.x = [torch.empty((T, H), dtype=layer.adt, device=dev) for _ in range(2)]
+        self.y = [torch.empty((T, H), dtype=layer.adt, device=dev) for _ in range(2)]
+        self.s_in, self.s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]    # x[b] uploaded
+        self.ev_used = [torch.cuda.Event() for _ in range(2)]  # the pass on x[b] is done and y[b] written
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]   # y[b] downloaded
+        self.graphs = None
+        if use_graphs:
+            self.graphs = [layer.capture(self.x[b], fn=lambda xx, b=b: layer.forward(xx, y=self.y[b]))
+                           for b in range(2)]
+        self.i = 0
+
+    def begin(self) -> None:
+        """Orders the copy streams after the work already on the current
+        stream (for instance a timing event)."""
+        cs = torch.cuda.current_stream()
+        self.s_in.wait_stream(cs)
+        self.s_out.wait_stream(cs)
+
+    def step(self, x_host: torch.Tensor, y_host: torch.Tensor) -> None:
+        b, cs = self.i & 1, torch.cuda.current_stream()
+        if self.i >= 2:
+            self.s_in.wait_event(self.ev_used[b])  # the pass two steps back has read x[b]
+        with torch.cuda.stream(self.s_in):
+            self.x[b].copy_(x_host, non_blocking=True)
+            self.ev_in[b].record(self.s_in)
+        cs.wait_event(self.ev_in[b])
+        if self.i >= 2:
+            cs.wait_event(self.ev_out[b])  # y[b] of two steps back has been downloaded
+        if self.graphs is not None:
+            self.graphs[b].replay()
+        else:
+            self.layer.forward(self.x[b], y=self.y[b])
+        self.ev_used[b].record(cs)
+        self.s_out.wait_event(self.ev_used[b])
+        with torch.cuda.stream(self.s_out):
+            y_host.copy_(self.y[b], non_blocking=True)
+            self.ev_out[b].record(self.s_out)
+        self.i += 1
+
+    def finish(self) -> None:
+        cs = torch.cuda.current_stream()
+        cs.wait_stream(self.s_in)
+        cs.wait_stream(self.s_out)

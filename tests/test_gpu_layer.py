@@ -43,6 +43,30 @@ def test_tiny_layer_forward():
     assert abi.moe_device_status() == 0
 
 
+@pytest.mark.parametrize("T,graphs", [(64, True), (8, False)])
+def test_host_pipeline_matches_forward(bf16_layer, T, graphs):
+    """Batches streamed from pinned host memory by HostPipeline (uploads and
+    downloads overlapped with the neighbouring forwards) come back bit for bit
+    equal to the device forward of the same batches, including when more
+    batches than buffers are in flight."""
+    from bit_expert_gemm_b200.layer import HostPipeline
+    wl, w = bf16_layer
+    layer = MoELayer(w, wl.k, "bf16", T_max=T)
+    xs = [synth.make_tokens(wl, T, seed=s, device=DEV) for s in range(5)]
+    want = [layer.forward(x).clone() for x in xs]
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty((T, wl.H), dtype=torch.bfloat16).pin_memory() for _ in xs]
+    pipe = HostPipeline(layer, T, use_graphs=graphs)
+    pipe.begin()
+    for i in range(len(xs)):
+        pipe.step(xh[i], yh[i])
+    pipe.finish()
+    torch.cuda.synchronize()
+    for i in range(len(xs)):
+        assert torch.equal(yh[i], want[i].cpu()), i
+    assert abi.moe_device_status() == 0
+
+
 @pytest.mark.parametrize("T", [1, 8, 64])
 def test_bf16_layer_decode(bf16_layer, T):
     wl, w = bf16_layer
