@@ -52,6 +52,10 @@ _SIGS = {
     "moe_experts_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "moe_experts_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P,
                                  _SZ, _P]),
+    "moe_experts_awq_g32_prepacked": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P,
+                                           _P, _P, _SZ, _P]),
+    "moe_awq_packed_bytes": (_SZ, [_I, _I, _I]),
+    "moe_awq_prepack_g32": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
     "moe_grouped_swiglu_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "moe_awq_dequant_g32": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_nvfp4_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -277,6 +281,41 @@ def moe_experts_awq_g32(x, row_token, expert_offsets, rows: int, qw_gu, qz_gu, s
     _call("moe_experts_awq_g32", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E, _p(qw_gu), _p(qz_gu),
           _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), _p(w_sh_gate_up), _p(w_sh_down), int(out_fp32), _p(f),
           _p(shared_out), _p(ws), ws.numel(), _stream(stream))
+    return f, shared_out
+
+
+def moe_awq_prepack_g32(qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d, out=None, stream=None):
+    """Tile-packed copy of one layer's routed AWQ weights (uint8 device buffer) for moe_experts_awq_g32_prepacked."""
+    E, H = qw_gu.shape[0], qw_gu.shape[1]
+    I = qw_gu.shape[2] * 8 // 2
+    nbytes = int(load().moe_awq_packed_bytes(E, H, I))
+    if nbytes == 0:
+        raise ValueError(f"moe_awq_prepack_g32: unsupported sizes E={E} H={H} I={I}")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=qw_gu.device)
+    _call("moe_awq_prepack_g32", _p(qw_gu), _p(qz_gu), _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), E, H, I, _p(out),
+          out.numel(), _stream(stream))
+    return out
+
+
+def moe_experts_awq_g32_prepacked(x, row_token, expert_offsets, rows: int, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
+                                  awq_packed, w_sh_gate_up, w_sh_down, out_fp32: bool = False, f=None,
+                                  shared_out=None, ws=None, stream=None):
+    """moe_experts_awq_g32 with the routed weights also tile-packed (read by the T <= 16 path)."""
+    T, H = x.shape
+    E = qw_gu.shape[0]
+    I = qw_gu.shape[2] * 8 // 2
+    dev = x.device
+    _need(x, torch.float16, "x")
+    if f is None:
+        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else torch.float16, device=dev)
+    if shared_out is None:
+        shared_out = torch.empty((T, H), dtype=torch.float16, device=dev)
+    if ws is None:
+        ws = workspace(MOE_OP_EXPERTS_AWQ_G32, T, H, E, max(1, rows // max(T, 1)), I, dev)
+    _call("moe_experts_awq_g32_prepacked", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E, _p(qw_gu),
+          _p(qz_gu), _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), _p(awq_packed), _p(w_sh_gate_up), _p(w_sh_down),
+          int(out_fp32), _p(f), _p(shared_out), _p(ws), ws.numel(), _stream(stream))
     return f, shared_out
 
 

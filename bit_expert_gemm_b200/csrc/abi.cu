@@ -45,7 +45,10 @@ int decode_experts_fused_awq(const void* x, const int32_t* row_token, const int3
                              int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
                              const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gu,
                              const void* w_sh_d, int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
-                             cudaStream_t stream);
+                             cudaStream_t stream, const void* qpack);
+size_t awq_packed_bytes(int E, int H, int I);
+int awq_prepack(const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
+                const int32_t* qz_d, const void* sc_d, int E, int H, int I, void* out, cudaStream_t stream);
 int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
                          int E, const void* w_gu, const void* w_d, const void* w_sh_gu, const void* w_sh_d, int dtype,
                          int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -399,11 +402,11 @@ int moe_experts_bf16(const void* x, const int32_t* row_token, const int32_t* exp
   return dense_swiglu(x, T, H, I, w_sh_gate_up, w_sh_down, dtype, shared_out, static_cast<uint16_t*>(ws), st);
 }
 
-int moe_experts_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows, int H,
-                        int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
-                        const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gate_up,
-                        const void* w_sh_down, int out_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
-                        void* stream) {
+static int experts_awq_impl(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows,
+                            int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
+                            const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* awq_packed,
+                            const void* w_sh_gate_up, const void* w_sh_down, int out_fp32, void* f, void* shared_out,
+                            void* ws, size_t ws_bytes, void* stream) {
   MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG,
               "moe_experts_awq_g32: bad sizes");
   MOE_REQUIRE(H > 0 && I > 0 && H % 128 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
@@ -422,7 +425,8 @@ int moe_experts_awq_g32(const void* x, const int32_t* row_token, const int32_t* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (T <= kFusedMaxT && fused_decode_enabled())
     return decode_experts_fused_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d,
-                                    sc_d, w_sh_gate_up, w_sh_down, out_fp32, f, shared_out, ws, ws_bytes, st);
+                                    sc_d, w_sh_gate_up, w_sh_down, out_fp32, f, shared_out, ws, ws_bytes, st,
+                                    awq_packed);
   int rc = MOE_OK;
   if (rows > 0) {
     rc = grouped_swiglu_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
@@ -430,6 +434,47 @@ int moe_experts_awq_g32(const void* x, const int32_t* row_token, const int32_t* 
     if (rc) return rc;
   }
   return dense_swiglu(x, T, H, I, w_sh_gate_up, w_sh_down, MOE_DTYPE_F16, shared_out, static_cast<uint16_t*>(ws), st);
+}
+
+int moe_experts_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows, int H,
+                        int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
+                        const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gate_up,
+                        const void* w_sh_down, int out_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
+                        void* stream) {
+  return experts_awq_impl(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
+                          nullptr, w_sh_gate_up, w_sh_down, out_fp32, f, shared_out, ws, ws_bytes, stream);
+}
+
+int moe_experts_awq_g32_prepacked(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
+                                  int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
+                                  const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
+                                  const void* awq_packed, const void* w_sh_gate_up, const void* w_sh_down,
+                                  int out_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(awq_packed != nullptr || T == 0, MOE_ERR_INVALID_ARG, "moe_experts_awq_g32_prepacked: null awq_packed");
+  MOE_REQUIRE(aligned16(awq_packed), MOE_ERR_INVALID_ARG,
+              "moe_experts_awq_g32_prepacked: awq_packed must be 16-byte aligned");
+  return experts_awq_impl(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
+                          awq_packed, w_sh_gate_up, w_sh_down, out_fp32, f, shared_out, ws, ws_bytes, stream);
+}
+
+size_t moe_awq_packed_bytes(int E, int H, int I) {
+  if (E < 1 || H <= 0 || I <= 0 || H % 128 || I % 64) return 0;
+  return awq_packed_bytes(E, H, I);
+}
+
+int moe_awq_prepack_g32(const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
+                        const int32_t* qz_d, const void* sc_d, int E, int H, int I, void* out, size_t out_bytes,
+                        void* stream) {
+  MOE_REQUIRE(E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG, "moe_awq_prepack_g32: E=%d", E);
+  MOE_REQUIRE(H > 0 && I > 0 && H % 128 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_awq_prepack_g32: need H %% 128 == 0 and I %% 64 == 0 (H=%d I=%d)", H, I);
+  MOE_REQUIRE(qw_gu && qz_gu && sc_gu && qw_d && qz_d && sc_d && out, MOE_ERR_INVALID_ARG,
+              "moe_awq_prepack_g32: null pointer");
+  MOE_REQUIRE(aligned16(out), MOE_ERR_INVALID_ARG, "moe_awq_prepack_g32: out must be 16-byte aligned");
+  const size_t need = awq_packed_bytes(E, H, I);
+  MOE_REQUIRE(out_bytes >= need, MOE_ERR_WORKSPACE, "moe_awq_prepack_g32: out holds %zu bytes, need %zu", out_bytes,
+              need);
+  return awq_prepack(qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d, E, H, I, out, static_cast<cudaStream_t>(stream));
 }
 
 int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,

@@ -86,4 +86,87 @@ int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scale
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Tile-packed AWQ weights for the fused decode kernel.  Per expert, first the
+// gate/up units (j, kt) for j < I/64, kt < H/64, then the down units (j, m)
+// for j < I/64, m < H/128; each unit is kAwqUnitBytes = 4736 bytes laid out
+// exactly as the kernel stages one 64-row K sub-tile in shared memory, so a
+// single bulk copy brings it:
+//   codes  [r0 16][wc 16][i 4] words: K row r0 + 16 i, code word wc of the
+//          unit's 128 output columns (4096 bytes);
+//   scales [2 groups][128 columns] FP16 (512 bytes);
+//   zeros  [2 groups][16 words] (128 bytes).
+// Gate/up unit (j, kt): K rows 64 kt.., output words 8j..8j+7 of the gate
+// half (wc < 8) and I/8 + 8j.. of the up half (wc >= 8); down unit (j, m):
+// K rows 64 j.. (the down projection's input features), output words
+// 16 m..16 m + 15.  Values are copied, not changed.
+// ---------------------------------------------------------------------------
+constexpr int kAwqUnitBytes = 4736;
+
+size_t awq_packed_bytes(int E, int H, int I) {
+  return size_t(E) * size_t(I / 64) * size_t(H / 64 + H / 128) * kAwqUnitBytes;
+}
+
+// grid (units per expert, E), 256 threads
+__global__ void __launch_bounds__(256) k_awq_pack(const uint32_t* __restrict__ qw_gu, const uint32_t* __restrict__ qz_gu,
+                                                  const uint16_t* __restrict__ sc_gu, const uint32_t* __restrict__ qw_d,
+                                                  const uint32_t* __restrict__ qz_d, const uint16_t* __restrict__ sc_d,
+                                                  int H, int I, uint8_t* __restrict__ out) {
+  const int u = blockIdx.x, e = blockIdx.y, t = threadIdx.x;
+  const int nka = H / 64, nkb = H / 128, J = I / 64;
+  const int NA = J * nka;
+  uint8_t* dst = out + (size_t(e) * (NA + J * nkb) + u) * kAwqUnitBytes;
+  const bool gu = u < NA;
+  int j, m = 0, k0, W;
+  const uint32_t *qw, *qz;
+  const uint16_t* sc;
+  if (gu) {
+    j = u / nka;
+    k0 = 64 * (u - j * nka);
+    W = 2 * I / 8;
+    qw = qw_gu + size_t(e) * H * W;
+    qz = qz_gu + size_t(e) * (H / 32) * W;
+    sc = sc_gu + size_t(e) * (H / 32) * (2 * I);
+  } else {
+    const int v = u - NA;
+    j = v / nkb;
+    m = v - j * nkb;
+    k0 = 64 * j;
+    W = H / 8;
+    qw = qw_d + size_t(e) * I * W;
+    qz = qz_d + size_t(e) * (I / 32) * W;
+    sc = sc_d + size_t(e) * (I / 32) * H;
+  }
+  auto word = [&](int wc) { return gu ? (wc < 8 ? 8 * j + wc : I / 8 + 8 * j + wc - 8) : 16 * m + wc; };
+  const int g0 = k0 / 32;
+  {  // codes: thread t = (r0, wc) copies rows r0, r0 + 16, r0 + 32, r0 + 48 of word wc
+    const int r0 = t >> 4, wc = t & 15;
+    uint4 c;
+    c.x = qw[size_t(k0 + r0) * W + word(wc)];
+    c.y = qw[size_t(k0 + r0 + 16) * W + word(wc)];
+    c.z = qw[size_t(k0 + r0 + 32) * W + word(wc)];
+    c.w = qw[size_t(k0 + r0 + 48) * W + word(wc)];
+    reinterpret_cast<uint4*>(dst)[t] = c;
+  }
+  {  // scales: thread t = (group, column)
+    const int gi = t >> 7, c = t & 127;
+    reinterpret_cast<uint16_t*>(dst + 4096)[t] = sc[size_t(g0 + gi) * (W * 8) + word(c >> 3) * 8 + (c & 7)];
+  }
+  if (t < 32) {  // zero points
+    const int gi = t >> 4, wc = t & 15;
+    reinterpret_cast<uint32_t*>(dst + 4608)[t] = qz[size_t(g0 + gi) * W + word(wc)];
+  }
+}
+
+int awq_prepack(const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
+                const int32_t* qz_d, const void* sc_d, int E, int H, int I, void* out, cudaStream_t stream) {
+  const int units = (I / 64) * (H / 64 + H / 128);
+  k_awq_pack<<<dim3(units, E), 256, 0, stream>>>(
+      reinterpret_cast<const uint32_t*>(qw_gu), reinterpret_cast<const uint32_t*>(qz_gu),
+      static_cast<const uint16_t*>(sc_gu), reinterpret_cast<const uint32_t*>(qw_d),
+      reinterpret_cast<const uint32_t*>(qz_d), static_cast<const uint16_t*>(sc_d), H, I, static_cast<uint8_t*>(out));
+  MOE_CHECK_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
 }  // namespace moe

@@ -24,7 +24,9 @@
 //   WQ = 1: routed experts in AWQ W4A16 g32 (input-major codes, zero points
 //     and FP16 scales, FP16 activations), the shared expert 16-bit as above.
 //     The producer stages each routed sub-tile's codes, scales and zero
-//     points (4.6 KB instead of 16 KB of FP16); four dequantisation warps
+//     points (4.6 KB instead of 16 KB of FP16): from the tile-packed copy of
+//     the weights (awq.cu) with one bulk copy per sub-tile when the caller
+//     provides it, else with six TMA boxes from the checkpoint layout; eight dequantisation warps
 //     expand it, exactly (fp16_rn((q - z) * s)), into an MN-major swizzled
 //     FP16 tile, and the MMA reads that.
 //
@@ -68,6 +70,9 @@ constexpr int Q_SCALES = Q_CODES + 64 * 16 * 4;
 constexpr int Q_ZEROS = Q_SCALES + 2 * 128 * 2;
 constexpr int Q_END = Q_ZEROS + 2 * 128;
 constexpr uint32_t Q_TX = 64 * 16 * 4 + 2 * 128 * 2 + 2 * 16 * 4;  // bytes the TMA brings per AWQ sub-tile
+constexpr int kAwqUnitBytes = 4736;  // one tile-packed AWQ unit (awq.cu): codes, scales, zeros of a sub-tile
+static_assert(Q_TX == kAwqUnitBytes && Q_SCALES == Q_CODES + 4096 && Q_ZEROS == Q_SCALES + 512,
+              "a packed AWQ unit is the sub-tile's staging image");
 // MN-major FP16 weight tile (AWQ): 64-element atoms along M are LBO apart,
 // 8-row K groups SBO apart; one MMA (K = 16) spans two K groups
 constexpr uint32_t AQ_LBO = (BK / 8) * 1024;
@@ -92,6 +97,7 @@ struct Args {
   const int* row_token; // [rows] token of each routed row
   const void* x;        // [T, H] 16-bit tokens
   float* partial;       // [I/64][rows + T][H] FP32
+  const uint8_t* qpack; // AWQ: tile-packed routed weights (awq.cu layout), or null (TMA from qc/qs/qz)
   int bf16;
   int* status;
   unsigned long long limit_ns;
@@ -272,14 +278,20 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
         if (lane == 0)
           mbar_arrive_expect_tx(&full_bar[stage], uint32_t(nsub) * (q ? Q_TX : uint32_t(A_BYTES)));
         __syncwarp();
-        // copy `lane` of the stage: per sub-tile 6 (AWQ phase A), 3 (AWQ
-        // phase B), 2 (16-bit phase A) or 1 (16-bit phase B)
-        const int per = q ? (pa ? 6 : 3) : (pa ? 2 : 1);
+        // copy `lane` of the stage: per sub-tile 1 (packed AWQ), 6 (AWQ
+        // phase A), 3 (AWQ phase B), 2 (16-bit phase A) or 1 (16-bit phase B)
+        const int per = q ? (args.qpack ? 1 : (pa ? 6 : 3)) : (pa ? 2 : 1);
         const int u = lane / per, which = lane - u * per;
         if (u < nsub) {
           uint8_t* d = sub(stage, u);
           uint64_t* fb = &full_bar[stage];
-          if (pa) {
+          if (q && args.qpack) {
+            // the sub-tile's packed unit: gate/up (j, kt) or down (j, m) of expert g
+            const int J = I / BK, nka = H / BK, nkb = H / BM;
+            const size_t unit = pa ? size_t(j) * nka + size_t(st * KSUB + u)
+                                   : size_t(J) * nka + size_t(j) * nkb + size_t(m0 + u);
+            bulk_load(d + Q_CODES, args.qpack + (size_t(g) * J * (nka + nkb) + unit) * kAwqUnitBytes, Q_TX, fb);
+          } else if (pa) {
             const int kx = (st * KSUB + u) * BK;
             if (q) {
               // gate columns 64j.., up columns I + 64j.. of the input-major codes
@@ -510,6 +522,8 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
     const int r0 = dt >> 4;  // 0..15
     const uint32_t atom_off = uint32_t(wc >> 3) * AQ_LBO;
     const uint32_t chunk = uint32_t(wc & 7);
+    const bool packed = args.qpack != nullptr;
+    static_assert(NRW == 4, "a packed unit holds four K rows per thread and code word");
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -533,15 +547,31 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
           for (int u = 0; u < KSUB; ++u) {
             if (u < nsub) {
               const uint8_t* d = sub(stage, u);
-              const uint32_t* codes = reinterpret_cast<const uint32_t*>(d + Q_CODES + half * 2048) + wl;
-              const uint16_t* sc = reinterpret_cast<const uint16_t*>(d + Q_SCALES + half * 256) + wl * 8;
-              const uint32_t* zr = reinterpret_cast<const uint32_t*>(d + Q_ZEROS + half * 128) + wl;
+              if (packed) {
+                // packed unit: this thread's four code words are adjacent; scales and
+                // zeros of word wc at column wc * 8 / word wc of each group's row
+                const uint4 c4 = *reinterpret_cast<const uint4*>(d + Q_CODES + (r0 * 16 + wc) * 16);
+                cv[u][0] = c4.x;
+                cv[u][1] = c4.y;
+                cv[u][2] = c4.z;
+                cv[u][3] = c4.w;
+                const uint16_t* sc = reinterpret_cast<const uint16_t*>(d + Q_SCALES) + wc * 8;
+                const uint32_t* zr = reinterpret_cast<const uint32_t*>(d + Q_ZEROS) + wc;
+                sv[u][0] = *reinterpret_cast<const uint4*>(sc);
+                sv[u][1] = *reinterpret_cast<const uint4*>(sc + 128);
+                z[u][0] = zr[0];
+                z[u][1] = zr[16];
+              } else {
+                const uint32_t* codes = reinterpret_cast<const uint32_t*>(d + Q_CODES + half * 2048) + wl;
+                const uint16_t* sc = reinterpret_cast<const uint16_t*>(d + Q_SCALES + half * 256) + wl * 8;
+                const uint32_t* zr = reinterpret_cast<const uint32_t*>(d + Q_ZEROS + half * 128) + wl;
 #pragma unroll
-              for (int i = 0; i < NRW; ++i) cv[u][i] = codes[(r0 + 16 * i) * cw];
-              sv[u][0] = *reinterpret_cast<const uint4*>(sc);
-              sv[u][1] = *reinterpret_cast<const uint4*>(sc + cw * 8);
-              z[u][0] = zr[0];
-              z[u][1] = zr[cw];
+                for (int i = 0; i < NRW; ++i) cv[u][i] = codes[(r0 + 16 * i) * cw];
+                sv[u][0] = *reinterpret_cast<const uint4*>(sc);
+                sv[u][1] = *reinterpret_cast<const uint4*>(sc + cw * 8);
+                z[u][0] = zr[0];
+                z[u][1] = zr[cw];
+              }
             }
           }
 #pragma unroll
@@ -683,15 +713,17 @@ int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t*
 
 // The same with the routed experts in AWQ W4A16 g32 (qw_* input-major codes,
 // qz_* zero points, sc_* FP16 scales; FP16 activations) and the shared
-// expert in FP16.
+// expert in FP16.  qpack: the tile-packed copy of the routed weights (awq.cu
+// awq_prepack) or null; when given, the kernel reads only it.
 int decode_experts_fused_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
                              int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
                              const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gu,
                              const void* w_sh_d, int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const void* qpack) {
   Args a;
   int rc = fill_args(a, x, row_token, offsets, T, rows, H, I, E, MOE_DTYPE_F16, ws, ws_bytes);
   if (rc) return rc;
+  a.qpack = static_cast<const uint8_t*>(qpack);
   Maps m;
   memset(&m, 0, sizeof(m));
   const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;

@@ -79,6 +79,12 @@ class MoELayer:
             self.I = weights["w_gate_up"].shape[1] // 2
         elif fmt == "awq_g32":
             self.I = weights["qw_gu"].shape[2] * 8 // 2
+            if T_max <= 16 and "awq_packed" not in weights:
+                # decode-sized layer: the routed weights also tile-packed, so that the
+                # weight-streaming kernel fetches each sub-tile with one bulk copy
+                self.w = weights = dict(weights)
+                weights["awq_packed"] = abi.moe_awq_prepack_g32(weights["qw_gu"], weights["qz_gu"], weights["sc_gu"],
+                                                                weights["qw_d"], weights["qz_d"], weights["sc_d"])
         elif fmt == "nvfp4":
             if "w_gu" not in weights:
                 self.w = weights = prepare_nvfp4_weights(weights)
@@ -177,6 +183,11 @@ class MoELayer:
             abi.moe_experts_bf16(x, self.row_token[:rows], self.offsets, rows, w["w_gate_up"], w["w_down"],
                                  w["w_sh_gate_up"], w["w_sh_down"], out_fp32=f.dtype == torch.float32, f=f,
                                  shared_out=sh, ws=self.ws_exp)
+        elif "awq_packed" in w:
+            abi.moe_experts_awq_g32_prepacked(x, self.row_token[:rows], self.offsets, rows, w["qw_gu"], w["qz_gu"],
+                                              w["sc_gu"], w["qw_d"], w["qz_d"], w["sc_d"], w["awq_packed"],
+                                              w["w_sh_gate_up"], w["w_sh_down"], out_fp32=f.dtype == torch.float32,
+                                              f=f, shared_out=sh, ws=self.ws_exp)
         else:
             abi.moe_experts_awq_g32(x, self.row_token[:rows], self.offsets, rows, w["qw_gu"], w["qz_gu"], w["sc_gu"],
                                     w["qw_d"], w["qz_d"], w["sc_d"], w["w_sh_gate_up"], w["w_sh_down"],

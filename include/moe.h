@@ -261,6 +261,38 @@ MOE_API int moe_experts_awq_g32(const void* x, const int32_t* row_token, const i
                                 void* shared_out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Tile-packed copy of one layer's routed AWQ weights [AWQ], made once, for
+ * the T <= 16 path of moe_experts_awq_g32_prepacked: the same codes, zero
+ * points and scales (no value changes, same total size) regrouped so that
+ * every 64-input-row sub-tile the decode kernel streams is one contiguous
+ * 4736-byte unit.  Inputs as in moe_grouped_swiglu_awq_g32; out: device
+ * buffer of moe_awq_packed_bytes(E, H, I) bytes, 16-byte aligned, owned by
+ * the caller (its layout is internal to the library).
+ * moe_awq_packed_bytes returns 0 for unsupported sizes.
+ * Limits: H % 128 == 0, I % 64 == 0; out_bytes large enough
+ * (MOE_ERR_WORKSPACE otherwise).
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_awq_packed_bytes(int E, int H, int I);
+MOE_API int moe_awq_prepack_g32(const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
+                                const int32_t* qz_d, const void* sc_d, int E, int H, int I, void* out,
+                                size_t out_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_experts_awq_g32 with the routed weights also given tile-packed
+ * (awq_packed, from moe_awq_prepack_g32 on the same qw/qz/sc): for T <= 16
+ * the decode kernel reads only awq_packed (one bulk copy per sub-tile
+ * instead of six tensor-map boxes); larger T reads qw/qz/sc as before.
+ * Results are identical to moe_experts_awq_g32's.  All other arguments,
+ * limits and the workspace as there; awq_packed must not be NULL.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_experts_awq_g32_prepacked(const void* x, const int32_t* row_token, const int32_t* expert_offsets,
+                                          int T, int rows, int H, int I, int E, const int32_t* qw_gu,
+                                          const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
+                                          const int32_t* qz_d, const void* sc_d, const void* awq_packed,
+                                          const void* w_sh_gate_up, const void* w_sh_down, int out_fp32, void* f,
+                                          void* shared_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * AWQ dequantisation [AWQ], the same device code the grouped GEMM runs on
  * each weight tile: out[b, k, n] = fp16_rn((q - z) * s) for `batch` stacked
  * projections in the layout above (qweight [batch, K, N/8], qzeros

@@ -96,3 +96,19 @@ def test_nvfp4_prepack_sizes_and_checks():
                  buf, None, None, 0, buf, None, 0, None) == abi.MOE_ERR_INVALID_ARG  # packed gate/up scales missing
     assert _code("moe_grouped_swiglu_nvfp4_prepacked", None, None, None, 0, 0, 256, 128, 4, None, None, None, None,
                  None, None, None, None, 0, None, None, 0, None) == abi.MOE_OK
+
+
+def test_awq_prepack_sizes_and_checks():
+    lib = abi.load()
+    # packed units: I/64 x (H/64 + H/128) per expert, 4736 bytes each = the AWQ bytes of an expert
+    assert lib.moe_awq_packed_bytes(512, 2048, 640) == 512 * 10 * 48 * 4736 == 512 * 2273280
+    assert lib.moe_awq_packed_bytes(4, 100, 64) == 0
+    buf = ctypes.c_void_p(256)  # never dereferenced: the checks come first
+    assert _code("moe_awq_prepack_g32", buf, buf, buf, buf, buf, buf, 4, 2048, 100, buf, 1 << 30, None) == \
+        abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_awq_prepack_g32", buf, buf, buf, None, buf, buf, 4, 2048, 640, buf, 1 << 30, None) == \
+        abi.MOE_ERR_INVALID_ARG
+    assert _code("moe_awq_prepack_g32", buf, buf, buf, buf, buf, buf, 4, 2048, 640, buf, 1000, None) == \
+        abi.MOE_ERR_WORKSPACE
+    assert _code("moe_experts_awq_g32_prepacked", buf, buf, buf, 1, 10, 2048, 640, 16, buf, buf, buf, buf, buf, buf,
+                 None, buf, buf, 0, buf, buf, buf, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG  # awq_packed is null

@@ -73,6 +73,50 @@ def test_experts_awq_routed_and_shared(T, H, I, E, k, out_fp32):
     sref, _ = moe.swiglu_expert(xs, sg[:I], sg[I:], f64(w["w_sh_down"]))
     err_sh = rel_err(f64(sh), sref)
     assert err_sh < 1e-2, err_sh
+    # the tile-packed weights give the same outputs, bit for bit (T <= 16 reads only them)
+    packed = abi.moe_awq_prepack_g32(w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"], w["qz_d"], w["sc_d"])
+    fp, shp = abi.moe_experts_awq_g32_prepacked(x, rt, off, T * k, w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"],
+                                                w["qz_d"], w["sc_d"], packed, w["w_sh_gate_up"], w["w_sh_down"],
+                                                out_fp32=out_fp32)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0
+    assert torch.equal(fp, f) and torch.equal(shp, sh)
+
+
+def test_awq_prepack_layout():
+    """Every byte of the tile-packed copy against the layout spelled out in
+    numpy: per expert the gate/up units (j, kt), then the down units (j, m);
+    per unit codes [r0][wc][i] (K row r0 + 16 i, code word wc), scales
+    [2 groups][128 columns], zeros [2 groups][16 words]."""
+    E, H, I = 3, 256, 128
+    wl = dataclasses.replace(synth.WORKLOADS["awq_g32"], H=H, I=I, I_sh=I, E=E, k=2)
+    w = synth.make_weights(wl, seed=7, device=DEV)
+    packed = abi.moe_awq_prepack_g32(w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"], w["qz_d"], w["sc_d"])
+    torch.cuda.synchronize()
+    got = packed.cpu().numpy()
+    h = {k: w[k].cpu().numpy() for k in ("qw_gu", "qz_gu", "sc_gu", "qw_d", "qz_d", "sc_d")}
+    J, nka, nkb = I // 64, H // 64, H // 128
+    units = []
+    for e in range(E):
+        for j in range(J):
+            for kt in range(nka):
+                words = [8 * j + c for c in range(8)] + [I // 8 + 8 * j + c for c in range(8)]
+                units.append((h["qw_gu"][e], h["qz_gu"][e], h["sc_gu"][e], 64 * kt, words))
+        for j in range(J):
+            for m in range(nkb):
+                units.append((h["qw_d"][e], h["qz_d"][e], h["sc_d"][e], 64 * j, [16 * m + c for c in range(16)]))
+    want = []
+    for qw, qz, sc, k0, words in units:
+        codes = np.array([[[qw[k0 + r0 + 16 * i, words[wc]] for i in range(4)] for wc in range(16)]
+                          for r0 in range(16)], dtype=np.int32)
+        cols = np.array([8 * words[c // 8] + c % 8 for c in range(128)])
+        scales = np.stack([sc[k0 // 32 + gi, cols] for gi in range(2)]).astype(np.float16)
+        zeros = np.stack([qz[k0 // 32 + gi, words] for gi in range(2)]).astype(np.int32)
+        want.append(np.concatenate([codes.view(np.uint8).ravel(), scales.view(np.uint8).ravel(),
+                                    zeros.view(np.uint8).ravel()]))
+    want = np.concatenate(want)
+    assert got.size == abi.load().moe_awq_packed_bytes(E, H, I) == want.size
+    assert np.array_equal(got, want)
 
 
 FFN_CASES = [
