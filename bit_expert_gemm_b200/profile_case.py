@@ -10,8 +10,8 @@ memory for a multi-pass capture).
 The routing is drawn by the library's own router (moe_route_permute) from
 the synthetic tokens and router weights, as in a layer forward; the expert
 call is the one MoELayer makes for the format: moe_experts_bf16 (routed +
-shared experts), moe_experts_awq_g32 (routed AWQ + FP16 shared experts) or
-moe_grouped_swiglu_nvfp4_prepacked (routed NVFP4 experts).
+shared experts), moe_experts_awq_g32_prepacked (routed AWQ + FP16 shared
+experts) or moe_grouped_swiglu_nvfp4_prepacked (routed NVFP4 experts).
 """
 
 from __future__ import annotations
@@ -56,9 +56,12 @@ def main(argv=None) -> None:
             abi.moe_grouped_swiglu_nvfp4_prepacked(xb, rt, off, rows, w["w_gu"], w["sfp_gu"], w["gs_gu"], w["w_d"],
                                                    w["sfp_d"], w["gs_d"])
     elif a.fmt == "awq_g32":
+        # as MoELayer does: decode-sized calls read the tile-packed copy of the routed weights
+        packed = abi.moe_awq_prepack_g32(w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"], w["qz_d"], w["sc_d"])
+
         def call():
-            abi.moe_experts_awq_g32(x, rt, off, rows, w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"], w["qz_d"],
-                                    w["sc_d"], w["w_sh_gate_up"], w["w_sh_down"])
+            abi.moe_experts_awq_g32_prepacked(x, rt, off, rows, w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"],
+                                              w["qz_d"], w["sc_d"], packed, w["w_sh_gate_up"], w["w_sh_down"])
     else:
         def call():
             abi.moe_experts_bf16(x, rt, off, rows, w["w_gate_up"], w["w_down"], w["w_sh_gate_up"], w["w_sh_down"])
