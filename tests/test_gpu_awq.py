@@ -48,7 +48,8 @@ def _awq_expert_fn(w, I):
     return ew
 
 
-@pytest.mark.parametrize("T,H,I,E,k,out_fp32", [(1, 2048, 640, 512, 10, False), (8, 512, 128, 16, 4, True),
+@pytest.mark.parametrize("T,H,I,E,k,out_fp32", [(1, 2048, 640, 512, 10, False), (2, 512, 128, 16, 4, False),
+                                                (4, 256, 256, 8, 2, True), (8, 512, 128, 16, 4, True),
                                                 (16, 1024, 192, 64, 6, False), (3, 256, 64, 16, 2, True),
                                                 (40, 512, 128, 16, 4, False)])
 def test_experts_awq_routed_and_shared(T, H, I, E, k, out_fp32):

@@ -157,7 +157,8 @@ def test_select_bit_exact(E):
 
 @pytest.mark.parametrize("T,H,I,E,k,out_fp32,act", [
     # T <= 16: one split-K kernel + partial sums
-    (1, 2048, 640, 512, 10, False, "bf16"), (8, 512, 128, 16, 4, False, "bf16"), (3, 256, 64, 16, 2, False, "bf16"),
+    (1, 2048, 640, 512, 10, False, "bf16"), (2, 512, 128, 16, 4, True, "bf16"), (4, 256, 256, 16, 3, False, "f16"),
+    (3, 512, 384, 32, 2, False, "bf16"), (8, 512, 128, 16, 4, False, "bf16"), (3, 256, 64, 16, 2, False, "bf16"),
     (16, 1024, 192, 64, 6, True, "bf16"), (5, 384, 128, 32, 4, False, "f16"),
     # 16 < T <= 128: two weight-streaming GEMMs
     (17, 512, 128, 16, 3, False, "bf16"), (64, 2048, 640, 64, 10, True, "bf16"), (128, 256, 64, 16, 2, False, "bf16"),
