@@ -18,11 +18,16 @@
 // reads: copies issued by the MMA thread itself into one shared slot held
 // the MMA pipe to about a third of its rate.
 //
+// With row_token, A rows are gathered in the kernel: four gather warps copy
+// the 128-byte row segments of each K step from the per-token source with
+// cp.async straight into the 128-byte-swizzled A tile (the layout the TMA
+// would write), arriving on the stage barrier; rows past the group read zero.
+//
 // Warp roles: 0 and 8 TMA producers (A with its scales, B with its scales:
 // one thread issuing every copy of a stage held the loads to about 86 GB/s
 // per SM, since copy instructions block while the TMA unit is busy),
 // 1 UMMA issuer (TMEM owner), 2..5 epilogue, 6 and 7 scale-factor copies
-// (A and B).
+// (A and B), 9..12 A-row gather (with row_token).
 #include <cstring>
 
 #include "common.cuh"
@@ -49,7 +54,8 @@ constexpr int STAGE_BYTES = SFB_OFF + 4 * SF_ATOM;  // 36 KB
 #endif
 constexpr int STAGES = NVFP4_STAGES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-constexpr int kThreads = 288;
+constexpr int kThreads = 416;
+constexpr int kGatherWarp0 = 9;
 constexpr int SF_TILE = 4 * SF_ATOM;     // scales of one operand tile for one K step
 constexpr uint32_t TMEM_COLS = 512;      // 2 x 128 accumulator + a scale slot per stage
 constexpr uint32_t SF_COL = 2 * BN;      // slot s at SF_COL + 32 s: A (4 MMAs x 4 columns), then B
@@ -69,6 +75,9 @@ struct Args {
   void* out;
   int ldo, out_fp32;
   float* amax_out;  // SwiGLU: atomic max of |h| (float bits), may be null
+  const int32_t* row_token;  // gathered A: A row r = source row row_token[r], or null (A rows in order)
+  const uint8_t* a_src;      // gathered A: [a_src_rows, K/2] codes
+  int a_src_rows;
   int* status;
   unsigned long long limit_ns;
 };
@@ -106,6 +115,13 @@ constexpr uint32_t kIdescMxf4 = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 1
 struct TileMap {
   int g, m, n;
 };
+
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 __device__ void build_tile_table(const Args& a, int* goff, int* tile_start, int* warp_sums) {
   const int G = a.G, tid = threadIdx.x;
@@ -171,7 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 2);  // one expect_tx arrival from each producer
+      // one expect_tx arrival from each producer (+ one per gather thread)
+      mbar_init(&full_bar[s], 2 + (args.row_token ? 128 : 0));
       mbar_init(&empty_bar[s], 1);
       mbar_init(&sfready_bar[s], 2);  // one tcgen05.commit from each copy warp
     }
@@ -222,8 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
           if (pa) {
-            mbar_arrive_expect_tx(&full_bar[stage], A_BYTES + SF_TILE);
-            tma_load_2d(stg(stage), &tmA, &full_bar[stage], kt * BKB, a_row);
+            const bool gathered = args.row_token != nullptr;  // then the gather warps bring A
+            mbar_arrive_expect_tx(&full_bar[stage], (gathered ? 0 : A_BYTES) + SF_TILE);
+            if (!gathered) tma_load_2d(stg(stage), &tmA, &full_bar[stage], kt * BKB, a_row);
             bulk_load(stg(stage) + SFA_OFF, args.sfa + (size_t(tile_start[t.g] + t.m) * KT + kt) * SF_TILE, SF_TILE,
                       &full_bar[stage]);
           } else {
@@ -282,6 +300,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&drain_bar);
       volatile int never = 0;
       mbar_wait(&drain_bar, 0, &never, nullptr, lim);
+    }
+  } else if (warp >= kGatherWarp0) {
+    if (args.row_token) {
+      // ---------------- A row gather: warps 9..12 ----------------
+      // Thread gt copies 16-byte chunk (gt % 8) of tile rows gt/8, gt/8 + 16, ...
+      const int gt = threadIdx.x - kGatherWarp0 * 32;
+      const int chunk = gt & 7, rbase = gt >> 3;
+      const size_t pitch = size_t(args.K) / 2;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        TileMap t = decode_tile(L, nt, tile_start, G);
+        const int a_row = goff[t.g] + t.m * BM;
+        const int g_end = goff[t.g + 1];
+        int tok[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = a_row + rbase + 16 * i;
+          const int tk = (r < g_end && r < args.rows) ? __ldg(args.row_token + r) : -1;
+          tok[i] = (tk >= 0 && tk < args.a_src_rows) ? tk : -1;
+        }
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
+          const uint32_t dst0 = smem_u32(stg(stage));
+          const size_t kb = size_t(kt) * BKB + size_t(chunk) * 16;  // byte of the row
+          const bool in_k = kb < pitch;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = rbase + 16 * i;
+            const uint32_t dst = dst0 + uint32_t(r * 128 + ((chunk ^ (r & 7)) << 4));
+            const bool v = tok[i] >= 0 && in_k;
+            const uint8_t* g = args.a_src + (v ? size_t(tok[i]) * pitch + kb : 0);
+            cp_async_16_zfill(dst, g, v ? 16u : 0u);
+          }
+          cp_async_arrive_noinc(&full_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");  // every copy has landed before the CTA exits
     }
   } else if (warp == 6 || warp == 7) {
     if (lane == 0) {
@@ -407,7 +465,7 @@ int launch_grouped_gemm_nvfp4(const uint8_t* A, const uint8_t* sfa, int a_rows, 
                               int b_rows_total, const int* group_offsets, int G, int rows, int K, int n_out,
                               int b_rows_per_group, int up_offset, int swiglu, const float* gs_act,
                               const float* gs_w, int gs_w_stride, void* out, int ldo, int out_fp32, float* amax_out,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, const int32_t* row_token) {
   MOE_REQUIRE(K % 64 == 0 && K > 0, MOE_ERR_UNSUPPORTED, "NVFP4 GEMM K=%d is not a positive multiple of 64", K);
   MOE_REQUIRE(G >= 1 && G <= kGemmMaxGroups, MOE_ERR_UNSUPPORTED, "NVFP4 GEMM group count %d", G);
   const int bnh = swiglu ? BN / 2 : BN;
@@ -438,6 +496,9 @@ int launch_grouped_gemm_nvfp4(const uint8_t* A, const uint8_t* sfa, int a_rows, 
   a.ldo = ldo;
   a.out_fp32 = out_fp32;
   a.amax_out = amax_out;
+  a.row_token = row_token;  // A = per-source rows [a_rows, K/2], gathered through row_token
+  a.a_src = A;
+  a.a_src_rows = a_rows;
   a.status = device_status_ptr();
   a.limit_ns = wait_limit_ns();
   static bool attr_set[64] = {false};

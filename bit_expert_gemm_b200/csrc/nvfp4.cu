@@ -13,7 +13,7 @@ int launch_grouped_gemm_nvfp4(const uint8_t* A, const uint8_t* sfa, int a_rows, 
                               int b_rows_total, const int* group_offsets, int G, int rows, int K, int n_out,
                               int b_rows_per_group, int up_offset, int swiglu, const float* gs_act,
                               const float* gs_w, int gs_w_stride, void* out, int ldo, int out_fp32, float* amax_out,
-                              cudaStream_t stream);
+                              cudaStream_t stream, const int32_t* row_token);
 
 // amax[b] = max |v| over tensor b of `batch` tensors of `n` 16-bit values
 // (stored as float bits: non-negative floats order like integers).
@@ -82,26 +82,6 @@ __global__ void __launch_bounds__(256) k_nvfp4_quant(const T16* __restrict__ v, 
   sf[out_row * nb + blk] = uint8_t(s);
 }
 
-// Gathers NVFP4 rows: out row r = row row_token[r] of the codes [*, K/2] and
-// scales [*, K/16]; one warp per row (K % 64 == 0).
-__global__ void __launch_bounds__(256) k_gather_fp4_rows(const uint8_t* __restrict__ codes,
-                                                         const uint8_t* __restrict__ sf,
-                                                         const int32_t* __restrict__ row_token, int rows, int K,
-                                                         uint8_t* __restrict__ codes_out, uint8_t* __restrict__ sf_out) {
-  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  const size_t t = size_t(row_token[r]);
-  const int nc = K / 32;  // 16-byte chunks of codes per row
-  const uint4* cs = reinterpret_cast<const uint4*>(codes + t * (K / 2));
-  uint4* cd = reinterpret_cast<uint4*>(codes_out + size_t(r) * (K / 2));
-  for (int c = lane; c < nc; c += 32) cd[c] = __ldg(cs + c);
-  const int ns = K / 64;  // 4-byte words of scales per row
-  const uint32_t* ss = reinterpret_cast<const uint32_t*>(sf + t * (K / 16));
-  uint32_t* sd = reinterpret_cast<uint32_t*>(sf_out + size_t(r) * (K / 16));
-  for (int c = lane; c < ns; c += 32) sd[c] = __ldg(ss + c);
-}
-
 // ---------------------------------------------------------------------------
 // Scale factors in the block-scaled GEMM's operand-tile order.  For operand
 // tile t (128 rows) and K step kt (256 elements = 16 scales per row): four
@@ -150,11 +130,14 @@ __global__ void __launch_bounds__(1024) k_tile_starts(const int32_t* __restrict_
 }
 
 // A operand (activations in permuted row order): tile t is rows
-// offsets[g] + 128 m .. of group g, t = tile_start[g] + m.  Grid (max tiles,
-// KT), 128 threads (one per tile row).
+// offsets[g] + 128 m .. of group g, t = tile_start[g] + m; with row_token the
+// scales of permuted row r are those of source row row_token[r].  Grid (max
+// tiles, KT), 128 threads (one per tile row).
 __global__ void __launch_bounds__(128) k_pack_sf_a(const uint8_t* __restrict__ sf, int K,
                                                    const int32_t* __restrict__ offsets, int G,
-                                                   const int32_t* __restrict__ tile_start, uint8_t* __restrict__ out) {
+                                                   const int32_t* __restrict__ tile_start,
+                                                   const int32_t* __restrict__ row_token, int src_rows,
+                                                   uint8_t* __restrict__ out) {
   const int t = blockIdx.x, kt = blockIdx.y, i = threadIdx.x;
   if (t >= tile_start[G]) return;
   int lo = 0, hi = G - 1;
@@ -164,8 +147,13 @@ __global__ void __launch_bounds__(128) k_pack_sf_a(const uint8_t* __restrict__ s
   }
   const int m = t - tile_start[lo];
   const long row = long(offsets[lo]) + long(m) * 128 + i;
-  pack_sf_row(sf, K / 16, row < offsets[lo + 1], size_t(row), kt, i,
-              out + (size_t(t) * gridDim.y + kt) * kSfTileBytes);
+  bool valid = row < offsets[lo + 1];
+  long src = row;
+  if (valid && row_token) {
+    src = row_token[row];
+    valid = src >= 0 && src < src_rows;
+  }
+  pack_sf_row(sf, K / 16, valid, size_t(valid ? src : 0), kt, i, out + (size_t(t) * gridDim.y + kt) * kSfTileBytes);
 }
 
 // B operand (weights): tile (g, n) is, for SwiGLU, the 64 gate rows n*64.. and
@@ -232,9 +220,10 @@ int nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const f
 
 // ---------------------------------------------------------------------------
 // Grouped SwiGLU with NVFP4 weights and on-the-fly NVFP4 activations:
-//   amax(x) -> quantise each token -> gather the FP4 rows -> scales in tile
-//   order -> GEMM1 (+SwiGLU, h in BF16, amax(h)) -> quantise h -> scales in
-//   tile order -> GEMM2.
+//   amax(x) -> quantise each token -> scales of the permuted rows in tile
+//   order -> GEMM1 (gathering the FP4 rows of the permuted order itself;
+//   +SwiGLU, h in BF16, amax(h)) -> quantise h -> scales in tile order ->
+//   GEMM2.
 // ---------------------------------------------------------------------------
 struct Nvfp4Ws {
   uint8_t *xq, *xsf, *xq_tok, *xsf_tok, *hq, *hsf;
@@ -306,23 +295,20 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
   }
   MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_grouped_swiglu_nvfp4: workspace of %zu bytes is too small", ws_bytes);
   if (rows == 0) return MOE_OK;
-  // x: amax over the whole [T, H] input, each token quantised once, then the
-  // FP4 rows gathered in permuted order (identical to quantising the gathered
-  // rows: the quantisation is per row with the one global scale of x)
-  // (identity rows, row_token == NULL: quantised in place, no gather)
+  // x: amax over the whole [T, H] input, each token quantised once; GEMM1
+  // reads the FP4 rows of the permuted order through row_token (identical to
+  // quantising the gathered rows: the quantisation is per row with the one
+  // global scale of x), and the scale packing reads the per-token scales the
+  // same way (identity rows, row_token == NULL: quantised in place)
   int rc = quantize_rows(x, MOE_DTYPE_BF16, nullptr, 1, T, H, 0, long(T) * H, act_gs_in, w.amax,
                          row_token ? w.xq_tok : w.xq, row_token ? w.xsf_tok : w.xsf, w.gs, stream);
   if (rc) return rc;
-  if (row_token) {
-    k_gather_fp4_rows<<<(rows * 32 + 255) / 256, 256, 0, stream>>>(w.xq_tok, w.xsf_tok, row_token, rows, H, w.xq,
-                                                                    w.xsf);
-    MOE_CHECK_CUDA(cudaGetLastError());
-  }
   // scale factors in GEMM tile order: A tiles of the permuted rows, B tiles of the weights
   const int tiles = (rows + 127) / 128 + E;
   const int kt1 = (H + 255) / 256, kt2 = (I + 255) / 256;
   k_tile_starts<<<1, 1024, 0, stream>>>(offsets, E, w.tile_start);
-  k_pack_sf_a<<<dim3(tiles, kt1), 128, 0, stream>>>(w.xsf, H, offsets, E, w.tile_start, w.xsf_p);
+  k_pack_sf_a<<<dim3(tiles, kt1), 128, 0, stream>>>(row_token ? w.xsf_tok : w.xsf, H, offsets, E, w.tile_start,
+                                                    row_token, T, w.xsf_p);
   const uint8_t* w1sf = w1sf_packed;
   if (!w1sf) {  // weight scales not packed by the caller: pack them for this call
     k_pack_sf_b<<<dim3(E * (I / 64), kt1), 128, 0, stream>>>(sf_gu, H, I / 64, 2 * I, 1, I, w.w1sf_p);
@@ -330,13 +316,15 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
   }
   MOE_CHECK_CUDA(cudaGetLastError());
   MOE_CHECK_CUDA(cudaMemsetAsync(w.amax + 1, 0, sizeof(unsigned), stream));
-  rc = launch_grouped_gemm_nvfp4(w.xq, w.xsf_p, rows, w_gu, w1sf, E * 2 * I, offsets, E, rows, H, I, 2 * I, I, 1,
-                                 w.gs, gs_gu, 2, w.h, I, 0, reinterpret_cast<float*>(w.amax + 1), stream);
+  // A: the per-token FP4 rows gathered in the GEMM (row_token), or the rows in order
+  rc = launch_grouped_gemm_nvfp4(row_token ? w.xq_tok : w.xq, w.xsf_p, row_token ? T : rows, w_gu, w1sf, E * 2 * I,
+                                 offsets, E, rows, H, I, 2 * I, I, 1, w.gs, gs_gu, 2, w.h, I, 0,
+                                 reinterpret_cast<float*>(w.amax + 1), stream, row_token);
   if (rc) return rc;
   rc = quantize_rows(w.h, MOE_DTYPE_BF16, nullptr, 1, rows, I, 0, 0, act_gs_in ? act_gs_in + 1 : nullptr, w.amax + 1,
                      w.hq, w.hsf, w.gs + 1, stream);
   if (rc) return rc;
-  k_pack_sf_a<<<dim3(tiles, kt2), 128, 0, stream>>>(w.hsf, I, offsets, E, w.tile_start, w.hsf_p);
+  k_pack_sf_a<<<dim3(tiles, kt2), 128, 0, stream>>>(w.hsf, I, offsets, E, w.tile_start, nullptr, rows, w.hsf_p);
   const uint8_t* w2sf = w2sf_packed;
   if (!w2sf) {
     k_pack_sf_b<<<dim3(E * (H / 128), kt2), 128, 0, stream>>>(sf_d, I, H / 128, H, 0, 0, w.w2sf_p);
@@ -344,7 +332,7 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
   }
   MOE_CHECK_CUDA(cudaGetLastError());
   rc = launch_grouped_gemm_nvfp4(w.hq, w.hsf_p, rows, w_d, w2sf, E * H, offsets, E, rows, I, H, H, 0, 0, w.gs + 1,
-                                 gs_d, 1, f, H, out_fp32, nullptr, stream);
+                                 gs_d, 1, f, H, out_fp32, nullptr, stream, nullptr);
   if (rc) return rc;
   if (act_gs_out) MOE_CHECK_CUDA(cudaMemcpyAsync(act_gs_out, w.gs, 2 * sizeof(float), cudaMemcpyDeviceToDevice, stream));
   return MOE_OK;
