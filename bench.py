@@ -83,19 +83,26 @@ def parse():
 # distributed plumbing (one process per GPU; no collective in the data path)
 # ---------------------------------------------------------------------------
 class Dist:
-    def __init__(self):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE): NCCL
+    for the barrier and the max over ranks of the device-timed region; gloo
+    on hosts without CUDA (the CPU tests of this logic)."""
+
+    def __init__(self, backend: str = ""):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
         if self.world > 1:
             import datetime
 
             import torch.distributed as dist
 
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {}
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=300), **kw)
             self.pg = dist
 
     def barrier(self):
@@ -105,7 +112,7 @@ class Dist:
     def max(self, v: float) -> float:
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device="cuda" if self.backend == "nccl" else "cpu")
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 

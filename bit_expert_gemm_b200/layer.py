@@ -245,6 +245,31 @@ class MoELayer:
         return y
 
 
+def refill_allreduce(sum_sq: torch.Tensor, count: torch.Tensor, group=None) -> None:
+    """Combines the Refill-RMS statistics of all ranks in place: every rank
+    ends with the sums and counts of the whole data set, so razor_select
+    keeps the same experts everywhere.  The statistics are additive; they are
+    gathered and added in rank order (not reduced by the collective), so the
+    FP64 sums, and the selection, do not depend on the reduction order.
+    sum_sq [E] FP64 and count [E] int64, on the device of the process group's
+    backend (CUDA for NCCL, CPU for gloo)."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    if world == 1:
+        return
+    parts_s = [torch.empty_like(sum_sq) for _ in range(world)]
+    parts_c = [torch.empty_like(count) for _ in range(world)]
+    dist.all_gather(parts_s, sum_sq.contiguous(), group=group)
+    dist.all_gather(parts_c, count.contiguous(), group=group)
+    total_s, total_c = parts_s[0].clone(), parts_c[0].clone()
+    for ps, pc in zip(parts_s[1:], parts_c[1:]):
+        total_s += ps
+        total_c += pc
+    sum_sq.copy_(total_s)
+    count.copy_(total_c)
+
+
 class HostPipeline:
     """Streams token batches from pinned host memory through one layer and
     back, overlapping the upload of batch i+1 and the download of batch i-1
