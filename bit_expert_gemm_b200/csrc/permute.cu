@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(256) k_perm_setbits(const int32_t* __restrict_
 // One block per expert: popcount prefix over the expert's words.
 __global__ void __launch_bounds__(256) k_perm_expert_scan(const uint32_t* __restrict__ mask, int W,
                                                           int32_t* __restrict__ wordpre, int32_t* __restrict__ count) {
+  griddep_wait();  // the mask comes from the kernel before (programmatic dependent launch in route_permute)
+  griddep_launch_dependents();
   const int e = blockIdx.x;
   const uint32_t* m = mask + size_t(e) * W;
   int32_t* pre = wordpre + size_t(e) * W;
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(256) k_perm_expert_scan(const uint32_t* __rest
 // One block of 1024 threads: exclusive scan of count[0..E) -> offsets[0..E].
 __global__ void __launch_bounds__(1024) k_perm_offsets(const int32_t* __restrict__ count, int E,
                                                        int32_t* __restrict__ offsets) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ int warp_tot[32];
   const int i = threadIdx.x;
   const int v = i < E ? count[i] : 0;
@@ -81,6 +85,8 @@ __global__ void __launch_bounds__(256) k_perm_scatter(const int32_t* __restrict_
                                                       const int32_t* __restrict__ offsets,
                                                       int32_t* __restrict__ row_token,
                                                       int32_t* __restrict__ slot_row) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int e = idx[i];
@@ -143,6 +149,24 @@ int permute(const int32_t* topk_idx, int T, int ks, int E, int32_t* offsets, int
                                                         slot_row);
     MOE_CHECK_CUDA(cudaGetLastError());
   }
+  return MOE_OK;
+}
+
+// The permutation from an expert bitmask already built (route_permute: the
+// top-k kernel sets the bits): per-expert scan, offsets, scatter, each a
+// programmatic dependent of the kernel before.  mask, wordpre [E * W], count [E]
+// from the permutation workspace.
+int permute_from_mask(const int32_t* topk_idx, int T, int ks, int E, const uint32_t* mask, int32_t* wordpre,
+                      int32_t* count, int32_t* offsets, int32_t* row_token, int32_t* slot_row, cudaStream_t stream) {
+  const int W = (T + 31) / 32;
+  const int n = T * ks;
+  MOE_CHECK_CUDA(launch_pdl(k_perm_expert_scan, dim3(E), dim3(256), 0, stream, mask, W, wordpre, count));
+  MOE_CHECK_CUDA(launch_pdl(k_perm_offsets, dim3(1), dim3(1024), 0, stream, static_cast<const int32_t*>(count), E,
+                            offsets));
+  if (n > 0)
+    MOE_CHECK_CUDA(launch_pdl(k_perm_scatter, dim3((n + 255) / 256), dim3(256), 0, stream, topk_idx, n, ks, E, W, mask,
+                              static_cast<const int32_t*>(wordpre), static_cast<const int32_t*>(offsets), row_token,
+                              slot_row));
   return MOE_OK;
 }
 

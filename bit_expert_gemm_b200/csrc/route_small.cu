@@ -28,6 +28,11 @@ size_t permute_ws_bytes(int T, int E);
 int route_topk(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
                int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, void* ws, size_t ws_bytes,
                cudaStream_t stream);
+int route_topk_bits(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
+                    int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, void* ws, size_t ws_bytes,
+                    uint32_t* mask, cudaStream_t stream);
+int permute_from_mask(const int32_t* topk_idx, int T, int ks, int E, const uint32_t* mask, int32_t* wordpre,
+                      int32_t* count, int32_t* offsets, int32_t* row_token, int32_t* slot_row, cudaStream_t stream);
 int permute(const int32_t* topk_idx, int T, int ks, int E, int32_t* offsets, int32_t* row_token, int32_t* slot_row,
             void* ws, size_t ws_bytes, cudaStream_t stream);
 
@@ -203,10 +208,17 @@ int route_permute(const void* x, int T, int H, const void* w_router, const float
     void* ws_r = carve.take<uint8_t>(route_ws_bytes(T, E));
     void* ws_p = carve.take<uint8_t>(permute_ws_bytes(T, E));
     MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_route_permute: workspace of %zu bytes is too small", ws_bytes);
-    int rc = route_topk(x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w, topk_logit, ws_r,
-                        route_ws_bytes(T, E), stream);
+    // router GEMM, top-k setting the expert bitmask as it selects, then the
+    // per-expert scan, offsets and scatter as programmatic dependents
+    WsCarver pc(ws_p, permute_ws_bytes(T, E));
+    const int W = (T + 31) / 32;
+    uint32_t* mask = pc.take<uint32_t>(size_t(E) * W);
+    int32_t* wordpre = pc.take<int32_t>(size_t(E) * W);
+    int32_t* count = pc.take<int32_t>(size_t(E));
+    int rc = route_topk_bits(x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w, topk_logit, ws_r,
+                             route_ws_bytes(T, E), mask, stream);
     if (rc) return rc;
-    return permute(topk_idx, T, ks, E, offsets, row_token, slot_row, ws_p, permute_ws_bytes(T, E), stream);
+    return permute_from_mask(topk_idx, T, ks, E, mask, wordpre, count, offsets, row_token, slot_row, stream);
   }
   WsCarver carve(ws, ws_bytes);
   float* logits = carve.take<float>(size_t(T) * E);
