@@ -132,6 +132,14 @@ def make_weights(wl: Workload, seed: int = 0, device="cpu", E: Optional[int] = N
     return w
 
 
+def make_shared_gate(wl: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
+    """Optional shared-expert gate vector [H] ~ N(0, 1/sqrt(H)) in the
+    activation dtype, from its own generator (the layer's other draws are
+    unchanged by it)."""
+    g = _gen(7_777_777 + seed, device)
+    return _normal(g, (wl.H,), wl.H ** -0.5, _dt(wl.act), device)
+
+
 def make_tokens(wl: Workload, T: int, seed: int = 0, batch: int = 0, device="cpu") -> torch.Tensor:
     """x [T, H] ~ N(0, 1) in the workload's activation dtype."""
     g = _gen(1_000_003 * (seed + 1) + 7919 * T + 104_729 * batch, device)

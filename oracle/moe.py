@@ -20,7 +20,9 @@ Readings where the pages are silent (each is listed in the design doc):
 * ties in the expert order go to the lower expert index;
 * within one expert the permuted rows are in ascending token order;
 * SwiGLU is silu(gate) * up with silu(g) = g / (1 + exp(-g));
-* the shared expert is added to the routed sum without a gate.
+* the shared expert is added to the routed sum without a gate; the AWQ
+  card lists a shared-expert gate tensor without its formula, and where one
+  is given it is read as a logistic gate per token, sigmoid(x . w_gate).
 """
 
 from __future__ import annotations
@@ -136,6 +138,13 @@ def combine(f_rows: np.ndarray, slot_row: np.ndarray, w: np.ndarray, shared: Opt
     return y
 
 
+def shared_gate(x: np.ndarray, w_gate: np.ndarray) -> np.ndarray:
+    """Per-token shared-expert gate 1 / (1 + exp(-x . w_gate)).
+    x [T, H], w_gate [H] -> [T]."""
+    z = np.asarray(x, np.float64) @ np.asarray(w_gate, np.float64)
+    return 1.0 / (1.0 + np.exp(-z))
+
+
 ExpertFn = Callable[[int], Sequence[np.ndarray]]
 
 
@@ -160,9 +169,11 @@ def routed_outputs(x: np.ndarray, perm: dict, expert_weights: ExpertFn):
     return f, h_all
 
 
-def moe_layer(x, w_router, bias, k: int, expert_weights: ExpertFn, shared_weights=None, extra: int = 0) -> dict:
+def moe_layer(x, w_router, bias, k: int, expert_weights: ExpertFn, shared_weights=None, extra: int = 0,
+              shared_gate_w=None) -> dict:
     """The whole routed-expert layer on tokens x [T, H] (float64):
-    route -> permute -> per-expert SwiGLU -> weighted combine (+ shared).
+    route -> permute -> per-expert SwiGLU -> weighted combine (+ shared,
+    times the per-token gate when shared_gate_w [H] is given).
     Returns route / permutation intermediates, f, h and y."""
     x = np.asarray(x, np.float64)
     E = np.asarray(w_router).shape[0]
@@ -172,5 +183,7 @@ def moe_layer(x, w_router, bias, k: int, expert_weights: ExpertFn, shared_weight
     shared = None
     if shared_weights is not None:
         shared, _ = swiglu_expert(x, *shared_weights)
+        if shared_gate_w is not None:
+            shared = shared * shared_gate(x, shared_gate_w)[:, None]
     y = combine(f, perm["slot_row"], r["w"], shared)
     return dict(route=r, perm=perm, f=f, h=h, shared=shared, y=y)

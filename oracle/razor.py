@@ -14,7 +14,9 @@ and calibration":
 * the statistics are additive: existing ones were reused and recombined.
 The opening paragraphs add that the kept experts' weights and router rows are
 sliced "in matching order" and that the keep manifest lists original expert
-indices in output order.
+indices in output order.  The MTP item of the same section keeps the MTP
+layer's experts by the L2 norm of their original router rows
+(mtp_policy=router_norm), because the text calibration never runs that layer.
 
 Readings (listed in DESIGN.md): "local output" is the MoE block output, so
 the shared expert cancels; the change is measured with the L2 norm over the
@@ -124,3 +126,27 @@ def select(sum_sq: np.ndarray, count: np.ndarray, keep: int):
     ranking = np.lexsort((np.arange(E), -s))  # primary: -score, secondary: index
     kept = np.sort(ranking[:keep])
     return kept, ranking, s
+
+
+def router_norm(w_router: np.ndarray) -> np.ndarray:
+    """mtp_policy=router_norm: ||w_router[e, :]||_2 for every expert e."""
+    w = np.asarray(w_router, np.float64)
+    return np.sqrt(np.sum(w * w, axis=1))
+
+
+def select_by_router_norm(w_router: np.ndarray, keep: int):
+    """Keep the `keep` experts of largest router-row norm, ties to the lower
+    index; same return values as select()."""
+    w = np.asarray(w_router, np.float64)
+    return select(np.sum(w * w, axis=1), np.ones(w.shape[0], np.int64), keep)
+
+
+def slice_experts(a: np.ndarray, kept) -> np.ndarray:
+    """The kept experts' blocks in output order: out[j] = a[kept[j]], for any
+    tensor whose leading axis is the expert index (router rows, bias, expert
+    weights)."""
+    a = np.asarray(a)
+    out = np.empty((len(kept),) + a.shape[1:], a.dtype)
+    for j, e in enumerate(kept):
+        out[j] = a[int(e)]
+    return out

@@ -152,3 +152,35 @@ def test_expert_structure_matches_published_parameter_counts():
     # and the assumed H = 2048 of the graded workloads would not reproduce them
     d2 = 2048
     assert g["main_base"] - g["main_keep256"] != L * 256 * (3 * d2 * I + d2)
+
+
+def test_shared_gate_closed_forms_and_library():
+    from scipy.special import expit
+
+    x = np.array([[1.0, 2.0], [-3.0, 0.5], [0.0, 0.0]])
+    g = np.array([0.5, -1.0])
+    assert np.allclose(moe.shared_gate(x, g), expit(x @ g), rtol=1e-15)
+    assert np.array_equal(moe.shared_gate(x, np.zeros(2)), np.full(3, 0.5))  # a zero gate halves the shared expert
+    assert moe.shared_gate(np.array([[40.0]]), np.array([1.0]))[0] == 1.0
+    assert moe.shared_gate(np.array([[-40.0]]), np.array([1.0]))[0] < 1e-17
+
+
+def test_layer_with_gate_scales_only_the_shared_expert():
+    wl = synth.WORKLOADS["tiny"]
+    w = synth.make_weights(wl, 4)
+    x = synth.make_tokens(wl, 32, 4).double().numpy()
+    gu, wd = w["w_gate_up"].double().numpy(), w["w_down"].double().numpy()
+    I = wl.I
+    ew = lambda e: (gu[e, :I], gu[e, I:], wd[e])  # noqa: E731
+    shg = w["w_sh_gate_up"].double().numpy()
+    sh = (shg[:I], shg[I:], w["w_sh_down"].double().numpy())
+    g = synth.make_shared_gate(wl, 4).double().numpy()
+    wr, b = w["w_router"].double().numpy(), w["bias"].double().numpy()
+    plain = moe.moe_layer(x, wr, b, wl.k, ew, sh)
+    routed = moe.moe_layer(x, wr, b, wl.k, ew, None)
+    gated = moe.moe_layer(x, wr, b, wl.k, ew, sh, shared_gate_w=g)
+    s_only = plain["y"] - routed["y"]
+    z = x @ g
+    assert np.allclose(gated["y"], routed["y"] + s_only / (1.0 + np.exp(-z))[:, None], rtol=1e-12, atol=1e-12)
+    half = moe.moe_layer(x, wr, b, wl.k, ew, sh, shared_gate_w=np.zeros_like(g))
+    assert np.allclose(half["y"], routed["y"] + 0.5 * s_only, rtol=1e-12, atol=1e-12)
