@@ -25,6 +25,7 @@ sample of the same workload on this machine's host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import glob
 import hashlib
 import json
@@ -42,7 +43,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from bit_expert_gemm_b200 import MoELayer, abi, synth  # noqa: E402
-from bit_expert_gemm_b200.layer import HostPipeline  # noqa: E402
+from bit_expert_gemm_b200.layer import HostPipeline, slice_layer_weights  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at E=512,k=10 (prefill TFLOP/s & decode HBM GB/s vs roofline)"
 L2_BYTES = 126 * 1024 * 1024
@@ -58,11 +59,22 @@ WORKLOADS = {
     "awq_decode_t8": ("awq_g32", 8, "forward"),
     "awq_decode_t32": ("awq_g32", 32, "forward"),
     "nvfp4_prefill": ("nvfp4", 16384, "forward"),
+    "nvfp4_decode_t1": ("nvfp4", 1, "forward"),
+    "nvfp4_decode_t64": ("nvfp4", 64, "forward"),
     "bf16_h2560_prefill": ("bf16_h2560", 8192, "forward"),
     # small case of the same kernels for full ncu captures (64 experts, 2048 tokens)
     "profile_e64_t2048": ("profile_e64", 2048, "forward"),
     "refill": ("refill", 32768, "refill"),
+    # RAZOR-pruned layers (the 65B and 96B budgets): the E=512 BF16 layer's
+    # Refill-RMS statistics over one 32768-token calibration row, the top 256
+    # or 384 experts kept, router rows, bias and expert weights sliced on the
+    # device, then the forward of the pruned layer
+    "bf16_razor256_prefill": ("bf16", 8192, "forward"),
+    "bf16_razor384_prefill": ("bf16", 8192, "forward"),
+    "bf16_razor256_decode_t1": ("bf16", 1, "forward"),
 }
+PRUNED = {"bf16_razor256_prefill": 256, "bf16_razor384_prefill": 384, "bf16_razor256_decode_t1": 256}
+CALIBRATION_T = 32768
 
 
 def parse():
@@ -332,6 +344,24 @@ def expert_roofline(wl, layers, T, rows, ffn_ms, peaks) -> dict:
             "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)", "experts_touched": touched}
 
 
+def razor_pruned_weights(wl, seed: int, keep: int, dev) -> dict:
+    """The layer of seed `seed` pruned to `keep` experts the RAZOR way, all on
+    the device through the C ABI: Refill-RMS statistics over one calibration
+    row of CALIBRATION_T tokens, razor_select, razor_slice of every
+    per-expert tensor with the kept set."""
+    w = synth.make_weights(wl, seed=seed, device=dev)
+    cal = MoELayer(w, wl.k, wl.fmt, T_max=CALIBRATION_T, extra=1)
+    ss = torch.zeros(wl.E, dtype=torch.float64, device=dev)
+    cc = torch.zeros(wl.E, dtype=torch.int64, device=dev)
+    cal.refill_pass(synth.make_tokens(wl, CALIBRATION_T, seed=seed, batch=1000, device=dev), ss, cc)
+    kept, _, _ = abi.razor_select(ss, cc, keep)
+    pruned = slice_layer_weights(w, kept)
+    torch.cuda.synchronize()
+    del cal, w
+    torch.cuda.empty_cache()
+    return pruned
+
+
 def run_native(args, dist: Dist) -> None:
     wname, T, kind = WORKLOADS[args.workload]
     wl = synth.WORKLOADS[wname]
@@ -339,7 +369,17 @@ def run_native(args, dist: Dist) -> None:
     torch.cuda.set_device(dev)
     extra = 1 if kind == "refill" else 0
     decode = T < 256
-    layers = [MoELayer(synth.make_weights(wl, seed=0, device=dev), wl.k, wl.fmt, T_max=T, extra=extra)]
+    keep = PRUNED.get(args.workload, 0)
+    if keep:
+        wl_full = wl
+        wl = dataclasses.replace(wl, E=keep)
+
+        def layer_weights(seed):
+            return razor_pruned_weights(wl_full, seed, keep, dev)
+    else:
+        def layer_weights(seed):
+            return synth.make_weights(wl, seed=seed, device=dev)
+    layers = [MoELayer(layer_weights(0), wl.k, wl.fmt, T_max=T, extra=extra)]
     layer_bytes = sum(t.numel() * t.element_size() for t in layers[0].w.values())
     if decode:
         # A decode step touches fewer expert bytes than L2 holds.  Rotate
@@ -352,7 +392,7 @@ def run_native(args, dist: Dist) -> None:
         n_layers = max(2, 1 + -(-3 * L2_BYTES // int(step_min)))
         n_layers = min(n_layers, 24, max(2, int(64e9 // layer_bytes)))
         for l in range(1, n_layers):
-            layers.append(MoELayer(synth.make_weights(wl, seed=l, device=dev), wl.k, wl.fmt, T_max=T, extra=extra))
+            layers.append(MoELayer(layer_weights(l), wl.k, wl.fmt, T_max=T, extra=extra))
     layer = layers[0]
     w = layer.w
     # token batches: distinct per rank, rotated so that the inputs of the
@@ -510,7 +550,9 @@ def run_native(args, dist: Dist) -> None:
                                        "nvfp4": "fp4 e2m1 x fp4 e2m1 (NVFP4)"}[wl.fmt],
         "data": "synthetic (seeded N(0,1) tokens, N(0,1/sqrt(fan_in)) weights)",
         "config": {"workload": f"{args.workload}: T={T} H={wl.H} E={wl.E} k={wl.k} I={wl.I} shared={wl.I_sh} "
-                               f"fmt={wl.fmt}" + (" +Refill-RMS accumulate/select" if kind == "refill" else ""),
+                               f"fmt={wl.fmt}" + (" +Refill-RMS accumulate/select" if kind == "refill" else "")
+                               + (f" (RAZOR-pruned from {wl_full.E} experts: Refill-RMS over one {CALIBRATION_T}-token "
+                                  f"calibration row, top {keep} kept, sliced on the device)" if keep else ""),
                    "tokens_per_step_per_gpu": T, "parallelism": f"dp{dist.world} (replicas, no collective)",
                    "launch": "eager C-ABI calls" if args.no_graph else "one CUDA graph per step (the C-ABI calls)",
                    "l2": (f"{n_units} layers with distinct weights in rotation ({layer_bytes / 2**30:.2f} GiB each); "

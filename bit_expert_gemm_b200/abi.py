@@ -68,6 +68,9 @@ _SIGS = {
     "moe_combine": (_I, [_P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "razor_refill_rms_accumulate": (_I, [_P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "razor_select": (_I, [_P, _P, _I, _I, _P, _P, _P, _P]),
+    "razor_router_norm": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_shared_gate": (_I, [_P, _I, _I, _P, _I, _P, _P]),
+    "razor_slice": (_I, [_P, _I, _SZ, _P, _I, _P, _P]),
 }
 
 _lib = None
@@ -464,3 +467,45 @@ def razor_select(sum_sq, count, keep: int, kept=None, ranking=None, score=None, 
         score = torch.empty((E,), dtype=torch.float64, device=dev)
     _call("razor_select", _p(sum_sq), _p(count), E, keep, _p(kept), _p(ranking), _p(score), _stream(stream))
     return kept[:keep], ranking, score
+
+
+def moe_shared_gate(x, w_gate, gate=None, stream=None):
+    """gate [T] FP32 = sigmoid(x . w_gate) for x [T, H], w_gate [H]."""
+    T, H = x.shape
+    if w_gate.dtype != x.dtype or tuple(w_gate.shape) != (H,):
+        raise ValueError("moe_shared_gate: w_gate must be [H] of x's dtype")
+    if gate is None:
+        gate = torch.empty((T,), dtype=torch.float32, device=x.device)
+    _need(gate, torch.float32, "gate")
+    _call("moe_shared_gate", _p(x), T, H, _p(w_gate), _dtype_code(x), _p(gate), _stream(stream))
+    return gate
+
+
+def razor_router_norm(w_router, sum_sq=None, count=None, stream=None):
+    """Router-norm keep statistics: sum_sq[e] = ||w_router[e]||^2 (FP64),
+    count[e] = 1, ready for razor_select."""
+    E, H = w_router.shape
+    dev = w_router.device
+    if sum_sq is None:
+        sum_sq = torch.empty((E,), dtype=torch.float64, device=dev)
+    if count is None:
+        count = torch.empty((E,), dtype=torch.int64, device=dev)
+    _need(sum_sq, torch.float64, "sum_sq")
+    _need(count, torch.int64, "count")
+    _call("razor_router_norm", _p(w_router), E, H, _dtype_code(w_router), _p(sum_sq), _p(count), _stream(stream))
+    return sum_sq, count
+
+
+def razor_slice(src, kept, out=None, stream=None):
+    """out[j] = src[kept[j]] along the leading (expert) dimension, byte-exact.
+    src [E, ...] contiguous of any dtype, kept [keep] int32 on the device."""
+    _need(kept, torch.int32, "kept")
+    E = src.shape[0]
+    keep = kept.shape[0]
+    if out is None:
+        out = torch.empty((keep, *src.shape[1:]), dtype=src.dtype, device=src.device)
+    if out.dtype != src.dtype or tuple(out.shape) != (keep, *src.shape[1:]):
+        raise ValueError("razor_slice: out must be [keep, ...] of src's dtype")
+    bpe = src[0].numel() * src.element_size() if E else 0
+    _call("razor_slice", _p(src), E, bpe, _p(kept), keep, _p(out), _stream(stream))
+    return out

@@ -66,6 +66,10 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
 size_t nvfp4_packed_sf_bytes(int E, int rows_per_expert, int K, int swiglu);
 int nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, int K, int swiglu, uint8_t* out,
                      cudaStream_t stream);
+int shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, float* gate, cudaStream_t stream);
+int router_norm(const void* w_router, int E, int H, int dtype, double* sum_sq, int64_t* count, cudaStream_t stream);
+int slice_experts(const void* src, int E, size_t bytes_per_expert, const int32_t* kept, int keep, void* dst,
+                  cudaStream_t stream);
 
 namespace {
 thread_local char g_err[1024] = "";
@@ -607,6 +611,39 @@ int razor_select(const double* sum_sq, const int64_t* count, int E, int keep, in
   MOE_REQUIRE(keep >= 0 && keep <= E, MOE_ERR_INVALID_ARG, "razor_select: keep=%d outside [0, E]", keep);
   MOE_REQUIRE(sum_sq && count && (kept_idx || keep == 0), MOE_ERR_INVALID_ARG, "razor_select: null pointer");
   return select_experts(sum_sq, count, E, keep, kept_idx, ranking, score, static_cast<cudaStream_t>(stream));
+}
+
+int moe_shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, float* gate, void* stream) {
+  MOE_REQUIRE(T >= 0 && H >= 8 && H % 8 == 0, MOE_ERR_UNSUPPORTED, "moe_shared_gate: T=%d H=%d (need H %% 8 == 0)", T,
+              H);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_shared_gate: dtype=%d",
+              dtype);
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(x && w_gate && gate, MOE_ERR_INVALID_ARG, "moe_shared_gate: null pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(w_gate), MOE_ERR_INVALID_ARG,
+              "moe_shared_gate: x and w_gate must be 16-byte aligned");
+  return shared_gate(x, T, H, w_gate, dtype, gate, static_cast<cudaStream_t>(stream));
+}
+
+int razor_router_norm(const void* w_router, int E, int H, int dtype, double* sum_sq, int64_t* count, void* stream) {
+  MOE_REQUIRE(E >= 1 && H >= 1, MOE_ERR_INVALID_ARG, "razor_router_norm: E=%d H=%d must be positive", E, H);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "razor_router_norm: dtype=%d",
+              dtype);
+  MOE_REQUIRE(w_router && sum_sq, MOE_ERR_INVALID_ARG, "razor_router_norm: null pointer");
+  return router_norm(w_router, E, H, dtype, sum_sq, count, static_cast<cudaStream_t>(stream));
+}
+
+int razor_slice(const void* src, int E, size_t bytes_per_expert, const int32_t* kept_idx, int keep, void* dst,
+                void* stream) {
+  MOE_REQUIRE(E >= 1, MOE_ERR_INVALID_ARG, "razor_slice: E=%d must be positive", E);
+  MOE_REQUIRE(keep >= 0 && keep <= E && keep <= 65535, MOE_ERR_INVALID_ARG,
+              "razor_slice: keep=%d outside [0, min(E, 65535)]", keep);
+  if (keep == 0 || bytes_per_expert == 0) return MOE_OK;
+  MOE_REQUIRE(src && dst && kept_idx, MOE_ERR_INVALID_ARG, "razor_slice: null pointer");
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+  const uintptr_t s1 = s0 + uintptr_t(E) * bytes_per_expert, d1 = d0 + uintptr_t(keep) * bytes_per_expert;
+  MOE_REQUIRE(d1 <= s0 || s1 <= d0, MOE_ERR_INVALID_ARG, "razor_slice: dst overlaps src");
+  return slice_experts(src, E, bytes_per_expert, kept_idx, keep, dst, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

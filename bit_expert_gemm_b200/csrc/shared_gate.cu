@@ -1,0 +1,69 @@
+// Shared-expert gate: gate[t] = sigmoid(x[t, :] . w_gate), one FP32 scalar
+// per token, which moe_combine multiplies into the shared expert's output.
+//
+// Qwen3.8-Flash-Next-AWQ-g32 card, "Checkpoint": the shared-expert gate is
+// one of the non-routed tensors stored next to the router and the shared
+// expert.  The card gives no formula; this is the plainest reading (a
+// row vector over the hidden size and a logistic gate per token).
+//
+// One warp per token: 16-byte loads of x and of the gate vector (8 16-bit
+// values each, lane-strided), FP32 products summed per lane, then a shuffle
+// tree; the logistic function uses the accurate expf and an IEEE division.
+// The kernel reads x once: HBM-bound at T*H*2 bytes.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+template <typename T16>
+__device__ __forceinline__ float2 to_f2(uint32_t v);
+template <>
+__device__ __forceinline__ float2 to_f2<__nv_bfloat16>(uint32_t v) {
+  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v));
+}
+template <>
+__device__ __forceinline__ float2 to_f2<__half>(uint32_t v) {
+  return __half22float2(*reinterpret_cast<__half2*>(&v));
+}
+
+template <typename T16>
+__global__ void __launch_bounds__(256) k_shared_gate(const T16* __restrict__ x, const T16* __restrict__ wg, int T,
+                                                     int H, float* __restrict__ gate) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + size_t(t) * H);
+  const uint4* gr = reinterpret_cast<const uint4*>(wg);
+  float acc = 0.f;
+  for (int c = lane; c < H / 8; c += 32) {
+    const uint4 a = __ldg(xr + c), b = __ldg(gr + c);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 p = to_f2<T16>(av[i]), q = to_f2<T16>(bv[i]);
+      acc = fmaf(p.x, q.x, acc);
+      acc = fmaf(p.y, q.y, acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) gate[t] = 1.0f / (1.0f + expf(-acc));
+}
+
+}  // namespace
+
+int shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, float* gate, cudaStream_t stream) {
+  if (T == 0) return MOE_OK;
+  const dim3 grid((T + 7) / 8);
+  if (dtype == MOE_DTYPE_BF16)
+    k_shared_gate<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x),
+                                                           static_cast<const __nv_bfloat16*>(w_gate), T, H, gate);
+  else
+    k_shared_gate<__half><<<grid, 256, 0, stream>>>(static_cast<const __half*>(x), static_cast<const __half*>(w_gate),
+                                                    T, H, gate);
+  MOE_CHECK_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -110,6 +110,8 @@ class MoELayer:
             f_dt = self.adt
         self.f = torch.empty((rows, H), dtype=f_dt, device=d)
         self.shared = torch.empty((T_max, H), dtype=self.adt, device=d)
+        # optional shared-expert gate (weights key "w_sh_gate", [H]): sigmoid(x . w) per token
+        self.sh_gate = torch.empty((T_max,), dtype=torch.float32, device=d) if "w_sh_gate" in self.w else None
         self.y = torch.empty((T_max, H), dtype=self.adt, device=d)
         op = {"bf16": abi.MOE_OP_SWIGLU_BF16, "awq_g32": abi.MOE_OP_SWIGLU_AWQ_G32,
               "nvfp4": abi.MOE_OP_SWIGLU_NVFP4}[self.fmt]
@@ -200,10 +202,17 @@ class MoELayer:
         T = x.shape[0]
         assert T <= self.T_max and self.extra == 0
         self.route(x)
+        gate = self.shared_gate(x)
         f, sh = self.experts_and_shared(x)
         y = self.y[:T] if y is None else y
-        abi.moe_combine(f, self.slot_row[:T], self.topk_w[:T], shared_out=sh, y=y)
+        abi.moe_combine(f, self.slot_row[:T], self.topk_w[:T], shared_out=sh, shared_gate=gate, y=y)
         return y
+
+    def shared_gate(self, x: torch.Tensor) -> Optional[torch.Tensor]:
+        """Per-token shared-expert gate (moe_shared_gate), or None without one."""
+        if self.sh_gate is None:
+            return None
+        return abi.moe_shared_gate(x, self.w["w_sh_gate"], gate=self.sh_gate[:x.shape[0]])
 
     def capture(self, x: torch.Tensor, fn=None, warmup: int = 1) -> "torch.cuda.CUDAGraph":
         """CUDA graph of fn(x) (default: forward).  Every launch of the pass
@@ -238,11 +247,59 @@ class MoELayer:
         T = x.shape[0]
         assert self.extra == 1
         self.route(x)
+        gate = self.shared_gate(x)
         f, sh = self.experts_and_shared(x)
         y = self.y[:T]
+        # the shared expert cancels in the score; with a gate, y is combined separately
         abi.razor_refill_rms_accumulate(f, self.slot_row[:T], self.topk_idx[:T], self.topk_logit[:T], self.offsets,
-                                        sum_sq, count, shared_out=sh, y_out=y, ws=self.ws_refill)
+                                        sum_sq, count, shared_out=None if gate is not None else sh,
+                                        y_out=None if gate is not None else y, ws=self.ws_refill)
+        if gate is not None:
+            abi.moe_combine(f, self.slot_row[:T], self.topk_w[:T], shared_out=sh, shared_gate=gate, y=y)
         return y
+
+
+# Tensors of a layer whose leading axis (or, for the flat tile-packed copies,
+# whose equal per-expert blocks) belong to one routed expert each.
+EXPERT_TENSORS = ("w_router", "bias", "w_gate_up", "w_down", "qw_gu", "qz_gu", "sc_gu", "qw_d", "qz_d", "sc_d",
+                  "w_gu", "sf_gu", "gs_gu", "w_d", "sf_d", "gs_d")
+EXPERT_PACKED = ("awq_packed", "sfp_gu", "sfp_d")
+
+
+def slice_layer_weights(w: Dict[str, torch.Tensor], kept: torch.Tensor) -> Dict[str, torch.Tensor]:
+    """The pruned layer: every per-expert tensor, router rows and bias
+    included, gathered with one kept list (razor_slice, in matching order);
+    the shared expert and any activation scales are unchanged.  kept [keep]
+    int32 on the device, normally razor_select's ascending kept set."""
+    E = w["w_router"].shape[0]
+    out = {}
+    for n, t in w.items():
+        if n in EXPERT_TENSORS:
+            out[n] = abi.razor_slice(t.contiguous(), kept)
+        elif n in EXPERT_PACKED:
+            out[n] = abi.razor_slice(t.reshape(E, -1), kept).reshape(-1)
+        else:
+            out[n] = t
+    return out
+
+
+def keep_manifest(kept, E: int, policy: str = "refill_rms", scores=None) -> dict:
+    """Keep manifest of one pruned layer: the original expert indices in
+    output order (expert j of the pruned layer is original expert
+    kept_expert_indices[j]), the budget, and how they were chosen
+    ("refill_rms": RMS-aggregated Refill scores; "router_norm": router-row
+    L2 norm).  Host-side bookkeeping; kept may be a tensor or a sequence."""
+    ids = [int(e) for e in (kept.tolist() if hasattr(kept, "tolist") else kept)]
+    if sorted(set(ids)) != ids or (ids and not 0 <= ids[0] <= ids[-1] < E):
+        raise ValueError("kept indices must be distinct, ascending and in [0, E)")
+    m = {"method": "razor", "policy": policy, "experts_before": E, "experts_kept": len(ids),
+         "kept_expert_indices": ids}
+    if policy == "refill_rms":
+        m["aggregation"] = "rms"
+    if scores is not None:
+        sc = scores.tolist() if hasattr(scores, "tolist") else list(scores)
+        m["kept_scores"] = [float(sc[e]) for e in ids]
+    return m
 
 
 def refill_allreduce(sum_sq: torch.Tensor, count: torch.Tensor, group=None) -> None:

@@ -387,6 +387,16 @@ MOE_API int moe_combine(const void* f, int f_fp32, const int32_t* slot_row, int 
                 void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Shared-expert gate [AWQ] ("Checkpoint": a shared-expert gate tensor is
+ * stored with the router and the shared expert; the card gives no formula,
+ * so this is the plainest reading):
+ *   gate[t] = 1 / (1 + exp(-sum_h x[t, h] * w_gate[h]))     (FP32 accumulate)
+ * to be passed as moe_combine's shared_gate.  x [T, H] and w_gate [H] dtype,
+ * both 16-byte aligned; gate [T] FP32.  Limits: H % 8 == 0.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, float* gate, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Refill-RMS accumulation, fused with the combine of a (k+1)-slot pass
  * [RAZOR].  For token t with selected set S (slots 0..k-1) and promoted
  * expert r (slot k), with p_j = exp(l_j - l_0) from topk_logit:
@@ -419,6 +429,43 @@ MOE_API int razor_refill_rms_accumulate(const void* f, int f_fp32, const int32_t
  * ------------------------------------------------------------------------- */
 MOE_API int razor_select(const double* sum_sq, const int64_t* count, int E, int keep, int32_t* kept_idx, int32_t* ranking,
                  double* score, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Router-norm keep policy [RAZOR] ("Selection and calibration", MTP item: the
+ * MTP layer's experts are kept by the L2 norm of their original router rows,
+ * mtp_policy=router_norm).  Writes sum_sq[e] = sum_h w_router[e, h]^2 (the
+ * 16-bit weights squared exactly in FP64 and summed in a fixed order) and,
+ * when count is not NULL, count[e] = 1: statistics in the form Refill-RMS
+ * produces, so razor_select with the same keep ranks the experts by
+ * sqrt(sum_sq / count) = ||w_router[e, :]||_2, ties to the lower index.
+ * Both outputs are overwritten, not accumulated.
+ * w_router [E, H] dtype; sum_sq [E] FP64; count [E] int64 or NULL.
+ * ------------------------------------------------------------------------- */
+MOE_API int razor_router_norm(const void* w_router, int E, int H, int dtype, double* sum_sq, int64_t* count,
+                              void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Slice of the kept experts [RAZOR] (opening paragraphs: the surviving
+ * expert weights and router rows are slices of the base checkpoint, in
+ * matching order; the keep manifest lists original indices in output order).
+ *
+ *   dst[j] = src[kept_idx[j]]     for j < keep, whole blocks of
+ *                                 bytes_per_expert bytes
+ *
+ * src holds E per-expert blocks back to back ([E, ...] with the expert index
+ * leading: router rows, a router bias, every expert weight, scale and zero
+ * tensor of any format, the tile-ordered copies of moe_awq_prepack_g32 and
+ * moe_nvfp4_prepack_sf); dst receives keep blocks.  Passing the same
+ * kept_idx (razor_select's ascending kept set) to every tensor of a layer
+ * slices them in matching order.  The copy is byte-exact; 16-byte vectors
+ * are used when both pointers and bytes_per_expert are multiples of 16.
+ * kept_idx [keep] int32 device array, any order; an index outside [0, E) is
+ * skipped (its dst block is left untouched) and recorded as
+ * MOE_ERR_INVALID_ARG in the device status word.  dst must not overlap src.
+ * Limits: 0 <= keep <= min(E, 65535).
+ * ------------------------------------------------------------------------- */
+MOE_API int razor_slice(const void* src, int E, size_t bytes_per_expert, const int32_t* kept_idx, int keep, void* dst,
+                        void* stream);
 
 #ifdef __cplusplus
 }

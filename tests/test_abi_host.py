@@ -112,3 +112,33 @@ def test_awq_prepack_sizes_and_checks():
         abi.MOE_ERR_WORKSPACE
     assert _code("moe_experts_awq_g32_prepacked", buf, buf, buf, 1, 10, 2048, 640, 16, buf, buf, buf, buf, buf, buf,
                  None, buf, buf, 0, buf, buf, buf, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG  # awq_packed is null
+
+
+def test_razor_slice_and_router_norm_reject_bad_arguments():
+    p = ctypes.c_void_p
+    # keep above E, negative keep, E <= 0
+    assert _code("razor_slice", p(256), 4, 16, p(512), 5, p(1 << 20), None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("razor_slice", p(256), 4, 16, p(512), -1, p(1 << 20), None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("razor_slice", p(256), 0, 16, p(512), 0, p(1 << 20), None) == abi.MOE_ERR_INVALID_ARG
+    # null pointers, and a dst that overlaps src (E * 4096 bytes from 4096)
+    assert _code("razor_slice", None, 4, 16, p(512), 2, p(1 << 20), None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("razor_slice", p(4096), 4, 4096, None, 2, p(1 << 20), None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("razor_slice", p(4096), 4, 4096, p(512), 2, p(8192), None) == abi.MOE_ERR_INVALID_ARG
+    assert "overlaps" in abi.load().moe_last_error().decode()
+    # nothing to copy: accepted without touching memory
+    assert _code("razor_slice", None, 4, 16, None, 0, None, None) == abi.MOE_OK
+    assert _code("razor_router_norm", None, 16, 256, 0, p(256), None, None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("razor_router_norm", p(256), 16, 256, 7, p(256), None, None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("razor_router_norm", p(256), 0, 256, 0, p(256), None, None) == abi.MOE_ERR_INVALID_ARG
+
+
+def test_keep_manifest():
+    from bit_expert_gemm_b200.layer import keep_manifest
+
+    m = keep_manifest([1, 4, 7], 8, scores=[0.0, 2.0, 0.5, 0.1, 3.0, 0.0, 0.0, 1.0])
+    assert m["kept_expert_indices"] == [1, 4, 7] and m["experts_kept"] == 3 and m["experts_before"] == 8
+    assert m["aggregation"] == "rms" and m["kept_scores"] == [2.0, 3.0, 1.0]
+    assert keep_manifest([0, 2], 4, policy="router_norm")["policy"] == "router_norm"
+    for bad in ([2, 1], [1, 1], [0, 8]):
+        with pytest.raises(ValueError):
+            keep_manifest(bad, 8)

@@ -254,3 +254,43 @@ def test_route_permute_empty_batch():
     abi.moe_route_permute(x, w["w_router"], w["bias"], 2, expert_offsets=off)
     torch.cuda.synchronize()
     assert off.cpu().tolist() == [0] * 17
+
+
+@pytest.mark.parametrize("T,H,act", [(1, 2048, "bf16"), (64, 256, "bf16"), (777, 2048, "f16"), (8192, 2048, "bf16"),
+                                     (5, 72, "bf16")])
+def test_shared_gate(T, H, act):
+    wl = _wl(H=H, act=act)
+    x = synth.make_tokens(wl, T, seed=T)
+    g = synth.make_shared_gate(wl, seed=T)
+    got = abi.moe_shared_gate(x.to(DEV), g.to(DEV))
+    want = moe.shared_gate(f64(x), f64(g))
+    torch.cuda.synchronize()
+    # FP32 dot products of H terms; the gate's slope is at most 1/4
+    assert np.max(np.abs(got.cpu().double().numpy() - want)) < 1e-5
+    assert abi.moe_device_status() == 0
+
+
+def test_layer_with_shared_gate_forward_and_refill():
+    from bit_expert_gemm_b200 import MoELayer
+    from tests.helpers import expert_fn_bf16, refill_stats_ref, shared_fn
+
+    wl = synth.WORKLOADS["tiny"]
+    w = synth.make_weights(wl, seed=6, device=DEV)
+    w["w_sh_gate"] = synth.make_shared_gate(wl, seed=6, device=DEV)
+    x = synth.make_tokens(wl, wl.T_prefill, seed=6, device=DEV)
+    ref = moe.moe_layer(f64(x), f64(w["w_router"]), f64(w["bias"]), wl.k, expert_fn_bf16(w, wl.I), shared_fn(w),
+                        shared_gate_w=f64(w["w_sh_gate"]))
+    ok = ref["route"]["margin"] > 1e-3
+    y = MoELayer(w, wl.k, "bf16", T_max=wl.T_prefill).forward(x)
+    assert rel_err(f64(y)[ok], ref["y"][ok]) < TOL_BF16
+    rl = MoELayer(w, wl.k, "bf16", T_max=wl.T_prefill, extra=1)
+    ss = torch.zeros(wl.E, dtype=torch.float64, device=DEV)
+    cc = torch.zeros(wl.E, dtype=torch.int64, device=DEV)
+    y2 = rl.refill_pass(x, ss, cc)
+    assert rel_err(f64(y2)[ok], ref["y"][ok]) < TOL_BF16
+    ref1 = moe.moe_layer(f64(x), f64(w["w_router"]), f64(w["bias"]), wl.k, expert_fn_bf16(w, wl.I), shared_fn(w),
+                         extra=1)
+    s_ref, c_ref, good = refill_stats_ref(ref1, wl.k, wl.E)  # the gate does not change the scores
+    assert np.array_equal(cc.cpu().numpy()[good], c_ref[good])
+    assert rel_err(ss.cpu().numpy()[good], s_ref[good]) < TOL_BF16
+    assert abi.moe_device_status() == 0
