@@ -40,6 +40,30 @@ def test_awq_dequant_zero_at_zero_point_and_vs_torch_half():
     assert np.array_equal(W, prod.to(torch.float16).double().numpy())
 
 
+def test_awq_dequant_bf16_mode_vs_torch_bfloat16():
+    """BF16 mode: the scale rounded to BF16 once, then one BF16 product --
+    torch's own bfloat16 conversion and multiplication on the CPU give the
+    same bits; q = z gives 0; a unit code difference gives the rounded scale,
+    whose change is within the card's 0.4 % per scale."""
+    rng = np.random.default_rng(3)
+    q, z, s = _awq_case(rng, K=96, N=40)
+    W = awq.dequant(awq.pack_nibbles(q), awq.pack_nibbles(z), s, mode="bf16")
+    g = np.arange(q.shape[0]) // 32
+    s_bf = torch.from_numpy(s[g].astype(np.float32)).to(torch.bfloat16)
+    d_bf = torch.from_numpy((q - z[g]).astype(np.float32)).to(torch.bfloat16)  # |q - z| <= 15: exact
+    assert np.array_equal(W, (d_bf * s_bf).double().numpy())
+    assert np.all(awq.dequant(awq.pack_nibbles(z[g]), awq.pack_nibbles(z), s, mode="bf16") == 0)
+    one = np.minimum(z[g] + 1, 15)
+    unit = awq.dequant(awq.pack_nibbles(one), awq.pack_nibbles(z), s, mode="bf16")
+    m = one - z[g] == 1
+    s64 = s[g].astype(np.float64)
+    assert np.array_equal(unit[m], s_bf.double().numpy()[m])
+    nz = m & (s64 > 0)
+    assert np.max(np.abs(unit[nz] - s64[nz]) / s64[nz]) <= 0.004
+    # the two modes differ (BF16 keeps 8 significant bits, FP16 11)
+    assert not np.array_equal(W, awq.dequant(awq.pack_nibbles(q), awq.pack_nibbles(z), s))
+
+
 def test_awq_quantize_inverts_dequant_and_error_bound():
     rng = np.random.default_rng(2)
     q, z, s = _awq_case(rng, K=128, N=64, lo_scale=2.0 ** -10)
