@@ -58,6 +58,9 @@ WORKLOADS = {
     "awq_decode_t1": ("awq_g32", 1, "forward"),
     "awq_decode_t8": ("awq_g32", 8, "forward"),
     "awq_decode_t32": ("awq_g32", 32, "forward"),
+    # the AWQ card's BF16 mode (BF16 activations, scales rounded to BF16)
+    "awq_bf16_prefill": ("awq_g32_bf16", 8192, "forward"),
+    "awq_bf16_decode_t1": ("awq_g32_bf16", 1, "forward"),
     "nvfp4_prefill": ("nvfp4", 16384, "forward"),
     "nvfp4_decode_t1": ("nvfp4", 1, "forward"),
     "nvfp4_decode_t64": ("nvfp4", 64, "forward"),
@@ -224,7 +227,8 @@ def oracle_tokens_per_s(wl, w, x: torch.Tensor, n_tokens: int, kind: str):
         if e not in cache:
             if wl.fmt == "awq_g32":
                 cache[e] = awq.expert_weights_out_in(host["qw_gu"], host["qz_gu"], host["sc_gu"], host["qw_d"],
-                                                     host["qz_d"], host["sc_d"], e, I)
+                                                     host["qz_d"], host["sc_d"], e, I,
+                                                     mode="bf16" if wl.act == "bf16" else "fp16")
             else:
                 g = to64(w["w_gate_up"][e])
                 ws = (g[:I], g[I:], to64(w["w_down"][e]))
@@ -546,7 +550,8 @@ def run_native(args, dist: Dist) -> None:
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": {"bf16": "bf16", "awq_g32": "f16 x int4 (AWQ g32)",
+        "vs_baseline": None, "dtype": {"bf16": "bf16", "awq_g32": f"{'bf16' if wl.act == 'bf16' else 'f16'} x int4 "
+                                                                 "(AWQ g32)",
                                        "nvfp4": "fp4 e2m1 x fp4 e2m1 (NVFP4)"}[wl.fmt],
         "data": "synthetic (seeded N(0,1) tokens, N(0,1/sqrt(fan_in)) weights)",
         "config": {"workload": f"{args.workload}: T={T} H={wl.H} E={wl.E} k={wl.k} I={wl.I} shared={wl.I_sh} "

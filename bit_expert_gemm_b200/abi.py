@@ -50,14 +50,15 @@ _SIGS = {
     "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_grouped_swiglu_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _SZ, _P]),
     "moe_experts_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
-    "moe_experts_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P,
-                                 _SZ, _P]),
-    "moe_experts_awq_g32_prepacked": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P,
-                                           _P, _P, _SZ, _P]),
+    "moe_experts_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P,
+                                 _P, _SZ, _P]),
+    "moe_experts_awq_g32_prepacked": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I,
+                                           _P, _P, _P, _SZ, _P]),
     "moe_awq_packed_bytes": (_SZ, [_I, _I, _I]),
     "moe_awq_prepack_g32": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
-    "moe_grouped_swiglu_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
-    "moe_awq_dequant_g32": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
+    "moe_grouped_swiglu_awq_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ,
+                                        _P]),
+    "moe_awq_dequant_g32": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "moe_nvfp4_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_grouped_swiglu_nvfp4": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ,
                                       _P]),
@@ -269,20 +270,21 @@ def moe_experts_bf16(x, row_token, expert_offsets, rows: int, w_gate_up, w_down,
 
 def moe_experts_awq_g32(x, row_token, expert_offsets, rows: int, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d, w_sh_gate_up,
                         w_sh_down, out_fp32: bool = False, f=None, shared_out=None, ws=None, stream=None):
-    """Routed AWQ experts (f [rows, H]) and the FP16 shared expert (shared_out [T, H]) in one call."""
+    """Routed AWQ experts (f [rows, H]) and the 16-bit shared expert (shared_out [T, H]) in one call; x FP16,
+    or BF16 for the BF16 mode (scales rounded to BF16, BF16 weights; the shared expert in x's dtype)."""
     T, H = x.shape
     E = qw_gu.shape[0]
     I = qw_gu.shape[2] * 8 // 2
     dev = x.device
-    _need(x, torch.float16, "x")
+    dcode = _dtype_code(x)
     if f is None:
-        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else torch.float16, device=dev)
+        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else x.dtype, device=dev)
     if shared_out is None:
-        shared_out = torch.empty((T, H), dtype=torch.float16, device=dev)
+        shared_out = torch.empty((T, H), dtype=x.dtype, device=dev)
     if ws is None:
         ws = workspace(MOE_OP_EXPERTS_AWQ_G32, T, H, E, max(1, rows // max(T, 1)), I, dev)
     _call("moe_experts_awq_g32", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E, _p(qw_gu), _p(qz_gu),
-          _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), _p(w_sh_gate_up), _p(w_sh_down), int(out_fp32), _p(f),
+          _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), _p(w_sh_gate_up), _p(w_sh_down), dcode, int(out_fp32), _p(f),
           _p(shared_out), _p(ws), ws.numel(), _stream(stream))
     return f, shared_out
 
@@ -309,16 +311,16 @@ def moe_experts_awq_g32_prepacked(x, row_token, expert_offsets, rows: int, qw_gu
     E = qw_gu.shape[0]
     I = qw_gu.shape[2] * 8 // 2
     dev = x.device
-    _need(x, torch.float16, "x")
+    dcode = _dtype_code(x)
     if f is None:
-        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else torch.float16, device=dev)
+        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else x.dtype, device=dev)
     if shared_out is None:
-        shared_out = torch.empty((T, H), dtype=torch.float16, device=dev)
+        shared_out = torch.empty((T, H), dtype=x.dtype, device=dev)
     if ws is None:
         ws = workspace(MOE_OP_EXPERTS_AWQ_G32, T, H, E, max(1, rows // max(T, 1)), I, dev)
     _call("moe_experts_awq_g32_prepacked", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E, _p(qw_gu),
           _p(qz_gu), _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), _p(awq_packed), _p(w_sh_gate_up), _p(w_sh_down),
-          int(out_fp32), _p(f), _p(shared_out), _p(ws), ws.numel(), _stream(stream))
+          dcode, int(out_fp32), _p(f), _p(shared_out), _p(ws), ws.numel(), _stream(stream))
     return f, shared_out
 
 
@@ -328,20 +330,20 @@ def moe_grouped_swiglu_awq_g32(x, row_token, expert_offsets, rows: int, qw_gu, q
     E = qw_gu.shape[0]
     I = qw_gu.shape[2] * 8 // 2
     dev = x.device
-    _need(x, torch.float16, "x")
+    dcode = _dtype_code(x)  # FP16, or BF16 for the BF16 mode
     if f is None:
-        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else torch.float16, device=dev)
+        f = torch.empty((rows, H), dtype=torch.float32 if out_fp32 else x.dtype, device=dev)
     if ws is None:
         ws = workspace(MOE_OP_SWIGLU_AWQ_G32, rows, H, E, 1, I, dev)
     _call("moe_grouped_swiglu_awq_g32", _p(x), _p(row_token), _p(expert_offsets), T, rows, H, I, E, _p(qw_gu),
-          _p(qz_gu), _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), int(out_fp32), _p(f), _p(ws), ws.numel(),
+          _p(qz_gu), _p(sc_gu), _p(qw_d), _p(qz_d), _p(sc_d), dcode, int(out_fp32), _p(f), _p(ws), ws.numel(),
           _stream(stream))
     return f
 
 
-def moe_awq_dequant_g32(qweight, qzeros, scales, out=None, stream=None):
-    """qweight [B, K, N/8] (or [K, N/8]) -> FP16 [B, K, N]: the exact weights
-    the AWQ GEMM multiplies with."""
+def moe_awq_dequant_g32(qweight, qzeros, scales, out=None, dtype=torch.float16, stream=None):
+    """qweight [B, K, N/8] (or [K, N/8]) -> [B, K, N] of dtype (FP16, or BF16
+    for the BF16 mode): the exact weights the AWQ GEMM multiplies with."""
     squeeze = qweight.dim() == 2
     qw = qweight.unsqueeze(0) if squeeze else qweight
     qz = qzeros.unsqueeze(0) if squeeze else qzeros
@@ -352,8 +354,8 @@ def moe_awq_dequant_g32(qweight, qzeros, scales, out=None, stream=None):
     _need(qz, torch.int32, "qzeros")
     _need(sc, torch.float16, "scales")
     if out is None:
-        out = torch.empty((B, K, N), dtype=torch.float16, device=qw.device)
-    _call("moe_awq_dequant_g32", _p(qw), _p(qz), _p(sc), B, K, N, _p(out), _stream(stream))
+        out = torch.empty((B, K, N), dtype=dtype, device=qw.device)
+    _call("moe_awq_dequant_g32", _p(qw), _p(qz), _p(sc), B, K, N, _dtype_code(out), _p(out), _stream(stream))
     return out[0] if squeeze else out
 
 

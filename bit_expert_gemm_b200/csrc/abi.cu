@@ -34,18 +34,18 @@ int select_experts(const double* sum_sq, const int64_t* count, int E, int keep, 
 size_t awq_ws_bytes(int rows, int H, int I, int E);
 int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
                        int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
-                       const int32_t* qz_d, const void* sc_d, int out_fp32, void* f, void* ws, size_t ws_bytes,
-                       cudaStream_t stream);
-int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N, void* out,
-                cudaStream_t stream);
+                       const int32_t* qz_d, const void* sc_d, int dtype, int out_fp32, void* f, void* ws,
+                       size_t ws_bytes, cudaStream_t stream);
+int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N, int dtype,
+                void* out, cudaStream_t stream);
 size_t nvfp4_quant_ws_bytes(int batch, int rows, int K);
 size_t decode_ws_bytes(int rows, int T, int I);
 size_t decode_fused_ws_bytes(int rows, int T, int H, int I);
 int decode_experts_fused_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
                              int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
                              const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gu,
-                             const void* w_sh_d, int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
-                             cudaStream_t stream, const void* qpack);
+                             const void* w_sh_d, int dtype, int f_fp32, void* f, void* shared_out, void* ws,
+                             size_t ws_bytes, cudaStream_t stream, const void* qpack);
 size_t awq_packed_bytes(int E, int H, int I);
 int awq_prepack(const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
                 const int32_t* qz_d, const void* sc_d, int E, int H, int I, void* out, cudaStream_t stream);
@@ -263,7 +263,7 @@ using namespace moe;
 
 extern "C" {
 
-int moe_abi_version(void) { return 1; }
+int moe_abi_version(void) { return 2; }
 
 const char* moe_last_error(void) { return g_err; }
 
@@ -409,10 +409,12 @@ int moe_experts_bf16(const void* x, const int32_t* row_token, const int32_t* exp
 static int experts_awq_impl(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows,
                             int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
                             const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* awq_packed,
-                            const void* w_sh_gate_up, const void* w_sh_down, int out_fp32, void* f, void* shared_out,
-                            void* ws, size_t ws_bytes, void* stream) {
+                            const void* w_sh_gate_up, const void* w_sh_down, int dtype, int out_fp32, void* f,
+                            void* shared_out, void* ws, size_t ws_bytes, void* stream) {
   MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG,
               "moe_experts_awq_g32: bad sizes");
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_experts_awq_g32: dtype=%d",
+              dtype);
   MOE_REQUIRE(H > 0 && I > 0 && H % 128 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
               "moe_experts_awq_g32: need H %% 128 == 0 and I %% 64 == 0 (H=%d I=%d)", H, I);
   if (T == 0) return MOE_OK;
@@ -429,36 +431,36 @@ static int experts_awq_impl(const void* x, const int32_t* row_token, const int32
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (T <= kFusedMaxT && fused_decode_enabled())
     return decode_experts_fused_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d,
-                                    sc_d, w_sh_gate_up, w_sh_down, out_fp32, f, shared_out, ws, ws_bytes, st,
+                                    sc_d, w_sh_gate_up, w_sh_down, dtype, out_fp32, f, shared_out, ws, ws_bytes, st,
                                     awq_packed);
   int rc = MOE_OK;
   if (rows > 0) {
     rc = grouped_swiglu_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
-                            out_fp32, f, ws, ws_bytes, st);
+                            dtype, out_fp32, f, ws, ws_bytes, st);
     if (rc) return rc;
   }
-  return dense_swiglu(x, T, H, I, w_sh_gate_up, w_sh_down, MOE_DTYPE_F16, shared_out, static_cast<uint16_t*>(ws), st);
+  return dense_swiglu(x, T, H, I, w_sh_gate_up, w_sh_down, dtype, shared_out, static_cast<uint16_t*>(ws), st);
 }
 
 int moe_experts_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows, int H,
                         int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
                         const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gate_up,
-                        const void* w_sh_down, int out_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
-                        void* stream) {
+                        const void* w_sh_down, int dtype, int out_fp32, void* f, void* shared_out, void* ws,
+                        size_t ws_bytes, void* stream) {
   return experts_awq_impl(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
-                          nullptr, w_sh_gate_up, w_sh_down, out_fp32, f, shared_out, ws, ws_bytes, stream);
+                          nullptr, w_sh_gate_up, w_sh_down, dtype, out_fp32, f, shared_out, ws, ws_bytes, stream);
 }
 
 int moe_experts_awq_g32_prepacked(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
                                   int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
                                   const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
-                                  const void* awq_packed, const void* w_sh_gate_up, const void* w_sh_down,
+                                  const void* awq_packed, const void* w_sh_gate_up, const void* w_sh_down, int dtype,
                                   int out_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes, void* stream) {
   MOE_REQUIRE(awq_packed != nullptr || T == 0, MOE_ERR_INVALID_ARG, "moe_experts_awq_g32_prepacked: null awq_packed");
   MOE_REQUIRE(aligned16(awq_packed), MOE_ERR_INVALID_ARG,
               "moe_experts_awq_g32_prepacked: awq_packed must be 16-byte aligned");
   return experts_awq_impl(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
-                          awq_packed, w_sh_gate_up, w_sh_down, out_fp32, f, shared_out, ws, ws_bytes, stream);
+                          awq_packed, w_sh_gate_up, w_sh_down, dtype, out_fp32, f, shared_out, ws, ws_bytes, stream);
 }
 
 size_t moe_awq_packed_bytes(int E, int H, int I) {
@@ -484,9 +486,11 @@ int moe_awq_prepack_g32(const int32_t* qw_gu, const int32_t* qz_gu, const void* 
 int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
                                int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
                                const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
-                               int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream) {
+                               int dtype, int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream) {
   MOE_REQUIRE(T >= 0 && rows >= 0 && E >= 1 && E <= kGemmMaxGroups, MOE_ERR_INVALID_ARG,
               "moe_grouped_swiglu_awq_g32: bad sizes");
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG,
+              "moe_grouped_swiglu_awq_g32: dtype=%d", dtype);
   MOE_REQUIRE(H > 0 && I > 0 && H % 64 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
               "moe_grouped_swiglu_awq_g32: H=%d and I=%d must be positive multiples of 64", H, I);
   MOE_REQUIRE(row_token || rows == T, MOE_ERR_INVALID_ARG, "moe_grouped_swiglu_awq_g32: without row_token rows must equal T");
@@ -494,18 +498,20 @@ int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const in
   MOE_REQUIRE(x && expert_offsets && qw_gu && qz_gu && sc_gu && qw_d && qz_d && sc_d && f, MOE_ERR_INVALID_ARG,
               "moe_grouped_swiglu_awq_g32: null pointer");
   return grouped_swiglu_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
-                            out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+                            dtype, out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int moe_awq_dequant_g32(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N,
-                        void* out, void* stream) {
+                        int dtype, void* out, void* stream) {
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_awq_dequant_g32: dtype=%d",
+              dtype);
   MOE_REQUIRE(batch >= 0 && K >= 0 && N >= 0 && K % 32 == 0 && N % 8 == 0, MOE_ERR_UNSUPPORTED,
               "moe_awq_dequant_g32: need K %% 32 == 0 and N %% 8 == 0 (K=%d N=%d)", K, N);
   if (long(batch) * K * N == 0) return MOE_OK;
   MOE_REQUIRE(qweight && qzeros && scales && out, MOE_ERR_INVALID_ARG, "moe_awq_dequant_g32: null pointer");
   MOE_REQUIRE(aligned16(scales) && aligned16(out), MOE_ERR_INVALID_ARG,
               "moe_awq_dequant_g32: scales / out must be 16-byte aligned");
-  return awq_dequant(qweight, qzeros, scales, batch, K, N, out, static_cast<cudaStream_t>(stream));
+  return awq_dequant(qweight, qzeros, scales, batch, K, N, dtype, out, static_cast<cudaStream_t>(stream));
 }
 
 int moe_nvfp4_quantize(const void* v, int batch, int rows, int K, int dtype, const float* global_scale_in,

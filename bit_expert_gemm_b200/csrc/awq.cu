@@ -1,6 +1,8 @@
 // AWQ W4A16 asymmetric group-32 experts: grouped SwiGLU on the tcgen05 GEMM
 // with in-kernel dequantisation, and a standalone dequantisation kernel that
-// uses the same device function (exposes the GEMM's FP16 weights for tests).
+// uses the same device function (exposes the GEMM's 16-bit weights for
+// tests).  dtype selects FP16 (the checkpoint's runtime) or the BF16 mode
+// (FP16 scales rounded to BF16, BF16 weights and activations).
 #include "common.cuh"
 #include "gemm_sm100.cuh"
 
@@ -18,8 +20,8 @@ size_t awq_ws_bytes(int rows, int H, int I, int E) {
 
 int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
                        int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
-                       const int32_t* qz_d, const void* sc_d, int out_fp32, void* f, void* ws, size_t ws_bytes,
-                       cudaStream_t stream) {
+                       const int32_t* qz_d, const void* sc_d, int dtype, int out_fp32, void* f, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
   (void)T;
   WsCarver carve(ws, ws_bytes);
   void* xp = row_token ? carve.take<uint16_t>(size_t(rows) * H) : nullptr;
@@ -45,7 +47,7 @@ int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* o
   g1.ldo = I;
   g1.out_fp32 = 0;
   g1.bias = nullptr;
-  g1.bf16 = 0;
+  g1.bf16 = dtype == MOE_DTYPE_BF16;
   g1.status = device_status_ptr();
   g1.limit_ns = wait_limit_ns();
   int rc = launch_grouped_gemm_awq(a, rows, qw_gu, qz_gu, sc_gu, 2 * I, g1, EPI_SWIGLU, pick_bn(rows, E, I, true),
@@ -62,6 +64,7 @@ int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* o
 }
 
 // out[b, k, 8w .. 8w+7] = dequantised word (b, k, w); one thread per word.
+template <bool BF>
 __global__ void __launch_bounds__(256) k_awq_dequant(const uint32_t* __restrict__ qw, const uint32_t* __restrict__ qz,
                                                      const uint4* __restrict__ sc, int K, int W, long total,
                                                      uint4* __restrict__ out) {
@@ -72,14 +75,15 @@ __global__ void __launch_bounds__(256) k_awq_dequant(const uint32_t* __restrict_
   const long b = bk / K;
   const int k = int(bk - b * K);
   const long grow = b * (K / 32) + k / 32;
-  out[i] = awq_dequant8(qw[i], qz[grow * W + w], sc[grow * W + w]);
+  out[i] = awq_dequant8<BF>(qw[i], qz[grow * W + w], sc[grow * W + w]);
 }
 
-int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N, void* out,
-                cudaStream_t stream) {
+int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N, int dtype,
+                void* out, cudaStream_t stream) {
   const long total = long(batch) * K * (N / 8);
   if (total == 0) return MOE_OK;
-  k_awq_dequant<<<int((total + 255) / 256), 256, 0, stream>>>(
+  auto kern = dtype == MOE_DTYPE_BF16 ? k_awq_dequant<true> : k_awq_dequant<false>;
+  kern<<<int((total + 255) / 256), 256, 0, stream>>>(
       reinterpret_cast<const uint32_t*>(qweight), reinterpret_cast<const uint32_t*>(qzeros),
       static_cast<const uint4*>(scales), K, N / 8, total, static_cast<uint4*>(out));
   MOE_CHECK_CUDA(cudaGetLastError());

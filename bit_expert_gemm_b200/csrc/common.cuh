@@ -374,42 +374,71 @@ struct Pack2<__half> {
 
 // AWQ dequantisation of one packed word: codes q_j (nibble j of W, output
 // column 8w+j), zero points z_j (nibble j of Z) and FP16 scales s_j (S holds
-// s_0..s_7) -> the 8 FP16 values fp16_rn((q_j - z_j) * s_j), as 4 packed
-// pairs (j = 2m low half, 2m+1 high half).  0x6400 | q is the FP16 value
-// 1024 + q, so one subtraction of two such values gives q - z exactly; the
-// single FP16 multiplication then rounds once, to nearest even.
+// s_0..s_7) -> 8 16-bit weights, as 4 packed pairs (j = 2m low half, 2m+1
+// high half).
 //
-// (W >> 4m) & 0x000F000F | 0x64006400 yields the pair (1024 + q_m,
-// 1024 + q_{m+4}) in one logic operation, so the arithmetic runs on the pairs
-// (m, m+4) and four byte permutations restore the column order.  The zero
-// points and scales of a group (AwqGroup) are prepared once for its 32 rows.
+// FP16 (BF = false): fp16_rn((q_j - z_j) * s_j).  0x6400 | q is the FP16
+// value 1024 + q, so one subtraction of two such values gives q - z exactly;
+// the single FP16 multiplication then rounds once, to nearest even.
+// BF16 mode (BF = true; the AWQ card's stock-runtime paragraph: the FP16
+// scales are rounded to BF16 on load and the arithmetic is BF16):
+// bf16_rn((q_j - z_j) * bf16_rn(s_j)).  0x4300 | q is the BF16 value 128 + q
+// (7 fraction bits), so the same one-subtraction trick stays exact, and the
+// scales are rounded once from FP16 when the group is prepared.
+//
+// (W >> 4m) & 0x000F000F | magic yields the pair (q_m, q_{m+4}) in one logic
+// operation, so the arithmetic runs on the pairs (m, m+4) and four byte
+// permutations restore the column order.  The zero points and scales of a
+// group (AwqGroup) are prepared once for its 32 rows.
 struct AwqGroup {
-  uint32_t z[4];  // FP16 pairs (1024 + z_m, 1024 + z_{m+4})
-  uint32_t s[4];  // FP16 pairs (s_m, s_{m+4})
+  uint32_t z[4];  // 16-bit pairs (magic + z_m, magic + z_{m+4})
+  uint32_t s[4];  // 16-bit pairs (s_m, s_{m+4}) in the operand type
 };
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2_rn(uint32_t v) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+template <bool BF = false>
 __device__ __forceinline__ AwqGroup awq_group(uint32_t Z, uint4 S) {
+  constexpr uint32_t magic = BF ? 0x43004300u : 0x64006400u;
   AwqGroup g;
 #pragma unroll
-  for (int m = 0; m < 4; ++m) g.z[m] = ((Z >> (4 * m)) & 0x000F000Fu) | 0x64006400u;
+  for (int m = 0; m < 4; ++m) g.z[m] = ((Z >> (4 * m)) & 0x000F000Fu) | magic;
   g.s[0] = __byte_perm(S.x, S.z, 0x5410);
   g.s[1] = __byte_perm(S.x, S.z, 0x7632);
   g.s[2] = __byte_perm(S.y, S.w, 0x5410);
   g.s[3] = __byte_perm(S.y, S.w, 0x7632);
+  if (BF) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) g.s[m] = f16x2_to_bf16x2_rn(g.s[m]);
+  }
   return g;
 }
+template <bool BF = false>
 __device__ __forceinline__ uint4 awq_dequant8(uint32_t W, const AwqGroup& g) {
+  constexpr uint32_t magic = BF ? 0x43004300u : 0x64006400u;
   uint32_t d[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    uint32_t q = ((W >> (4 * m)) & 0x000F000Fu) | 0x64006400u;
-    __half2 t = __hsub2(*reinterpret_cast<__half2*>(&q), *reinterpret_cast<const __half2*>(&g.z[m]));
-    __half2 v = __hmul2(t, *reinterpret_cast<const __half2*>(&g.s[m]));
-    d[m] = *reinterpret_cast<uint32_t*>(&v);  // (c_m, c_{m+4})
+    const uint32_t q = ((W >> (4 * m)) & 0x000F000Fu) | magic;
+    if (BF) {
+      uint32_t t;
+      asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(q), "r"(g.z[m]));
+      asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d[m]) : "r"(t), "r"(g.s[m]));
+    } else {
+      __half2 t = __hsub2(*reinterpret_cast<const __half2*>(&q), *reinterpret_cast<const __half2*>(&g.z[m]));
+      __half2 v = __hmul2(t, *reinterpret_cast<const __half2*>(&g.s[m]));
+      d[m] = *reinterpret_cast<uint32_t*>(&v);  // (c_m, c_{m+4})
+    }
   }
   return make_uint4(__byte_perm(d[0], d[1], 0x5410), __byte_perm(d[2], d[3], 0x5410), __byte_perm(d[0], d[1], 0x7632),
                     __byte_perm(d[2], d[3], 0x7632));
 }
-__device__ __forceinline__ uint4 awq_dequant8(uint32_t W, uint32_t Z, uint4 S) { return awq_dequant8(W, awq_group(Z, S)); }
+template <bool BF = false>
+__device__ __forceinline__ uint4 awq_dequant8(uint32_t W, uint32_t Z, uint4 S) {
+  return awq_dequant8<BF>(W, awq_group<BF>(Z, S));
+}
 
 // Shared-memory matrix descriptor of an MN-major operand in the 128-byte
 // swizzled layout: atoms of 64 16-bit elements along MN by 8 rows along K

@@ -29,10 +29,12 @@
 //     provides it, else with six TMA boxes from the checkpoint layout; eight dequantisation warps
 //     expand it, exactly (fp16_rn((q - z) * s)), into an MN-major swizzled
 //     FP16 tile, and the MMA reads that.
+//   WQ = 2: the same in the BF16 mode (BF16 activations and shared expert;
+//     the FP16 scales rounded to BF16, bf16_rn((q - z) * s) tiles).
 //
 // Warp roles: 0 TMA producer, 1 UMMA issuer (TMEM owner), 2..5 epilogue,
 // 6..9 token gather (cp.async, arriving on the stage's barrier), 10..17 AWQ
-// dequantisation (WQ = 1).  TMEM: two 16-column phase-A accumulators
+// dequantisation (WQ = 1, 2).  TMEM: two 16-column phase-A accumulators
 // (columns 0..31) and one phase-B accumulator of H/128 blocks x 16 columns
 // (from column 32).
 #include "common.cuh"
@@ -578,11 +580,11 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
           for (int u = 0; u < KSUB; ++u) {
             if (u < nsub) {
               uint8_t* at = sub(stage, u) + atom_off;
-              const AwqGroup g0 = awq_group(z[u][0], sv[u][0]), g1 = awq_group(z[u][1], sv[u][1]);
+              const AwqGroup g0 = awq_group<WQ == 2>(z[u][0], sv[u][0]), g1 = awq_group<WQ == 2>(z[u][1], sv[u][1]);
 #pragma unroll
               for (int i = 0; i < NRW; ++i) {
                 const int r = r0 + 16 * i;  // rows 0..31 use group 0, 32..63 group 1
-                const uint4 v = awq_dequant8(cv[u][i], i < NRW / 2 ? g0 : g1);
+                const uint4 v = awq_dequant8<WQ == 2>(cv[u][i], i < NRW / 2 ? g0 : g1);
                 const uint32_t off = uint32_t(r >> 3) * AQ_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
                 *reinterpret_cast<uint4*>(at + off) = v;
               }
@@ -712,16 +714,18 @@ int decode_experts_fused(const void* x, const int32_t* row_token, const int32_t*
 }
 
 // The same with the routed experts in AWQ W4A16 g32 (qw_* input-major codes,
-// qz_* zero points, sc_* FP16 scales; FP16 activations) and the shared
-// expert in FP16.  qpack: the tile-packed copy of the routed weights (awq.cu
-// awq_prepack) or null; when given, the kernel reads only it.
+// qz_* zero points, sc_* FP16 scales) and a 16-bit shared expert: FP16
+// activations, or the BF16 mode (dtype BF16: scales rounded to BF16, BF16
+// weights, activations and shared expert; template WQ = 2).  qpack: the
+// tile-packed copy of the routed weights (awq.cu awq_prepack) or null; when
+// given, the kernel reads only it.
 int decode_experts_fused_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H,
                              int I, int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu,
                              const int32_t* qw_d, const int32_t* qz_d, const void* sc_d, const void* w_sh_gu,
-                             const void* w_sh_d, int f_fp32, void* f, void* shared_out, void* ws, size_t ws_bytes,
-                             cudaStream_t stream, const void* qpack) {
+                             const void* w_sh_d, int dtype, int f_fp32, void* f, void* shared_out, void* ws,
+                             size_t ws_bytes, cudaStream_t stream, const void* qpack) {
   Args a;
-  int rc = fill_args(a, x, row_token, offsets, T, rows, H, I, E, MOE_DTYPE_F16, ws, ws_bytes);
+  int rc = fill_args(a, x, row_token, offsets, T, rows, H, I, E, dtype, ws, ws_bytes);
   if (rc) return rc;
   a.qpack = static_cast<const uint8_t*>(qpack);
   Maps m;
@@ -737,6 +741,7 @@ int decode_experts_fused_awq(const void* x, const int32_t* row_token, const int3
   if (!rc) rc = make_tmap_2d(&m.qs_d, sc_d, E * (I / 32), H, 2, 2, BM, none);
   if (!rc) rc = make_tmap_2d(&m.qz_d, qz_d, E * (I / 32), H / 8, 4, 2, 16, none);
   if (rc) return rc;
+  if (a.bf16) return launch_fused<2>(m, a, f_fp32, f, shared_out, stream);
   return launch_fused<1>(m, a, f_fp32, f, shared_out, stream);
 }
 

@@ -16,7 +16,7 @@ constexpr int kGatherThreads = 128;   // 4 row-gather warps (A rows loaded throu
 constexpr int kStoreStride = 128 + 16;  // epilogue staging: bytes per row of a 32-column chunk, padded
 constexpr int kSmemBudget = 196 * 1024;
 
-enum { W_DENSE = 0, W_AWQ = 1 };
+enum { W_DENSE = 0, W_AWQ = 1, W_AWQ_BF16 = 2 };  // AWQ_BF16: the BF16 mode of the AWQ dequantisation
 
 template <int BN, int EPI, int WQ, int AG>
 struct GemmCfg {
@@ -438,11 +438,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ, AG>::THREADS, 1)
         uint32_t cw[NR];
 #pragma unroll
         for (int i = 0; i < NR; ++i) cw[i] = codes[(r0 + i * RP) * W2];
-        const AwqGroup g0 = awq_group(z0, s0), g1 = awq_group(z1, s1);
+        const AwqGroup g0 = awq_group<WQ == W_AWQ_BF16>(z0, s0), g1 = awq_group<WQ == W_AWQ_BF16>(z1, s1);
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
           const int r = r0 + i * RP;
-          const uint4 v = awq_dequant8(cw[i], r < 32 ? g0 : g1);
+          const uint4 v = awq_dequant8<WQ == W_AWQ_BF16>(cw[i], r < 32 ? g0 : g1);
           const uint32_t off = uint32_t(r >> 3) * Cfg::B_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
           *reinterpret_cast<uint4*>(btile + off) = v;
         }
@@ -589,7 +589,6 @@ int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, c
                             cudaStream_t stream) {
   int rc = check_common(args, epi, bn);
   if (rc) return rc;
-  MOE_REQUIRE(args.bf16 == 0, MOE_ERR_UNSUPPORTED, "AWQ GEMM runs on FP16 activations");
   MOE_REQUIRE(args.K % 32 == 0, MOE_ERR_UNSUPPORTED, "AWQ K=%d is not a multiple of the group size 32", args.K);
   if (a_rows == 0) return MOE_OK;
   const int bnh = epi == EPI_SWIGLU ? bn / 2 : bn;
@@ -607,6 +606,7 @@ int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, c
   rc = make_tmap_2d(&bm.zeros, qzeros, G * (args.K / 32), n_total / 8, 4, 2, bnh / 8, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
   MOE_REQUIRE(args.row_token == nullptr, MOE_ERR_UNSUPPORTED, "AWQ GEMM reads pre-gathered rows");
+  if (args.bf16) return dispatch<W_AWQ_BF16, 0>(ta, bm, args, epi, bn, stream);
   return dispatch<W_AWQ, 0>(ta, bm, args, epi, bn, stream);
 }
 

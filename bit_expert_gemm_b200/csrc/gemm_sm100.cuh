@@ -47,12 +47,13 @@ struct GemmArgs {
 int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_total, const GemmArgs& args, int epi,
                         int bn, cudaStream_t stream);
 
-// Same GEMM with AWQ W4A16 group-32 weights as B (FP16 operands).  Per group
-// the stored projection has K input rows and n_total output columns:
-// qweight [G*K, n_total/8] int32, qzeros [G*K/32, n_total/8] int32, scales
-// [G*K/32, n_total] FP16.  Dequantisation warps turn each staged tile of
-// codes into FP16 weights in shared memory (exactly fp16_rn((q-z)*s)) that
-// the tensor cores read MN-major.  args.up_offset is the column of the up
+// Same GEMM with AWQ W4A16 group-32 weights as B.  Per group the stored
+// projection has K input rows and n_total output columns: qweight [G*K,
+// n_total/8] int32, qzeros [G*K/32, n_total/8] int32, scales [G*K/32,
+// n_total] FP16.  Dequantisation warps turn each staged tile of codes into
+// 16-bit weights in shared memory that the tensor cores read MN-major:
+// exactly fp16_rn((q-z)*s) with FP16 operands (args.bf16 = 0), or
+// bf16_rn((q-z)*bf16_rn(s)) in the BF16 mode (args.bf16 = 1).  args.up_offset is the column of the up
 // half (SwiGLU); args.b_rows_per_group is unused.
 int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, const int32_t* qzeros,
                             const void* scales, int n_total, const GemmArgs& args, int epi, int bn,

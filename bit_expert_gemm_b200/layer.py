@@ -105,9 +105,8 @@ class MoELayer:
         self.offsets = torch.empty((E + 1,), dtype=i32, device=d)
         self.row_token = torch.empty((rows,), dtype=i32, device=d)
         self.slot_row = torch.empty((T_max, ks), dtype=i32, device=d)
-        f_dt = torch.float32 if self.extra else (torch.float16 if self.fmt == "awq_g32" else torch.bfloat16)
-        if self.fmt == "bf16" and not self.extra:
-            f_dt = self.adt
+        # routed rows f: FP32 for Refill, else the activation dtype (BF16 for NVFP4)
+        f_dt = torch.float32 if self.extra else (self.adt if self.fmt in ("bf16", "awq_g32") else torch.bfloat16)
         self.f = torch.empty((rows, H), dtype=f_dt, device=d)
         self.shared = torch.empty((T_max, H), dtype=self.adt, device=d)
         # optional shared-expert gate (weights key "w_sh_gate", [H]): sigmoid(x . w) per token

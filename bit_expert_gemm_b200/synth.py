@@ -52,6 +52,10 @@ WORKLOADS: Dict[str, Workload] = {
     # AWQ W4A16 g32 experts, FP16 activations, FP16 router and shared expert
     "awq_g32": Workload("awq_g32", H=2048, E=512, k=10, I=640, I_sh=640, bias_std=1.5, fmt="awq_g32", act="f16",
                         T_prefill=8192, T_decode=(1, 8, 32)),
+    # the same AWQ experts in the BF16 mode: BF16 activations, router and shared
+    # expert; the FP16 scales are rounded to BF16 by the kernels
+    "awq_g32_bf16": Workload("awq_g32_bf16", H=2048, E=512, k=10, I=640, I_sh=640, bias_std=1.5, fmt="awq_g32",
+                             act="bf16", T_prefill=8192, T_decode=(1, 8, 32)),
     # NVFP4 W4A4 experts of a 50%-pruned layer; BF16 router and shared expert
     "nvfp4": Workload("nvfp4", H=2048, E=256, k=10, I=640, I_sh=640, bias_std=1.5, fmt="nvfp4", act="bf16",
                       T_prefill=16384),

@@ -220,10 +220,14 @@ MOE_API int moe_experts_bf16(const void* x, const int32_t* row_token, const int3
 
 /* ---------------------------------------------------------------------------
  * Grouped SwiGLU expert FFN with AWQ W4A16 asymmetric group-32 weights [AWQ].
- * Same maths as moe_grouped_swiglu_bf16 with FP16 activations, h rounded to
- * FP16, and each weight dequantised exactly as
- *     W[k, n] = fp16_rn((q[k, n] - z[k/32, n]) * s[k/32, n])
- * (the inverse of the card's code rule).  Layout per projection with input
+ * Same maths as moe_grouped_swiglu_bf16 with 16-bit activations of `dtype`,
+ * h rounded to that type, and each weight dequantised exactly as
+ *     MOE_DTYPE_F16:  W[k, n] = fp16_rn((q[k, n] - z[k/32, n]) * s[k/32, n])
+ * (the inverse of the card's code rule), or in the BF16 mode the card's
+ * stock-runtime paragraph describes (FP16 scales rounded to BF16 on load,
+ * BF16 arithmetic, at most 0.4 % relative change per scale):
+ *     MOE_DTYPE_BF16: W[k, n] = bf16_rn((q - z) * bf16_rn(s)).
+ * The stored scales are FP16 in both modes.  Layout per projection with input
  * dim K and output dim N, input-major ("GEMM" orientation):
  *     qweight [K, N/8] int32: word w of row k holds the codes of output
  *             columns 8w .. 8w+7, column 8w+i in bits 4i .. 4i+3;
@@ -233,19 +237,20 @@ MOE_API int moe_experts_bf16(const void* x, const int32_t* row_token, const int3
  *   qw_gu [E, H, 2I/8], qz_gu [E, H/32, 2I/8], sc_gu [E, H/32, 2I].
  * Down projection: K = I, N = H: qw_d [E, I, H/8], qz_d [E, I/32, H/8],
  *   sc_d [E, I/32, H].
- * x [T, H] FP16; f [rows, H], FP32 when out_fp32 != 0, else FP16.
+ * x [T, H] dtype; f [rows, H], FP32 when out_fp32 != 0, else dtype.
  * Limits: H % 64 == 0, I % 64 == 0.  Workspace: MOE_OP_SWIGLU_AWQ_G32.
  * ------------------------------------------------------------------------- */
 MOE_API int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
                                int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
                                const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
-                               int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream);
+                               int dtype, int out_fp32, void* f, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Routed AWQ experts and the FP16 shared expert of one layer in one call
+ * Routed AWQ experts and the 16-bit shared expert of one layer in one call
  * [AWQ] [ARCH]: the routed part is moe_grouped_swiglu_awq_g32 (f [rows, H]),
  * the shared part the SwiGLU of every token with w_sh_gate_up [2I, H] and
- * w_sh_down [H, I] FP16 (shared_out [T, H] FP16).  For T <= 16 (decode) both
+ * w_sh_down [H, I] of `dtype` (shared_out [T, H] dtype: FP16, or BF16 in the
+ * BF16 mode).  For T <= 16 (decode) both
  * run in one weight-streaming kernel: the routed weights stream as packed
  * codes, zero points and scales and are dequantised in shared memory, the
  * second GEMM is split along I into FP32 partials in the workspace that a
@@ -257,7 +262,7 @@ MOE_API int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, 
 MOE_API int moe_experts_awq_g32(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
                                 int rows, int H, int I, int E, const int32_t* qw_gu, const int32_t* qz_gu,
                                 const void* sc_gu, const int32_t* qw_d, const int32_t* qz_d, const void* sc_d,
-                                const void* w_sh_gate_up, const void* w_sh_down, int out_fp32, void* f,
+                                const void* w_sh_gate_up, const void* w_sh_down, int dtype, int out_fp32, void* f,
                                 void* shared_out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
@@ -289,18 +294,19 @@ MOE_API int moe_experts_awq_g32_prepacked(const void* x, const int32_t* row_toke
                                           int T, int rows, int H, int I, int E, const int32_t* qw_gu,
                                           const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
                                           const int32_t* qz_d, const void* sc_d, const void* awq_packed,
-                                          const void* w_sh_gate_up, const void* w_sh_down, int out_fp32, void* f,
-                                          void* shared_out, void* ws, size_t ws_bytes, void* stream);
+                                          const void* w_sh_gate_up, const void* w_sh_down, int dtype, int out_fp32,
+                                          void* f, void* shared_out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * AWQ dequantisation [AWQ], the same device code the grouped GEMM runs on
- * each weight tile: out[b, k, n] = fp16_rn((q - z) * s) for `batch` stacked
- * projections in the layout above (qweight [batch, K, N/8], qzeros
- * [batch, K/32, N/8], scales [batch, K/32, N]); out [batch, K, N] FP16,
- * input-major like the stored codes.  Limits: K % 32 == 0, N % 8 == 0.
+ * each weight tile: out[b, k, n] = fp16_rn((q - z) * s) (dtype F16) or
+ * bf16_rn((q - z) * bf16_rn(s)) (dtype BF16) for `batch` stacked projections
+ * in the layout above (qweight [batch, K, N/8], qzeros [batch, K/32, N/8],
+ * scales [batch, K/32, N] FP16); out [batch, K, N] of dtype, input-major
+ * like the stored codes.  Limits: K % 32 == 0, N % 8 == 0.
  * ------------------------------------------------------------------------- */
 MOE_API int moe_awq_dequant_g32(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K,
-                                int N, void* out, void* stream);
+                                int N, int dtype, void* out, void* stream);
 
 /* ---------------------------------------------------------------------------
  * NVFP4 quantisation of `batch` tensors [rows, K] of 16-bit values [NVFP4]

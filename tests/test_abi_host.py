@@ -16,7 +16,7 @@ def test_library_exports_every_header_symbol():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(abi._SIGS)  # the binding covers exactly the header
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
 
 
 def test_workspace_sizes():
@@ -111,7 +111,14 @@ def test_awq_prepack_sizes_and_checks():
     assert _code("moe_awq_prepack_g32", buf, buf, buf, buf, buf, buf, 4, 2048, 640, buf, 1000, None) == \
         abi.MOE_ERR_WORKSPACE
     assert _code("moe_experts_awq_g32_prepacked", buf, buf, buf, 1, 10, 2048, 640, 16, buf, buf, buf, buf, buf, buf,
-                 None, buf, buf, 0, buf, buf, buf, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG  # awq_packed is null
+                 None, buf, buf, abi.MOE_DTYPE_F16, 0, buf, buf, buf, 1 << 30, None) == \
+        abi.MOE_ERR_INVALID_ARG  # awq_packed is null
+    # the AWQ calls take FP16 or (BF16 mode) BF16 activations, nothing else
+    assert _code("moe_experts_awq_g32", buf, buf, buf, 1, 10, 2048, 640, 16, buf, buf, buf, buf, buf, buf, buf, buf,
+                 7, 0, buf, buf, buf, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("moe_grouped_swiglu_awq_g32", buf, buf, buf, 1, 10, 2048, 640, 16, buf, buf, buf, buf, buf, buf,
+                 7, 0, buf, buf, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG
+    assert _code("moe_awq_dequant_g32", buf, buf, buf, 1, 64, 64, 7, buf, None) == abi.MOE_ERR_INVALID_ARG
 
 
 def test_razor_slice_and_router_norm_reject_bad_arguments():
