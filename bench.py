@@ -63,6 +63,7 @@ WORKLOADS = {
     "awq_bf16_decode_t1": ("awq_g32_bf16", 1, "forward"),
     "nvfp4_prefill": ("nvfp4", 16384, "forward"),
     "nvfp4_decode_t1": ("nvfp4", 1, "forward"),
+    "nvfp4_decode_t8": ("nvfp4", 8, "forward"),
     "nvfp4_decode_t64": ("nvfp4", 64, "forward"),
     "bf16_h2560_prefill": ("bf16_h2560", 8192, "forward"),
     # small case of the same kernels for full ncu captures (64 experts, 2048 tokens)
@@ -271,8 +272,9 @@ KERNEL_NAMES = {"bf16": "moe_experts_bf16 (routed + shared experts: GEMM1/SwiGLU
                         "decode-sized batches stream the weights as the M operand)",
                 "awq_g32": "moe_grouped_swiglu_awq_g32 (row gather + dequantising GEMM1/SwiGLU + GEMM2, tcgen05 "
                            "kind::f16)",
-                "nvfp4": "moe_grouped_swiglu_nvfp4 (activation quantisation + GEMM1/SwiGLU + h quantisation + GEMM2, "
-                         "tcgen05 kind::mxf4nvf4)"}
+                "nvfp4": "moe_grouped_swiglu_nvfp4_prepacked (activation quantisation + GEMM1/SwiGLU + h "
+                         "quantisation + GEMM2: tcgen05 kind::mxf4nvf4; T <= 16: CUDA-core GEMVs with exact dp4a "
+                         "group products) + the BF16 shared expert"}
 
 
 def measured_traffic(workload: str):
@@ -318,7 +320,7 @@ def expert_roofline(wl, layers, T, rows, ffn_ms, peaks) -> dict:
     touched = statistics.mean(touched_each)
     expert_bytes = touched * per_expert
     flops = expert_flops(rows, wl.H, wl.I)
-    with_shared = layer.ws_exp is not None  # the timed call also runs the shared expert
+    with_shared = True  # the timed region (experts_and_shared) also runs the shared expert
     if with_shared:
         sh_bytes = sum(w[k].numel() * w[k].element_size() for k in ("w_sh_gate_up", "w_sh_down"))
         expert_bytes += sh_bytes

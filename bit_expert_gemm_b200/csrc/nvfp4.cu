@@ -1,12 +1,29 @@
 // NVFP4 W4A4: per-tensor amax, group-16 quantisation (E2M1 codes, E4M3 block
 // scales, FP32 global scale), and the grouped SwiGLU built on the
 // block-scaled tcgen05 GEMM (gemm_nvfp4.cu).
+#include <cstdlib>
+
 #include "common.cuh"
 #include "nvfp4.cuh"
 
 namespace moe {
 
 int gather_rows(const void* x, const int32_t* row_token, int rows, int H, void* out, cudaStream_t stream);
+// decode batches (decode_fp4.cu)
+int nvfp4_decode(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
+                 int E, const uint8_t* w_gu, const uint8_t* w1sf, const float* gs_gu, const uint8_t* w_d,
+                 const uint8_t* w2sf, const float* gs_d, const float* act_gs_in, int out_fp32, void* f, uint8_t* xq,
+                 uint8_t* xsf, uint16_t* h, unsigned* amax, float* gs, int32_t* active, cudaStream_t stream);
+
+// BIT_EXPERT_GEMM_FP4_DECODE=0 sends decode batches through the grouped FP4 GEMMs too.
+static bool fp4_decode_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* s = getenv("BIT_EXPERT_GEMM_FP4_DECODE");
+    on = (s && s[0] == '0') ? 0 : 1;
+  }
+  return on != 0;
+}
 
 struct Nvfp4GemmArgs;  // gemm_nvfp4.cu
 int launch_grouped_gemm_nvfp4(const uint8_t* A, const uint8_t* sfa, int a_rows, const uint8_t* B, const uint8_t* sfb,
@@ -295,6 +312,28 @@ int grouped_swiglu_nvfp4(const void* x, const int32_t* row_token, const int32_t*
   }
   MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_grouped_swiglu_nvfp4: workspace of %zu bytes is too small", ws_bytes);
   if (rows == 0) return MOE_OK;
+  if (T <= kFp4DecodeMaxT && E <= 1024 && fp4_decode_enabled()) {
+    // decode batch: CUDA-core GEMVs over the touched experts (decode_fp4.cu),
+    // reading the weight scales in tile order
+    const uint8_t* w1sf = w1sf_packed;
+    const uint8_t* w2sf = w2sf_packed;
+    const int kt1 = (H + 255) / 256, kt2 = (I + 255) / 256;
+    if (!w1sf) {
+      k_pack_sf_b<<<dim3(E * (I / 64), kt1), 128, 0, stream>>>(sf_gu, H, I / 64, 2 * I, 1, I, w.w1sf_p);
+      w1sf = w.w1sf_p;
+    }
+    if (!w2sf) {
+      k_pack_sf_b<<<dim3(E * (H / 128), kt2), 128, 0, stream>>>(sf_d, I, H / 128, H, 0, 0, w.w2sf_p);
+      w2sf = w.w2sf_p;
+    }
+    MOE_CHECK_CUDA(cudaGetLastError());
+    int rc = nvfp4_decode(x, row_token, offsets, T, rows, H, I, E, w_gu, w1sf, gs_gu, w_d, w2sf, gs_d, act_gs_in,
+                          out_fp32, f, w.xq_tok, w.xsf_tok, w.h, w.amax, w.gs, w.tile_start, stream);
+    if (rc) return rc;
+    if (act_gs_out)
+      MOE_CHECK_CUDA(cudaMemcpyAsync(act_gs_out, w.gs, 2 * sizeof(float), cudaMemcpyDeviceToDevice, stream));
+    return MOE_OK;
+  }
   // x: amax over the whole [T, H] input, each token quantised once; GEMM1
   // reads the FP4 rows of the permuted order through row_token (identical to
   // quantising the gathered rows: the quantisation is per row with the one

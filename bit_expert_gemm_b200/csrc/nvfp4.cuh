@@ -5,6 +5,9 @@
 
 namespace moe {
 
+// Largest decode batch the CUDA-core NVFP4 path takes (decode_fp4.cu).
+constexpr int kFp4DecodeMaxT = 16;
+
 // FP32 -> E4M3 (round to nearest even, saturating to +-448).
 __device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
   uint16_t r;

@@ -12,6 +12,8 @@ the synthetic tokens and router weights, as in a layer forward; the expert
 call is the one MoELayer makes for the format: moe_experts_bf16 (routed +
 shared experts), moe_experts_awq_g32_prepacked (routed AWQ + FP16 shared
 experts) or moe_grouped_swiglu_nvfp4_prepacked (routed NVFP4 experts).
+With --layer the whole layer forward (MoELayer: routing, experts, shared
+expert, combine) runs instead, for launch lists of a complete step.
 """
 
 from __future__ import annotations
@@ -22,7 +24,7 @@ import dataclasses
 import torch
 
 from . import abi, synth
-from .layer import prepare_nvfp4_weights
+from .layer import MoELayer, prepare_nvfp4_weights
 
 WORKLOAD_OF = {"bf16": "bf16", "awq_g32": "awq_g32", "nvfp4": "nvfp4"}
 
@@ -34,6 +36,7 @@ def main(argv=None) -> None:
     ap.add_argument("--experts", type=int, default=0, help="override E (0: the workload's)")
     ap.add_argument("--calls", type=int, default=4)
     ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--layer", action="store_true", help="the whole layer forward instead of the expert call")
     a = ap.parse_args(argv)
     if not torch.cuda.is_available():
         raise SystemExit("profile_case needs a CUDA device")
@@ -45,7 +48,12 @@ def main(argv=None) -> None:
     x = synth.make_tokens(wl, a.tokens, seed=a.seed, device=dev)
     _, _, _, off, rt, _ = abi.moe_route_permute(x, w["w_router"], w["bias"], wl.k)
     rows = a.tokens * wl.k
-    if a.fmt == "nvfp4":
+    if a.layer:
+        layer = MoELayer(w, wl.k, a.fmt, T_max=a.tokens)
+
+        def call():
+            layer.forward(x)
+    elif a.fmt == "nvfp4":
         w = prepare_nvfp4_weights(w)
         for key in ("w_gate_up", "w_down"):
             del w[key]
