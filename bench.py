@@ -524,7 +524,7 @@ def run_native(args, dist: Dist) -> None:
             for p in pipes.values():
                 p.finish()
 
-        for i in range(max(2, args.warmup, n_units)):
+        for i in range(max(2, args.warmup, 2 * n_units)):  # every (batch, output buffer) pair once
             e2e_step(i)
         e2e_finish()
         dist.barrier()
@@ -545,7 +545,9 @@ def run_native(args, dist: Dist) -> None:
                "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
                "d2h_bytes_per_step": int(yh[0].numel() * yh[0].element_size()),
                "path": "pinned host x -> H2D copy -> layer (CUDA graph of the C-ABI calls) -> D2H copy of y, "
-                       "with HostPipeline overlapping step i+1's upload and step i-1's download with step i"}
+                       + ("one CUDA graph per step holding the upload, the forward and the download (HostPipeline, "
+                          "decode-sized batch)" if T <= HostPipeline.whole_step_max_T and not args.no_graph else
+                          "with HostPipeline overlapping step i+1's upload and step i-1's download with step i")}
 
     if launches_per_step is None:  # eager: count one pass's launches from a throw-away capture
         launches_per_step = _count_step_kernels(layer, xs[0], lambda xx: step(layer, xx))

@@ -369,13 +369,26 @@ class HostPipeline:
     A host output buffer is complete once finish() (or a later wait on the
     current stream) has returned; a host input buffer may be reused once the
     step after next has been enqueued.
+
+    Decode-sized batches (T <= whole_step_max_T, with graphs) take one CUDA
+    graph per (host x, host y) pair instead, holding the upload, the forward
+    and the download: a step is then one graph launch on the host, which is
+    what bounds a decode step's end-to-end time (the copies are a few KB).
+    Those graphs are recorded on the first step with each pair of host
+    buffers, so a caller that streams from a fixed set of pinned buffers
+    records them all during its warm-up; a host input buffer may then be
+    rewritten once the step that reads it has completed on the GPU.
     """
+
+    whole_step_max_T = 256
 
     def __init__(self, layer: MoELayer, T: int, use_graphs: bool = True):
         assert T <= layer.T_max and layer.extra == 0
         H = layer.w["w_router"].shape[1]
         dev = layer.dev
         self.layer, self.T = layer, T
+        self.whole = use_graphs and T <= self.whole_step_max_T
+        self._step_graphs = {}
         self.x = [torch.empty((T, H), dtype=layer.adt, device=dev) for _ in range(2)]
         self.y = [torch.empty((T, H), dtype=layer.adt, device=dev) for _ in range(2)]
         self.s_in, self.s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -383,7 +396,7 @@ class HostPipeline:
         self.ev_used = [torch.cuda.Event() for _ in range(2)]  # the pass on x[b] is done and y[b] written
         self.ev_out = [torch.cuda.Event() for _ in range(2)]   # y[b] downloaded
         self.graphs = None
-        if use_graphs:
+        if use_graphs and not self.whole:
             self.graphs = [layer.capture(self.x[b], fn=lambda xx, b=b: layer.forward(xx, y=self.y[b]))
                            for b in range(2)]
         self.i = 0
@@ -395,7 +408,27 @@ class HostPipeline:
         self.s_in.wait_stream(cs)
         self.s_out.wait_stream(cs)
 
+    def _whole_step(self, x_host: torch.Tensor, y_host: torch.Tensor) -> None:
+        """Upload, forward and download of one batch as one graph launch."""
+        key = (x_host.data_ptr(), y_host.data_ptr())
+        g = self._step_graphs.get(key)
+        if g is None:
+            x, y, layer = self.x[0], self.y[0], self.layer
+
+            def body():
+                x.copy_(x_host, non_blocking=True)
+                layer.forward(x, y=y)
+                y_host.copy_(y, non_blocking=True)
+
+            g = layer.capture(x, fn=lambda _x: body())
+            self._step_graphs[key] = g
+        g.replay()
+        self.i += 1
+
     def step(self, x_host: torch.Tensor, y_host: torch.Tensor) -> None:
+        if self.whole:
+            self._whole_step(x_host, y_host)
+            return
         b, cs = self.i & 1, torch.cuda.current_stream()
         if self.i >= 2:
             self.s_in.wait_event(self.ev_used[b])  # the pass two steps back has read x[b]

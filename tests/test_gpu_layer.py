@@ -43,11 +43,12 @@ def test_tiny_layer_forward():
     assert abi.moe_device_status() == 0
 
 
-@pytest.mark.parametrize("T,graphs", [(64, True), (8, False)])
+@pytest.mark.parametrize("T,graphs", [(64, True), (1, True), (8, False), (300, True)])
 def test_host_pipeline_matches_forward(bf16_layer, T, graphs):
-    """Batches streamed from pinned host memory by HostPipeline (uploads and
-    downloads overlapped with the neighbouring forwards) come back bit for bit
-    equal to the device forward of the same batches, including when more
+    """Batches streamed from pinned host memory by HostPipeline (decode
+    sizes: one graph per step with the copies inside; larger batches: uploads
+    and downloads overlapped with the neighbouring forwards) come back bit for
+    bit equal to the device forward of the same batches, including when more
     batches than buffers are in flight."""
     from bit_expert_gemm_b200.layer import HostPipeline
     wl, w = bf16_layer
