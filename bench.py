@@ -274,7 +274,8 @@ KERNEL_NAMES = {"bf16": "moe_experts_bf16 (routed + shared experts: GEMM1/SwiGLU
                            "kind::f16)",
                 "nvfp4": "moe_grouped_swiglu_nvfp4_prepacked (activation quantisation + GEMM1/SwiGLU + h "
                          "quantisation + GEMM2: tcgen05 kind::mxf4nvf4; T <= 16: CUDA-core GEMVs with exact dp4a "
-                         "group products) + the BF16 shared expert"}
+                         "group products) + the BF16 shared expert (T <= 16: weight-streaming GEMVs on a second "
+                         "stream)"}
 
 
 def measured_traffic(workload: str):

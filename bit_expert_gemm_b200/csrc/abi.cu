@@ -1,5 +1,6 @@
 // extern "C" entry points declared in include/moe.h: host-side argument
 // checks, workspace sizing, and dispatch to the kernels.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -67,6 +68,10 @@ size_t nvfp4_packed_sf_bytes(int E, int rows_per_expert, int K, int swiglu);
 int nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, int K, int swiglu, uint8_t* out,
                      cudaStream_t stream);
 int shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, float* gate, cudaStream_t stream);
+size_t dense_gemv_ws_bytes(int T, int I);
+bool dense_gemv_fits(int T, int H, int I);
+int dense_swiglu_gemv(const void* x, const int32_t* offsets, int T, int H, int I, const void* w_gu, const void* w_d,
+                      int dtype, int out_fp32, void* out, void* ws, size_t ws_bytes, cudaStream_t stream);
 int router_norm(const void* w_router, int E, int H, int dtype, double* sum_sq, int64_t* count, cudaStream_t stream);
 int slice_experts(const void* src, int E, size_t bytes_per_expert, const int32_t* kept, int keep, void* dst,
                   cudaStream_t stream);
@@ -230,6 +235,16 @@ static constexpr int kFusedMaxT = 16;
 
 // The one-kernel split-K path for T <= 16; BIT_EXPERT_GEMM_DECODE_FUSED=0
 // selects the two-GEMM decode path instead (for comparisons).
+// BIT_EXPERT_GEMM_DENSE_GEMV=0 keeps a lone dense expert of a decode batch on the grouped GEMMs.
+static bool dense_gemv_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* s = getenv("BIT_EXPERT_GEMM_DENSE_GEMV");
+    on = (s && s[0] == '0') ? 0 : 1;
+  }
+  return on != 0;
+}
+
 static bool fused_decode_enabled() {
   static int on = -1;
   if (on < 0) {
@@ -288,6 +303,8 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k_slots, int I) {
     case MOE_OP_SWIGLU_BF16: {
       WsCounter c;
       c.take<uint16_t>(size_t(rows) * I);
+      // one dense expert on a decode batch: the GEMV path's FP32 partials
+      if (E == 1 && dense_gemv_fits(T, H, I)) c.used = std::max(c.used, dense_gemv_ws_bytes(T, I));
       return c.used;
     }
     case MOE_OP_SWIGLU_AWQ_G32: return awq_ws_bytes(rows, H, I, E);
@@ -368,6 +385,10 @@ int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, const int32
               "moe_grouped_swiglu_bf16: null pointer");
   MOE_REQUIRE(aligned16(x) && aligned16(w_gate_up) && aligned16(w_down) && aligned16(f), MOE_ERR_INVALID_ARG,
               "moe_grouped_swiglu_bf16: operands must be 16-byte aligned");
+  // one dense expert (E = 1, rows in order) on a decode batch: weight-streaming GEMVs
+  if (E == 1 && !row_token && dense_gemv_fits(T, H, I) && dense_gemv_enabled())
+    return dense_swiglu_gemv(x, expert_offsets, T, H, I, w_gate_up, w_down, dtype, out_fp32, f, ws, ws_bytes,
+                             static_cast<cudaStream_t>(stream));
   return swiglu_bf16(x, row_token, expert_offsets, T, rows, H, I, E, w_gate_up, w_down, dtype, out_fp32, f, ws,
                      ws_bytes, static_cast<cudaStream_t>(stream));
 }

@@ -118,16 +118,10 @@ class MoELayer:
         self.ws_route = abi.workspace(abi.MOE_OP_ROUTE_PERMUTE, T_max, H, E, ks, 0, d)
         self.ws_ffn = abi.workspace(op, T_max, H, E, ks, self.I, d)
         self.ws_sh = abi.workspace(abi.MOE_OP_SWIGLU_BF16, T_max, H, 1, 1, self.I_sh, d)
-        # decode-sized batches run a separate shared expert through the 16-bit
-        # weight-streaming kernel: moe_experts_bf16 with no routed rows
-        self._sh_stream = T_max <= 16 and H % 128 == 0 and self.I_sh % 64 == 0
+        # decode-sized batches run a separate shared expert (the library's
+        # weight-streaming GEMVs for one dense expert) on a second stream
+        self._sh_stream = T_max <= 16
         if self._sh_stream:
-            need = abi.moe_workspace_size(abi.MOE_OP_EXPERTS_BF16, T_max, H, 1, 1, self.I_sh)
-            if need > self.ws_sh.numel():
-                self.ws_sh = torch.empty(need, dtype=torch.uint8, device=d)
-            self._sh_no_rows = torch.zeros(2, dtype=i32, device=d)   # offsets of an empty routed group
-            self._sh_dummy_rt = torch.zeros(1, dtype=i32, device=d)
-            self._sh_dummy_f = torch.empty((1, H), dtype=self.adt, device=d)
             self._side = torch.cuda.Stream(device=d)
         if self.fmt in ("bf16", "awq_g32") and self.I_sh == self.I:
             # routed + shared experts in one call: big enough for every path it
@@ -177,13 +171,8 @@ class MoELayer:
     def shared_expert(self, x: torch.Tensor) -> torch.Tensor:
         T = x.shape[0]
         sh = self.shared[:T]
-        gu, wd = self.w["w_sh_gate_up"].unsqueeze(0), self.w["w_sh_down"].unsqueeze(0)
-        if self._sh_stream and T <= 16:
-            abi.moe_experts_bf16(x, self._sh_dummy_rt, self._sh_no_rows, 0, gu, wd, self.w["w_sh_gate_up"],
-                                 self.w["w_sh_down"], f=self._sh_dummy_f, shared_out=sh, ws=self.ws_sh)
-        else:
-            abi.moe_grouped_swiglu_bf16(x, None, self._shared_offsets(T), T, gu, wd, out_fp32=False, f=sh,
-                                        ws=self.ws_sh)
+        abi.moe_grouped_swiglu_bf16(x, None, self._shared_offsets(T), T, self.w["w_sh_gate_up"].unsqueeze(0),
+                                    self.w["w_sh_down"].unsqueeze(0), out_fp32=False, f=sh, ws=self.ws_sh)
         return sh
 
     def experts_and_shared(self, x: torch.Tensor):

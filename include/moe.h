@@ -190,8 +190,11 @@ MOE_API int moe_permute_noalloc(const int32_t* topk_idx, int T, int k_slots, int
  * with E = 1 and expert_offsets = {0, T}); expert_offsets [E+1] int32 on the
  * device, expert_offsets[E] == rows; w_gate_up [E, 2I, H] dtype; w_down
  * [E, H, I] dtype; f [rows, H], FP32 when out_fp32 != 0, else dtype.
+ * A dense expert (E = 1, row_token NULL) on T <= 16 tokens with H % 256 == 0
+ * runs as two weight-streaming GEMV launches over all SMs (FP32 sums, h
+ * rounded to dtype) instead of the tiled GEMMs.
  * Limits: H % 64 == 0, I % 64 == 0, E <= 1024.  Workspace:
- * MOE_OP_SWIGLU_BF16 (holds the gathered rows and h).
+ * MOE_OP_SWIGLU_BF16 (holds h, or the GEMV path's FP32 partials).
  * ------------------------------------------------------------------------- */
 MOE_API int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T,
                             int rows, int H, int I, int E, const void* w_gate_up, const void* w_down, int dtype,

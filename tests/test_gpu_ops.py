@@ -127,6 +127,31 @@ def test_dense_expert_identity_rows():
     assert rel_err(f64(f), ref) < 1e-2
 
 
+@pytest.mark.parametrize("T,H,I,act,out_fp32", [(1, 2048, 640, "bf16", False), (3, 2048, 640, "f16", True),
+                                               (8, 256, 64, "bf16", False), (16, 2560, 640, "bf16", True),
+                                               (13, 512, 128, "f16", False)])
+def test_dense_expert_decode_gemv(T, H, I, act, out_fp32):
+    """One dense expert (the shared expert) on a decode batch: the
+    weight-streaming GEMV path of moe_grouped_swiglu_bf16, against the
+    oracle; an expert row range that ends before the batch leaves the later
+    output rows untouched."""
+    wl, w, x, _ = _ffn_case(T, H, I, 1, 1, act, seed=T + 21)
+    gu, wd = w["w_gate_up"][0], w["w_down"][0]  # expert 0 as the dense expert
+    sg = f64(gu)
+    ref, _ = moe.swiglu_expert(f64(x), sg[:I], sg[I:], f64(wd))
+    off = torch.tensor([0, T], dtype=torch.int32, device=DEV)
+    f = abi.moe_grouped_swiglu_bf16(x, None, off, T, gu.unsqueeze(0), wd.unsqueeze(0), out_fp32=out_fp32)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0
+    assert rel_err(f64(f), ref) < TOL_BF16
+    if T > 2:
+        off2 = torch.tensor([0, T - 2], dtype=torch.int32, device=DEV)
+        f2 = torch.full_like(f, 7.0)
+        abi.moe_grouped_swiglu_bf16(x, None, off2, T, gu.unsqueeze(0), wd.unsqueeze(0), out_fp32=out_fp32, f=f2)
+        torch.cuda.synchronize()
+        assert torch.equal(f2[: T - 2], f[: T - 2]) and bool((f2[T - 2:] == 7.0).all())
+
+
 @pytest.mark.parametrize("T,H,E,k,ks,f32", [(1, 2048, 512, 10, 10, False), (300, 512, 16, 3, 4, False),
                                             (257, 2048, 64, 10, 11, True)])
 def test_combine(T, H, E, k, ks, f32):
