@@ -138,6 +138,16 @@ def combine(f_rows: np.ndarray, slot_row: np.ndarray, w: np.ndarray, shared: Opt
     return y
 
 
+def rmsnorm(x: np.ndarray, w: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """Pre-norm RMSNorm with a (1 + w) gain (architecture fact sheet:
+    "RMSNorm (1+w gain)", pre-norm, epsilon 1e-06): the MoE block's input is
+    x / sqrt(mean(x^2) + eps) * (1 + w) over the hidden dimension.
+    x [T, H], w [H] -> [T, H]."""
+    x = np.asarray(x, np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * (1.0 + np.asarray(w, np.float64))
+
+
 def shared_gate(x: np.ndarray, w_gate: np.ndarray) -> np.ndarray:
     """Per-token shared-expert gate 1 / (1 + exp(-x . w_gate)).
     x [T, H], w_gate [H] -> [T]."""

@@ -184,3 +184,20 @@ def test_layer_with_gate_scales_only_the_shared_expert():
     assert np.allclose(gated["y"], routed["y"] + s_only / (1.0 + np.exp(-z))[:, None], rtol=1e-12, atol=1e-12)
     half = moe.moe_layer(x, wr, b, wl.k, ew, sh, shared_gate_w=np.zeros_like(g))
     assert np.allclose(half["y"], routed["y"] + 0.5 * s_only, rtol=1e-12, atol=1e-12)
+
+
+def test_rmsnorm_against_torch_and_closed_forms():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((7, 64)) * 3.0
+    w = rng.standard_normal(64) * 0.1
+    got = moe.rmsnorm(x, w)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (64,), weight=torch.from_numpy(1.0 + w), eps=1e-6)
+    assert np.allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
+    # a constant row c: c / sqrt(c^2 + eps) * (1 + w); w = -1 silences a feature
+    c = np.full((1, 8), 2.0)
+    wz = np.zeros(8)
+    wz[3] = -1.0
+    y = moe.rmsnorm(c, wz)
+    assert np.allclose(y[0, [0, 1, 2, 4]], 2.0 / np.sqrt(4.0 + 1e-6), rtol=1e-15) and y[0, 3] == 0.0
+    # scale invariance away from eps
+    assert np.allclose(moe.rmsnorm(1e3 * x, w), got, rtol=1e-6)  # eps / mean(x^2) is about 1e-7 here
