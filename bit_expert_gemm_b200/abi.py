@@ -71,6 +71,7 @@ _SIGS = {
     "razor_select": (_I, [_P, _P, _I, _I, _P, _P, _P, _P]),
     "razor_router_norm": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "moe_shared_gate": (_I, [_P, _I, _I, _P, _I, _P, _P]),
+    "moe_rmsnorm": (_I, [_P, _I, _I, _P, ctypes.c_float, _I, _P, _P]),
     "razor_slice": (_I, [_P, _I, _SZ, _P, _I, _P, _P]),
 }
 
@@ -481,6 +482,17 @@ def moe_shared_gate(x, w_gate, gate=None, stream=None):
     _need(gate, torch.float32, "gate")
     _call("moe_shared_gate", _p(x), T, H, _p(w_gate), _dtype_code(x), _p(gate), _stream(stream))
     return gate
+
+
+def moe_rmsnorm(x, w, eps: float = 1e-6, y=None, stream=None):
+    """Pre-MoE RMSNorm with the (1 + w) gain: y [T, H] (may be x)."""
+    T, H = x.shape
+    if w.dtype != x.dtype or tuple(w.shape) != (H,):
+        raise ValueError("moe_rmsnorm: w must be [H] of x's dtype")
+    if y is None:
+        y = torch.empty_like(x)
+    _call("moe_rmsnorm", _p(x), T, H, _p(w), float(eps), _dtype_code(x), _p(y), _stream(stream))
+    return y
 
 
 def razor_router_norm(w_router, sum_sq=None, count=None, stream=None):

@@ -68,6 +68,7 @@ size_t nvfp4_packed_sf_bytes(int E, int rows_per_expert, int K, int swiglu);
 int nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, int K, int swiglu, uint8_t* out,
                      cudaStream_t stream);
 int shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, float* gate, cudaStream_t stream);
+int rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, cudaStream_t stream);
 size_t dense_gemv_ws_bytes(int T, int I);
 bool dense_gemv_fits(int T, int H, int I);
 int dense_swiglu_gemv(const void* x, const int32_t* offsets, int T, int H, int I, const void* w_gu, const void* w_d,
@@ -650,6 +651,18 @@ int moe_shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, 
   MOE_REQUIRE(aligned16(x) && aligned16(w_gate), MOE_ERR_INVALID_ARG,
               "moe_shared_gate: x and w_gate must be 16-byte aligned");
   return shared_gate(x, T, H, w_gate, dtype, gate, static_cast<cudaStream_t>(stream));
+}
+
+int moe_rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, void* stream) {
+  MOE_REQUIRE(T >= 0 && H >= 8 && H % 8 == 0, MOE_ERR_UNSUPPORTED, "moe_rmsnorm: T=%d H=%d (need H %% 8 == 0)", T,
+              H);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_rmsnorm: dtype=%d", dtype);
+  MOE_REQUIRE(eps >= 0.0f, MOE_ERR_INVALID_ARG, "moe_rmsnorm: eps must be >= 0");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(x && w && y, MOE_ERR_INVALID_ARG, "moe_rmsnorm: null pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(w) && aligned16(y), MOE_ERR_INVALID_ARG,
+              "moe_rmsnorm: x, w and y must be 16-byte aligned");
+  return rmsnorm(x, T, H, w, eps, dtype, y, static_cast<cudaStream_t>(stream));
 }
 
 int razor_router_norm(const void* w_router, int E, int H, int dtype, double* sum_sq, int64_t* count, void* stream) {

@@ -67,3 +67,71 @@ int shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, floa
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Pre-MoE RMSNorm with a (1 + w) gain (architecture fact sheet:
+// "RMSNorm (1+w gain)", pre-norm, epsilon 1e-06):
+//   y[t, h] = x[t, h] / sqrt(mean_h x[t, :]^2 + eps) * (1 + w[h])
+// One warp per token: the sum of squares in FP32 over 16-byte pieces
+// (lane-strided, then a shuffle tree), the scale with an IEEE square root and
+// division, then a second pass over the row (from L1/L2) that scales and
+// writes it in 16 bits; every lane rewrites only the pieces it reads, after
+// the sum is complete, so y may be x.
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+template <typename T16>
+__global__ void __launch_bounds__(256) k_rmsnorm(const T16* x, const T16* __restrict__ w, int T, int H, float eps,
+                                                 T16* y) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + size_t(t) * H);
+  const int nv = H / 8;
+  float ss = 0.f;
+  for (int c = lane; c < nv; c += 32) {
+    const uint4 v = xr[c];
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = Pack2<T16>::unpack(u[j]);
+      ss = fmaf(f.x, f.x, ss);
+      ss = fmaf(f.y, f.y, ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = 1.0f / sqrtf(ss / float(H) + eps);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  uint4* yr = reinterpret_cast<uint4*>(y + size_t(t) * H);
+  for (int c = lane; c < nv; c += 32) {
+    const uint4 v = xr[c], g = __ldg(wr + c);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w}, gw[4] = {g.x, g.y, g.z, g.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = Pack2<T16>::unpack(u[j]), gg = Pack2<T16>::unpack(gw[j]);
+      o[j] = Pack2<T16>::pack(f.x * r * (1.0f + gg.x), f.y * r * (1.0f + gg.y));
+    }
+    yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace
+
+int rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, cudaStream_t stream) {
+  if (T == 0) return MOE_OK;
+  const dim3 grid((T + 7) / 8);
+  if (dtype == MOE_DTYPE_BF16)
+    k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x),
+                                                       static_cast<const __nv_bfloat16*>(w), T, H, eps,
+                                                       static_cast<__nv_bfloat16*>(y));
+  else
+    k_rmsnorm<__half><<<grid, 256, 0, stream>>>(static_cast<const __half*>(x), static_cast<const __half*>(w), T, H,
+                                                eps, static_cast<__half*>(y));
+  MOE_CHECK_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -396,6 +396,15 @@ MOE_API int moe_combine(const void* f, int f_fp32, const int32_t* slot_row, int 
                 void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Pre-MoE RMSNorm [ARCH] ("RMSNorm (1+w gain)", pre-norm, epsilon 1e-06):
+ *   y[t, h] = x[t, h] / sqrt(mean_h x[t, :]^2 + eps) * (1 + w[h])
+ * with FP32 sums, rounded once to dtype.  x, y [T, H] dtype (y may be x);
+ * w [H] dtype; all 16-byte aligned.  The fact sheet's eps is 1e-6.
+ * Limits: H % 8 == 0.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Shared-expert gate [AWQ] ("Checkpoint": a shared-expert gate tensor is
  * stored with the router and the shared expert; the card gives no formula,
  * so this is the plainest reading):

@@ -149,3 +149,14 @@ def test_keep_manifest():
     for bad in ([2, 1], [1, 1], [0, 8]):
         with pytest.raises(ValueError):
             keep_manifest(bad, 8)
+
+
+def test_rmsnorm_rejects_bad_arguments():
+    p = ctypes.c_void_p
+    assert _code("moe_rmsnorm", p(256), 4, 100, p(512), ctypes.c_float(1e-6), 0, p(1024), None) == \
+        abi.MOE_ERR_UNSUPPORTED  # H % 8 != 0
+    assert _code("moe_rmsnorm", p(256), 4, 64, p(512), ctypes.c_float(1e-6), 9, p(1024), None) == \
+        abi.MOE_ERR_INVALID_ARG  # dtype
+    assert _code("moe_rmsnorm", p(260), 4, 64, p(512), ctypes.c_float(1e-6), 0, p(1024), None) == \
+        abi.MOE_ERR_INVALID_ARG  # misaligned x
+    assert _code("moe_rmsnorm", None, 0, 64, None, ctypes.c_float(1e-6), 0, None, None) == abi.MOE_OK  # empty batch

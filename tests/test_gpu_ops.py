@@ -319,3 +319,18 @@ def test_layer_with_shared_gate_forward_and_refill():
     assert np.array_equal(cc.cpu().numpy()[good], c_ref[good])
     assert rel_err(ss.cpu().numpy()[good], s_ref[good]) < TOL_BF16
     assert abi.moe_device_status() == 0
+
+
+@pytest.mark.parametrize("T,H,act,inplace", [(1, 2048, "bf16", False), (7, 256, "f16", True),
+                                             (8192, 2048, "bf16", False), (33, 2560, "bf16", True)])
+def test_rmsnorm(T, H, act, inplace):
+    wl = _wl(H=H, act=act)
+    x = synth.make_tokens(wl, T, seed=T + 3, device=DEV)
+    g = synth.make_shared_gate(wl, seed=T + 3, device=DEV)  # any [H] vector serves as the gain w
+    want = moe.rmsnorm(f64(x), f64(g))
+    y = abi.moe_rmsnorm(x, g, y=x if inplace else None)
+    torch.cuda.synchronize()
+    assert (y.data_ptr() == x.data_ptr()) == inplace
+    # FP32 sums, one rounding to 16 bits
+    assert rel_err(f64(y), want) < 1e-2
+    assert abi.moe_device_status() == 0
