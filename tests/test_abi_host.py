@@ -160,3 +160,25 @@ def test_rmsnorm_rejects_bad_arguments():
     assert _code("moe_rmsnorm", p(260), 4, 64, p(512), ctypes.c_float(1e-6), 0, p(1024), None) == \
         abi.MOE_ERR_INVALID_ARG  # misaligned x
     assert _code("moe_rmsnorm", None, 0, 64, None, ctypes.c_float(1e-6), 0, None, None) == abi.MOE_OK  # empty batch
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/moe.h compiles as strict C99, and a C program links against
+    libmoe_b200.so and calls it (moe_abi_version needs no GPU)."""
+    import os
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    inc = os.path.dirname(abi.HEADER)
+    libdir = os.path.dirname(abi.LIB_PATH)
+    src = tmp_path / "use_moe.c"
+    src.write_text('#include "moe.h"\nint main(void) { return moe_abi_version() == 2 ? 0 : 1; }\n')
+    exe = tmp_path / "use_moe"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", f"-I{inc}", str(src),
+                        f"-L{libdir}", "-lmoe_b200", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
