@@ -2,6 +2,7 @@
 cases, error bounds of the rounding rules, and torch conversions."""
 
 import numpy as np
+import pytest
 import torch
 
 from oracle import awq, formats, nvfp4
@@ -168,3 +169,42 @@ def test_w4a4_experts_compose_pinned_pieces():
     # absorbed exactly by the block scales; a 20x smaller one saturates them)
     f2, _, (sx2, sh2) = nvfp4.routed_outputs_w4a4(x, perm, deq, act_gs=(s_x / 20, s_h / 20))
     assert sx2 == np.float32(s_x / 20) and not np.allclose(f2, f)
+
+
+def test_w4a4_group_products_are_exact_integers():
+    """The identity the NVFP4 decode GEMVs rest on: inside one 16-element
+    group both operands are E2M1 values times one scale, 2*e2m1 is an integer
+    in {0, +-1, +-2, +-3, +-4, +-6, +-8, +-12}, so sum (2w)(2x) is an exact
+    integer of at most 16*144 in magnitude, and the dot product of the
+    dequantised operands equals sum_groups int * s_bw * s_bx * s_gw * s_gx / 4
+    exactly (float64)."""
+    rng = np.random.default_rng(11)
+    K = 256
+    w = (rng.standard_normal((3, K)) * 0.05).astype(np.float32)
+    x = rng.standard_normal((1, K)).astype(np.float32)
+    cw, sbw, gw = nvfp4.quantize(w)
+    cx, sbx, gx = nvfp4.quantize(x)
+    two_w = (2 * formats.e2m1_to_f64(cw)).astype(np.int64)
+    two_x = (2 * formats.e2m1_to_f64(cx)).astype(np.int64)
+    assert set(np.unique(np.abs(two_w))) <= {0, 1, 2, 3, 4, 6, 8, 12}
+    deq = nvfp4.dequant(cw, sbw, gw) @ nvfp4.dequant(cx, sbx, gx)[0]
+    for r in range(3):
+        acc = 0.0
+        for g in range(K // 16):
+            isum = int(np.dot(two_w[r, 16 * g:16 * g + 16], two_x[0, 16 * g:16 * g + 16]))
+            assert abs(isum) <= 16 * 144
+            acc += isum * formats.e4m3_to_f64(sbw[r, g]) * formats.e4m3_to_f64(sbx[0, g])
+        assert acc * float(gw) * float(gx) / 4 == pytest.approx(deq[r], rel=1e-15, abs=1e-300)
+
+
+def test_bf16_integer_bit_patterns_used_by_the_awq_bf16_mode():
+    """0x4300 | q is the BF16 value 128 + q for every code q in 0..15, and the
+    difference of two such values is q - z exactly (integers below 256 are
+    exact in BF16), so one rounding remains: the product with the scale."""
+    q = np.arange(16, dtype=np.uint16)
+    vals = formats.bf16_to_f64(np.uint16(0x4300) | q)
+    assert np.array_equal(vals, 128.0 + q)
+    d = vals[:, None] - vals[None, :]
+    assert np.array_equal(formats.bf16_to_f64(formats.f32_to_bf16(d.astype(np.float32))), d)
+    # the FP16 pattern of the FP16 mode: 0x6400 | q is 1024 + q
+    assert np.array_equal(formats.f16_to_f64((np.uint16(0x6400) | q).view(np.float16)), 1024.0 + q)
