@@ -1,9 +1,9 @@
 // RAZOR slicing and the router-norm keep policy.
 //
-// Qwen3.8-Flash-Next-RAZOR-65B-A6B-E256of512 card, opening paragraphs: the
-// surviving expert weights and router rows of a pruned layer are slices of
-// the base checkpoint, taken in matching order, and the keep manifest lists
-// the original expert indices in output order.  Same card, "Selection and
+// Qwen3.8-Flash-Next-RAZOR-65B-A6B-E256of512 card, opening paragraphs: a
+// pruned layer keeps the selected experts' weights and router rows, cut from
+// the original checkpoint in one and the same order, and its manifest lists
+// the original expert indices in the pruned layer's order.  Same card, "Selection and
 // calibration", MTP item: the MTP layer, which the text calibration never
 // runs, keeps the experts whose original router rows have the largest L2
 // norm (policy router_norm).

@@ -69,8 +69,9 @@ int shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, floa
 }  // namespace moe
 
 // ---------------------------------------------------------------------------
-// Pre-MoE RMSNorm with a (1 + w) gain (architecture fact sheet:
-// "RMSNorm (1+w gain)", pre-norm, epsilon 1e-06):
+// Pre-MoE RMSNorm with a (1 + w) gain (architecture fact sheet,
+// normalisation entries: RMSNorm whose gain is 1 + w, before the block,
+// epsilon 1e-6):
 //   y[t, h] = x[t, h] / sqrt(mean_h x[t, :]^2 + eps) * (1 + w[h])
 // One warp per token: the sum of squares in FP32 over 16-byte pieces
 // (lane-strided, then a shuffle tree), the scale with an IEEE square root and

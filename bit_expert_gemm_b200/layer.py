@@ -282,7 +282,7 @@ EXPERT_PACKED = ("awq_packed", "sfp_gu", "sfp_d")
 
 def slice_layer_weights(w: Dict[str, torch.Tensor], kept: torch.Tensor) -> Dict[str, torch.Tensor]:
     """The pruned layer: every per-expert tensor, router rows and bias
-    included, gathered with one kept list (razor_slice, in matching order);
+    included, gathered with one kept list (razor_slice, all in the same order);
     the shared expert and any activation scales are unchanged.  kept [keep]
     int32 on the device, normally razor_select's ascending kept set."""
     E = w["w_router"].shape[0]

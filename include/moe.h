@@ -16,8 +16,9 @@
  *           expert scales) and "Calibration" (code rule
  *           clip(round(w/scale + zero), 0, 15)).
  *   [NVFP4] Qwen3.8-Flash-Next-RAZOR-96B-A6B-NVFP4 card, component table
- *           ("Routed experts: NVFP4 W4A4 (group 16, FP8 block scales, FP32
- *           global scales)"; shared expert and router BF16).
+ *           (routed experts in NVFP4 for weights and activations: FP4 values
+ *           in groups of 16, an FP8 scale per group, an FP32 scale per
+ *           tensor; the shared expert and the router stay BF16).
  *   [RAZOR] Qwen3.8-Flash-Next-RAZOR-65B-A6B-E256of512 card, section
  *           "Selection and calibration" (Refill-RMS score, conditional RMS
  *           aggregation, keep the top 256 / 384, additive statistics) and the
@@ -396,7 +397,8 @@ MOE_API int moe_combine(const void* f, int f_fp32, const int32_t* slot_row, int 
                 void* stream);
 
 /* ---------------------------------------------------------------------------
- * Pre-MoE RMSNorm [ARCH] ("RMSNorm (1+w gain)", pre-norm, epsilon 1e-06):
+ * Pre-MoE RMSNorm [ARCH] (normalisation entries: RMSNorm whose gain is
+ * 1 + w, applied before the block, epsilon 1e-6):
  *   y[t, h] = x[t, h] / sqrt(mean_h x[t, :]^2 + eps) * (1 + w[h])
  * with FP32 sums, rounded once to dtype.  x, y [T, H] dtype (y may be x);
  * w [H] dtype; all 16-byte aligned.  The fact sheet's eps is 1e-6.
@@ -464,8 +466,9 @@ MOE_API int razor_router_norm(const void* w_router, int E, int H, int dtype, dou
 
 /* ---------------------------------------------------------------------------
  * Slice of the kept experts [RAZOR] (opening paragraphs: the surviving
- * expert weights and router rows are slices of the base checkpoint, in
- * matching order; the keep manifest lists original indices in output order).
+ * kept experts' weights and router rows are cut from the original checkpoint
+ * in the same order; the manifest lists the original indices in the order of
+ * the pruned layer).
  *
  *   dst[j] = src[kept_idx[j]]     for j < keep, whole blocks of
  *                                 bytes_per_expert bytes

@@ -3,11 +3,13 @@
 Test infrastructure (see the package docstring).
 
 Source: Qwen3.8-Flash-Next-AWQ-g32 card.
-* "Checkpoint": standard asymmetric AWQ W4A16, group size 32, integer zero
-  point, GEMM packing; gate_proj / up_proj / down_proj of every routed expert
-  are quantised; expert scales are FP16.
-* "Calibration": scales are rounded to FP16 before the codes are chosen, and
-  a code is clip(round(w / scale + zero), 0, 15).
+* "Checkpoint": 4-bit weights with 16-bit activations, asymmetric (an
+  integer zero point per group), groups of 32 inputs, the AWQ GEMM packing;
+  all three projections of every routed expert are quantised, with FP16
+  scales.
+* "Calibration": each scale is first rounded to FP16, then the code of a
+  weight is its rounded quotient by the scale plus the zero point, clipped
+  to 0..15.
 
 The inverse of that code rule is w = (q - z) * s; the kernel produces it in
 FP16, so the oracle's dequantised weight is fp16_rn((q - z) * s), computed

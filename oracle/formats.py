@@ -9,12 +9,12 @@ Formats and where the pages name them
 -------------------------------------
 * BF16 -- expert, router and shared-expert weights of the base and RAZOR
   checkpoints (RAZOR-65B model card, property table "Weight dtype").
-* FP16 -- AWQ expert scales and the FP16 "compensation carriers" (router and
-  shared expert) of the AWQ g32 card, sections "Checkpoint" and the paragraph
-  on compensation carriers; activations of that card's FP16 compute.
+* FP16 -- AWQ expert scales and the non-routed tensors stored in FP16
+  (router and shared expert) of the AWQ g32 card, section "Checkpoint" and
+  its paragraph on those tensors; activations of that card's FP16 compute.
 * FP8 E4M3 (the finite-only "FN" variant, max 448) -- NVFP4 block scales
-  (NVFP4 card, component table: "group 16, FP8 block scales").
-* FP4 E2M1 -- NVFP4 element codes (same table: "NVFP4 W4A4").
+  (NVFP4 card, component table: one FP8 scale per group of 16).
+* FP4 E2M1 -- NVFP4 element codes (same table: 4-bit weights and activations).
 """
 
 from __future__ import annotations

@@ -14,7 +14,7 @@ Sources (page title, then the section or table entry):
 * Qwen3.8-Flash-Next-AWQ-g32 card, "Checkpoint": the expert projections are
   gate_proj, up_proj and down_proj.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * weights are stored out x in (row j of w_gate is output feature j);
 * the synthetic router bias is added to the logits before the softmax;
 * ties in the expert order go to the lower expert index;
@@ -139,8 +139,9 @@ def combine(f_rows: np.ndarray, slot_row: np.ndarray, w: np.ndarray, shared: Opt
 
 
 def rmsnorm(x: np.ndarray, w: np.ndarray, eps: float = 1e-6) -> np.ndarray:
-    """Pre-norm RMSNorm with a (1 + w) gain (architecture fact sheet:
-    "RMSNorm (1+w gain)", pre-norm, epsilon 1e-06): the MoE block's input is
+    """Pre-norm RMSNorm with a (1 + w) gain (architecture fact sheet,
+    normalisation entries: gain 1 + w, before the block, epsilon 1e-6): the
+    MoE block's input is
     x / sqrt(mean(x^2) + eps) * (1 + w) over the hidden dimension.
     x [T, H], w [H] -> [T, H]."""
     x = np.asarray(x, np.float64)

@@ -3,11 +3,12 @@ one FP8 E4M3 scale per group and one FP32 global scale per tensor.
 
 Test infrastructure (see the package docstring).
 
-Source: Qwen3.8-Flash-Next-RAZOR-96B-A6B-NVFP4 card, component table:
-"Routed experts: NVFP4 W4A4 (group 16, FP8 block scales, FP32 global
-scales)"; the shared expert and router stay BF16.  The card names the
+Source: Qwen3.8-Flash-Next-RAZOR-96B-A6B-NVFP4 card, component table: the
+routed experts use NVFP4 for weights and activations (FP4 values in groups
+of 16, an FP8 scale per group, an FP32 scale per tensor); the shared expert
+and router stay BF16.  The card names the
 format but not the scale recipe; this oracle takes the plainest reading that
-makes every scale a decode-direction multiplier (listed in the design doc):
+makes every scale a decode-direction multiplier (a reading of the pages, which leave it open):
 
   s_g  = amax(|V|) / (6 * 448)                  float32, per tensor
   s_b  = e4m3_rn_sat(amax(|V_block|) / (6*s_g))   per 16 elements along K

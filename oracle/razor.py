@@ -5,20 +5,20 @@ Test infrastructure (see the package docstring).
 Source: Qwen3.8-Flash-Next-RAZOR-65B-A6B-E256of512 card (and the copy of the
 same text for the 384-expert budget on the NVFP4 card), section "Selection
 and calibration":
-* an expert's score is the RMS of the change of the layer's local output
-  when that selected expert is removed and the router promotes its
-  highest-ranked unselected expert;
-* the RMS is conditional on the calibration tokens routed to the expert (not
-  a corpus sum, not an arithmetic mean);
-* the highest-scoring 256 (or 384) experts of each layer are kept;
-* the statistics are additive: existing ones were reused and recombined.
+* an expert is scored by how much the layer's local output moves when that
+  expert is taken out of a token's selection and the router's best
+  unselected expert takes its place, aggregated as a root mean square;
+* the mean runs only over the calibration tokens that selected the expert
+  (neither a sum over the corpus nor a plain average);
+* each layer keeps its 256 (or 384) best-scoring experts;
+* the statistics add up across rows and runs (earlier ones were reused).
 The opening paragraphs add that the kept experts' weights and router rows are
-sliced "in matching order" and that the keep manifest lists original expert
-indices in output order.  The MTP item of the same section keeps the MTP
+cut from the original checkpoint in the same order, and that the keep
+manifest lists the original expert indices in the pruned layer's order.  The MTP item of the same section keeps the MTP
 layer's experts by the L2 norm of their original router rows
 (mtp_policy=router_norm), because the text calibration never runs that layer.
 
-Readings (listed in DESIGN.md): "local output" is the MoE block output, so
+Readings where the pages are silent: "local output" is the MoE block output, so
 the shared expert cancels; the change is measured with the L2 norm over the
 hidden dimension and the per-expert score is sqrt(sum ||delta||^2 / count);
 count[e] counts tokens whose selected set contains e (the promoted expert
