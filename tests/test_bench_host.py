@@ -1,0 +1,35 @@
+"""Host-side consistency of bench.py, without a GPU: every workload names a
+synthetic layer that exists, pruned workloads keep fewer experts than their
+layer has, the algorithmic FLOP count matches the expert maths, and the
+committed launch-list summary of the default workload is found (its DRAM
+traffic is reported while the kernel sources match the recorded hash, and
+null after a change)."""
+
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from bit_expert_gemm_b200 import synth  # noqa: E402
+
+
+def test_workload_table():
+    for name, (wname, T, kind) in bench.WORKLOADS.items():
+        wl = synth.WORKLOADS[wname]
+        assert kind in ("forward", "refill"), name
+        assert T >= 1 and wl.H % 64 == 0 and wl.I % 64 == 0, name
+    for name, keep in bench.PRUNED.items():
+        wname, T, kind = bench.WORKLOADS[name]
+        assert kind == "forward" and 0 < keep < synth.WORKLOADS[wname].E
+    assert bench.WORKLOADS["bf16_prefill"] == ("bf16", 8192, "forward")
+
+
+def test_expert_flops_and_default_traffic():
+    # gate, up and down of one routed row: 2 * 3 * H * I FLOP
+    assert bench.expert_flops(81920, 2048, 640) == 2.0 * 81920 * 3 * 2048 * 640
+    traffic, src = bench.measured_traffic("bf16_prefill")
+    assert src is not None and "moe_layer_bf16_prefill_t8192.md" in src
+    assert traffic is None or traffic > 2e9  # the expert call moves at least the touched experts' 2.1 GB
+    assert bench.measured_traffic("no_such_workload") == (None, None)
