@@ -29,9 +29,9 @@
 // rows; down quarter q of tile n is rows 128n + 32q...  Eight lanes share a
 // row (16 bytes of codes = 32 elements each per 256-element K step,
 // coalesced), each of the block's eight warps holds four rows, and the
-// eight partial sums of a row are added with three shuffles.  The item's activations (the expert's n_e <= 16
-// tokens) are staged in shared memory as signed 2*e2m1 bytes plus FP32 group
-// scales once per expert.
+// eight partial sums of a row are added with three shuffles.  The item's
+// activations (the expert's n_e <= 16 tokens) are staged in shared memory as
+// signed 2*e2m1 bytes plus FP32 group scales once per expert.
 #include <algorithm>
 
 #include "common.cuh"
@@ -76,7 +76,7 @@ struct Fp4DecArgs {
   const int32_t* offsets;   // [E+1]
   const int32_t* row_token; // [rows] token of each permuted row
   const int32_t* active;    // [1 + E]: count, then the experts with rows
-  int E, T, rows, H, I;
+  int E, T, H, I;
   // activations
   const uint8_t* xq;        // [T, H/2] codes of x (GEMM1)
   const uint8_t* xsf;       // [T, H/16] E4M3 scales of x
@@ -90,7 +90,6 @@ struct Fp4DecArgs {
   const float* gsw;         // [E, 2] gate/up or [E] down
   void* f;                  // [rows, H] GEMM2 output
   int f_fp32;
-  int* status;
 };
 
 // ---------------------------------------------------------------------------
@@ -392,7 +391,6 @@ int nvfp4_decode(const void* x, const int32_t* row_token, const int32_t* offsets
   a.active = active;
   a.E = E;
   a.T = T;
-  a.rows = rows;
   a.H = H;
   a.I = I;
   a.xq = xq;
@@ -401,7 +399,6 @@ int nvfp4_decode(const void* x, const int32_t* row_token, const int32_t* offsets
   a.amax = amax;
   a.gs_in = act_gs_in;
   a.h = reinterpret_cast<__nv_bfloat16*>(h);
-  a.status = device_status_ptr();
   k_fp4_prep<__nv_bfloat16><<<1, 1024, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), a, xq, xsf, active);
   MOE_CHECK_CUDA(cudaGetLastError());
   // work items: at most min(E, rows) experts x tiles x 4 slices; up to 8
