@@ -43,6 +43,7 @@ _SIGS = {
     "moe_abi_version": (_I, []),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_device_status": (_I, [_I, _P]),
+    "moe_selftest_bounded_wait": (_I, [_I, _P, _P]),
     "moe_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "moe_route_topk": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "moe_route_permute": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -139,6 +140,17 @@ def abi_version() -> int:
 
 def moe_device_status(clear: bool = True, stream=None) -> int:
     return load().moe_device_status(int(clear), _stream(stream))
+
+
+def moe_selftest_bounded_wait(limit_us: int, result: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Launches the bounded-wait self-test (a wait that nothing completes runs
+    out after limit_us); returns result [2] int32 (1 = that role's wait gave
+    up).  Read moe_device_status afterwards: MOE_ERR_TIMEOUT."""
+    if result is None:
+        result = torch.zeros(2, dtype=torch.int32, device="cuda")
+    _need(result, torch.int32, "result")
+    _call("moe_selftest_bounded_wait", int(limit_us), _p(result), _stream(stream))
+    return result
 
 
 def moe_workspace_size(op: int, T: int, H: int, E: int, k_slots: int, I: int) -> int:

@@ -166,7 +166,9 @@ int combine(const void* f, int f_fp32, const int32_t* slot_row, int ks, const fl
 //   delta_j = (U - p_j f_j + p_r f_r) / (Z - p_j + p_r) - y.
 // ||delta_j||^2 is written to d2[slot_row[t, j]] (the permuted row of the
 // assignment), the promoted slot's row gets -1; a second kernel sums each
-// expert's rows in a fixed order.
+// expert's rows in a fixed order.  A slot whose row is -1 (the permutation
+// skipped an out-of-range expert id and recorded it in the status word)
+// contributes zeros and writes nothing.
 // ---------------------------------------------------------------------------
 constexpr int kRefillMaxSlots = 16;
 
@@ -198,7 +200,14 @@ __global__ void __launch_bounds__(256) k_refill(const void* __restrict__ f, cons
     float fv[kRefillMaxSlots][4];
 #pragma unroll
     for (int j = 0; j < kRefillMaxSlots; ++j)
-      if (j < ks) load4<T16, F32>(f, size_t(row_sh[j]), H, c, fv[j]);
+      if (j < ks) {
+        if (row_sh[j] >= 0) {
+          load4<T16, F32>(f, size_t(row_sh[j]), H, c, fv[j]);
+        } else {  // an out-of-range expert id (recorded by the permutation): no row
+#pragma unroll
+          for (int i = 0; i < 4; ++i) fv[j][i] = 0.f;
+        }
+      }
     float U[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < kRefillMaxSlots - 1; ++j)
@@ -248,7 +257,7 @@ __global__ void __launch_bounds__(256) k_refill(const void* __restrict__ f, cons
     }
   }
   __syncthreads();
-  if (threadIdx.x < ks) {
+  if (threadIdx.x < ks && row_sh[threadIdx.x] >= 0) {
     const int j = threadIdx.x;
     if (j < k) {
       double s = 0.0;

@@ -15,6 +15,8 @@
 // start at zero (the expert bitmask) on the call's stream.  Two calls whose
 // kernels overlap on the GPU (different streams, no ordering between them)
 // race on the array.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moe {
@@ -34,7 +36,12 @@ constexpr size_t kNoAllocScratchBytes = size_t(kNoAllocMaxMaskWords) * 4 * 2 + 1
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+// Per-device cache of the array's device address.  Host threads may race to
+// fill an entry; they all store the same value, and the atomic makes that
+// race well defined.  The cache assumes the device's primary context lives
+// as long as the process: after cudaDeviceReset the library's module is
+// loaded again, possibly at another address, and the cached entry is stale.
+std::atomic<void*> g_scratch_ptr[kMaxDevices];
 
 // Device address of the scratch array on the current device.  The array's
 // name in host code is only a host-side stand-in; its device address comes
@@ -44,12 +51,13 @@ int scratch_address(void** out) {
   MOE_CHECK_CUDA(cudaGetDevice(&dev));
   MOE_REQUIRE(dev >= 0 && dev < kMaxDevices, MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: device %d >= %d", dev,
               kMaxDevices);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
     MOE_CHECK_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-    g_scratch_ptr[dev] = p;
+    MOE_REQUIRE(p != nullptr, MOE_ERR_CUDA, "moe_permute_noalloc: no device address for the scratch array");
+    g_scratch_ptr[dev].store(p, std::memory_order_release);
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return MOE_OK;
 }
 

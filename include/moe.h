@@ -100,6 +100,23 @@ MOE_API const char* moe_last_error(void);
  * it when `clear` is non-zero.  This is the only call that synchronises. */
 MOE_API int moe_device_status(int clear, void* stream);
 
+/* Self-test of the bounded device-side waits (failure handling; the pages
+ * have no counterpart).  Launches one CTA that does what a TMA / tcgen05
+ * kernel of this library does when a wait never completes: one role starts
+ * a bulk copy, then waits on an mbarrier that nothing completes, with a
+ * limit of limit_us microseconds; the wait runs out, records MOE_ERR_TIMEOUT
+ * in the device status word and raises the CTA's abort flag, and the role
+ * waits (bounded) for its copy to land.  A second role waiting on the same
+ * barrier with a 100x longer limit stops on the abort flag, drains the
+ * tensor core, and the CTA frees its tensor memory and exits.  result [2]
+ * int32 on the device: result[0] = 1 if the first role's wait gave up,
+ * result[1] = 1 if the second role's did.  The launch ends about 64 ms
+ * after limit_us at most (the flags are polled every 64 suspended tries).
+ * Clear the status word (moe_device_status(1, ...)) before the call and read
+ * it after; the GPU context stays usable.  Limits: 100 <= limit_us <=
+ * 1000000, else MOE_ERR_UNSUPPORTED with nothing launched. */
+MOE_API int moe_selftest_bounded_wait(int limit_us, int32_t* result, void* stream);
+
 /* Bytes of workspace that operation `op` needs for the given sizes
  * (T tokens, hidden size H, E experts, k_slots selected slots per token,
  * intermediate width I).  Returns 0 for an unknown op.  The result is an
@@ -171,7 +188,10 @@ MOE_API int moe_route_permute(const void* x, int T, int H, const void* w_router,
  * T = 32768 tokens); larger batches are rejected with MOE_ERR_UNSUPPORTED
  * (use moe_permute with a workspace).  The first call on a device looks up
  * the array's device address with that device current; make that first call
- * before any stream capture.  All calls on a device share the array and it
+ * before any stream capture.  The address is cached per device for the life
+ * of the process (host threads may make the first call concurrently): a
+ * process that resets a device (cudaDeviceReset) must not call this on that
+ * device afterwards.  All calls on a device share the array and it
  * keeps the last call's contents (the part that must start at zero is
  * cleared on the call's stream); calls whose work overlaps on the GPU, e.g.
  * on unordered streams, race on it.

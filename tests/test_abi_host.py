@@ -69,6 +69,10 @@ def test_calls_reject_null_pointers_and_bad_sizes():
     assert _code("razor_select", None, None, 0, 0, None, None, None, None) == abi.MOE_ERR_UNSUPPORTED
     assert _code("moe_nvfp4_quantize", None, 1, 4, 24, 0, None, None, None, None, None, 0, None) == \
         abi.MOE_ERR_UNSUPPORTED
+    # the bounded-wait self-test checks its limit and output before launching
+    assert _code("moe_selftest_bounded_wait", 50, ctypes.c_void_p(256), None) == abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_selftest_bounded_wait", 2_000_000, ctypes.c_void_p(256), None) == abi.MOE_ERR_UNSUPPORTED
+    assert _code("moe_selftest_bounded_wait", 2000, None, None) == abi.MOE_ERR_INVALID_ARG
 
 
 def test_zero_sized_calls_are_no_ops():

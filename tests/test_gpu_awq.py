@@ -11,7 +11,7 @@ import torch
 
 from bit_expert_gemm_b200 import MoELayer, abi, synth
 from oracle import awq, moe
-from tests.helpers import f64, rel_err
+from tests.helpers import f64, rel_err, tile_edge_sample
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -35,15 +35,18 @@ def test_awq_dequant_bit_exact(E, K, N):
         assert np.array_equal(g, r)
 
 
-def _awq_expert_fn(w, I):
-    cache = {}
+def _awq_expert_fn(w, I, cache: bool = True):
+    store = {}
     host = {k: _np(w[k]) for k in ("qw_gu", "qz_gu", "sc_gu", "qw_d", "qz_d", "sc_d")}
 
     def ew(e):
-        if e not in cache:
-            cache[e] = awq.expert_weights_out_in(host["qw_gu"], host["qz_gu"], host["sc_gu"], host["qw_d"],
-                                                 host["qz_d"], host["sc_d"], e, I)
-        return cache[e]
+        if e in store:
+            return store[e]
+        out = awq.expert_weights_out_in(host["qw_gu"], host["qz_gu"], host["sc_gu"], host["qw_d"], host["qz_d"],
+                                        host["sc_d"], e, I)
+        if cache:
+            store[e] = out
+        return out
 
     return ew
 
@@ -177,15 +180,23 @@ def test_awq_layer_decode(awq_layer, T):
 
 
 def test_awq_layer_prefill_sampled(awq_layer):
+    """Full AWQ prefill batch (T=8192) as the bench runs it; at least 1024
+    tokens recomputed by the oracle: every token with a row in the first or
+    last 128-row tile of the three most-loaded experts, plus random ones."""
     wl, w = awq_layer
     T = wl.T_prefill
     layer = MoELayer(w, wl.k, "awq_g32", T_max=T)
     x = synth.make_tokens(wl, T, seed=0, device=DEV)
     y = layer.forward(x)
     torch.cuda.synchronize()
-    sample = np.concatenate([np.random.default_rng(1).choice(T, 16, replace=False), [0, T - 1]])
-    ref = _oracle(wl, w, x[torch.as_tensor(sample, device=DEV)])
+    r_all = moe.route(f64(x), f64(w["w_router"]), f64(w["bias"]), wl.k)
+    sample = tile_edge_sample(T, moe.permute(r_all["idx"], wl.E), n_total=1024, seed=1)
+    assert len(sample) >= 1024
+    sh = f64(w["w_sh_gate_up"])
+    ref = moe.moe_layer(f64(x)[sample], f64(w["w_router"]), f64(w["bias"]), wl.k,
+                        _awq_expert_fn(w, wl.I, cache=False), (sh[:wl.I_sh], sh[wl.I_sh:], f64(w["w_sh_down"])))
     ok = ref["route"]["margin"] > 1e-3
+    assert ok.mean() > 0.9
     err = rel_err(f64(y)[sample][ok], ref["y"][ok])
     assert err <= TOL_4BIT, err
     assert abi.moe_device_status() == 0

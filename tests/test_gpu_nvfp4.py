@@ -13,7 +13,7 @@ import torch
 from bit_expert_gemm_b200 import MoELayer, abi, synth
 from bit_expert_gemm_b200.layer import prepare_nvfp4_weights
 from oracle import moe, nvfp4
-from tests.helpers import f64, rel_err, shared_fn
+from tests.helpers import f64, nvfp4_oracle_bank, rel_err, shared_fn
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -152,3 +152,44 @@ def test_nvfp4_layer_prefill_sampled_static_scales():
     err = rel_err(f64(y)[sample][ok], yref[ok])
     assert err <= TOL_4BIT, err
     assert abi.moe_device_status() == 0
+
+
+@pytest.mark.slow
+def test_nvfp4_layer_prefill_full_dynamic_scales():
+    """The NVFP4 workload at full size with the layer's own dynamic
+    activation scales, exactly as the bench runs it (E=256, T=16384, top-10).
+    The float64 oracle quantises the weights itself, takes s_x from all of x
+    and s_h from the whole BF16-rounded intermediate of all 163,840 permuted
+    rows, and computes every token's output; x's global scale must match bit
+    for bit, h's within 1e-2 (its amax is one FP32 sum per element, summed in
+    another order), and every decided token's output within 5e-2."""
+    wl = synth.WORKLOADS["nvfp4"]
+    T = wl.T_prefill
+    w = prepare_nvfp4_weights(synth.make_weights(wl, seed=0, device=DEV))
+    x = synth.make_tokens(wl, T, seed=0, device=DEV)
+    layer = MoELayer(w, wl.k, "nvfp4", T_max=T)
+    y = layer.forward(x).clone()
+    # the same expert call on the layer's own routing, now also reporting the
+    # activation scales it derived (the layer's call does not ask for them)
+    rows = T * wl.k
+    gs_out = torch.empty(2, dtype=torch.float32, device=DEV)
+    f2 = abi.moe_grouped_swiglu_nvfp4_prepacked(x, layer.row_token[:rows], layer.offsets, rows, w["w_gu"],
+                                                w["sfp_gu"], w["gs_gu"], w["w_d"], w["sfp_d"], w["gs_d"],
+                                                act_gs_out=gs_out, out_fp32=layer.f.dtype == torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(f2, layer.f[:rows])
+    assert abi.moe_device_status() == 0
+    xs = f64(x)
+    r = moe.route(xs, f64(w["w_router"]), f64(w["bias"]), wl.k)
+    perm = moe.permute(r["idx"], wl.E)
+    deq, _ = nvfp4_oracle_bank(w, wl.I, np.nonzero(perm["counts"])[0])
+    f, _, (s_x, s_h) = nvfp4.routed_outputs_w4a4(xs, perm, deq)
+    g = _np(gs_out)
+    assert g[0] == s_x
+    assert abs(g[1] / s_h - 1) < 1e-2, (g[1], s_h)
+    sh, _ = moe.swiglu_expert(xs, *shared_fn(w))
+    yref = moe.combine(f, perm["slot_row"], r["w"], sh)
+    ok = r["margin"] > 1e-3
+    assert ok.sum() >= 1024
+    err = rel_err(f64(y)[ok], yref[ok])
+    assert err <= TOL_4BIT, err

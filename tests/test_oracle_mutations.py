@@ -140,6 +140,25 @@ def _quantize_4sg(v, s_g=None):
     return f32_to_e2m1(q).reshape(rows, K), sb_code, s_g
 
 
+def _awq_halves_swapped(qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d, e, I, mode="fp16"):
+    wgu = awq.dequant(qw_gu[e], qz_gu[e], sc_gu[e], mode)
+    wd = awq.dequant(qw_d[e], qz_d[e], sc_d[e], mode)
+    return wgu[:, I:].T, wgu[:, :I].T, wd.T  # up taken as gate and gate as up
+
+
+def _nvfp4_shared_gate_up_scale(w_gate_up, w_down):
+    E, I2, _ = w_gate_up.shape
+    I = I2 // 2
+    raw, deq = {}, {}
+    for e in range(E):
+        c, sb, g = nvfp4.quantize(w_gate_up[e].astype(np.float32))  # gate and up as one tensor
+        raw[(e, "gate")], raw[(e, "up")] = (c[:I], sb[:I], g), (c[I:], sb[I:], g)
+        raw[(e, "down")] = nvfp4.quantize(w_down[e].astype(np.float32))
+        for name in ("gate", "up", "down"):
+            deq[(e, name)] = nvfp4.dequant(*raw[(e, name)])
+    return (lambda e: (deq[(e, "gate")], deq[(e, "up")], deq[(e, "down")])), raw
+
+
 MUTATIONS = [
     ("silu sign", lambda mp: mp.setattr(moe, "silu", _silu_sign),
      [tm.test_softmax_and_silu_vs_torch, tm.test_single_expert_layer_is_textbook_swiglu]),
@@ -180,6 +199,11 @@ MUTATIONS = [
      [tq.test_awq_dequant_zero_at_zero_point_and_vs_torch_half]),
     ("AWQ BF16 mode without scale rounding", lambda mp: mp.setattr(awq, "dequant", _dequant_bf16_unrounded_scale(awq.dequant)),
      [tq.test_awq_dequant_bf16_mode_vs_torch_bfloat16]),
+    ("AWQ gate and up halves swapped", lambda mp: mp.setattr(awq, "expert_weights_out_in", _awq_halves_swapped),
+     [tq.test_awq_expert_bank_split_and_orientation]),
+    ("NVFP4 one global scale shared by gate and up",
+     lambda mp: mp.setattr(nvfp4, "quantize_expert_weights", _nvfp4_shared_gate_up_scale),
+     [tq.test_nvfp4_expert_weights_one_global_scale_per_projection]),
     ("NVFP4 block scale from 4 s_g", lambda mp: mp.setattr(nvfp4, "quantize", _quantize_4sg),
      [tq.test_nvfp4_grid_values_round_trip_exactly, tq.test_nvfp4_error_bound_and_block_max]),
 ]

@@ -208,3 +208,84 @@ def test_bf16_integer_bit_patterns_used_by_the_awq_bf16_mode():
     assert np.array_equal(formats.bf16_to_f64(formats.f32_to_bf16(d.astype(np.float32))), d)
     # the FP16 pattern of the FP16 mode: 0x6400 | q is 1024 + q
     assert np.array_equal(formats.f16_to_f64((np.uint16(0x6400) | q).view(np.float16)), 1024.0 + q)
+
+
+def _hand_bank(E, H, I):
+    """Hand-built integer expert weights, out x in: gate [E, I, H], up
+    [E, I, H], down [E, H, I], every entry in -8..7 and the three
+    projections different from one another (and not symmetric), so that a
+    swapped half, a missing transpose or a wrong expert index changes the
+    result."""
+    i = np.arange(I)[:, None]
+    h = np.arange(H)[None, :]
+    e = np.arange(E)[:, None, None]
+    gate = ((3 * i + h + 5 * e) % 16) - 8
+    up = 7 - ((i + 5 * h + 3 * e) % 16)
+    down = ((7 * h.T + 3 * i.T + e) % 16) - 8  # [E, H, I]
+    return gate.astype(np.int64), up.astype(np.int64), down.astype(np.int64)
+
+
+def test_awq_expert_bank_split_and_orientation():
+    """expert_weights_out_in against the library's documented AWQ layout,
+    built by hand: the stored gate/up projection is input-major [H, 2I] with
+    output columns 0..I-1 the gate and I..2I-1 the up projection; down is
+    stored [I, H].  Zero points 8 and power-of-two scales (1 for gate/up
+    groups, 1/2 for down) make every dequantised weight an exact small
+    number, so the oracle must return exactly the hand-built matrices."""
+    E, H, I = 3, 64, 32
+    gate, up, down = _hand_bank(E, H, I)
+    codes_gu = np.concatenate([gate, up], axis=1).transpose(0, 2, 1) + 8  # [E, H, 2I] input-major
+    codes_d = down.transpose(0, 2, 1) + 8  # [E, I, H]
+    qw_gu = np.stack([awq.pack_nibbles(c) for c in codes_gu])
+    qw_d = np.stack([awq.pack_nibbles(c) for c in codes_d])
+    qz_gu = np.stack([awq.pack_nibbles(np.full((H // 32, 2 * I), 8)) for _ in range(E)])
+    qz_d = np.stack([awq.pack_nibbles(np.full((I // 32, H), 8)) for _ in range(E)])
+    sc_gu = np.ones((E, H // 32, 2 * I), np.float16)
+    sc_d = np.full((E, I // 32, H), 0.5, np.float16)
+    for e in range(E):
+        wg, wu, wd = awq.expert_weights_out_in(qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d, e, I)
+        assert wg.shape == (I, H) and wu.shape == (I, H) and wd.shape == (H, I)
+        assert np.array_equal(wg, gate[e])
+        assert np.array_equal(wu, up[e])
+        assert np.array_equal(wd, 0.5 * down[e])
+
+
+def test_nvfp4_expert_weights_one_global_scale_per_projection():
+    """quantize_expert_weights: gate, up and down of every expert are three
+    tensors, each with the global scale amax / (6 * 448) of its own values
+    (one FP32 scale per tensor), and the dequantised gate / up / down come
+    back in out x in orientation close to their own source rows."""
+    rng = np.random.default_rng(11)
+    E, H, I = 2, 64, 32
+    amax = {}
+    gu = np.empty((E, 2 * I, H))
+    wd = np.empty((E, H, I))
+    for e in range(E):
+        # each tensor's largest magnitude sits at a known place, with a known value
+        for name, shape, peak in (("gate", (I, H), 0.5 * (e + 1)), ("up", (I, H), 3.0 * (e + 1)),
+                                  ("down", (H, I), 0.125 * (e + 2))):
+            m = rng.uniform(-0.9, 0.9, shape) * peak
+            m[1, 2] = -peak
+            amax[(e, name)] = peak
+            if name == "gate":
+                gu[e, :I] = m
+            elif name == "up":
+                gu[e, I:] = m
+            else:
+                wd[e] = m
+    gu = gu.astype(np.float32).astype(np.float64)
+    wd = wd.astype(np.float32).astype(np.float64)
+    deq, raw = nvfp4.quantize_expert_weights(gu, wd)
+    for e in range(E):
+        scales = []
+        for name in ("gate", "up", "down"):
+            s_g = raw[(e, name)][2]
+            assert s_g == np.float32(np.float32(amax[(e, name)]) / np.float32(2688.0)), (e, name)
+            scales.append(s_g)
+        assert len(set(scales)) == 3
+        wg, wu, wdd = deq(e)
+        assert wg.shape == (I, H) and wu.shape == (I, H) and wdd.shape == (H, I)
+        for got, src, name in ((wg, gu[e, :I], "gate"), (wu, gu[e, I:], "up"), (wdd, wd[e], "down")):
+            # a 16-element group keeps its largest value within one E2M1 step and
+            # the E4M3 scale rounding: far below the gap between the tensors' ranges
+            assert np.max(np.abs(got - src)) <= 0.25 * amax[(e, name)], name
