@@ -84,8 +84,13 @@ WORKLOADS = {
     "bf16_razor256_prefill": ("bf16", 8192, "forward"),
     "bf16_razor384_prefill": ("bf16", 8192, "forward"),
     "bf16_razor256_decode_t1": ("bf16", 1, "forward"),
+    # the BF16 layer with its pre-MoE RMSNorm (gain 1 + w, eps 1e-6) and a
+    # shared-expert gate, both inside the routing call
+    "bf16_norm_prefill": ("bf16", 8192, "forward"),
+    "bf16_norm_decode_t1": ("bf16", 1, "forward"),
 }
 PRUNED = {"bf16_razor256_prefill": 256, "bf16_razor384_prefill": 384, "bf16_razor256_decode_t1": 256}
+WITH_NORM = {"bf16_norm_prefill", "bf16_norm_decode_t1"}
 CALIBRATION_T = 32768
 
 
@@ -252,7 +257,10 @@ def oracle_tokens_per_s(wl, w, x: torch.Tensor, n_tokens: int, kind: str):
     wr, b = to64(w["w_router"]), to64(w["bias"])
     sh = to64(w["w_sh_gate_up"])
     shared = (sh[: wl.I_sh], sh[wl.I_sh:], to64(w["w_sh_down"]))
+    gate_w = to64(w["w_sh_gate"]) if "w_sh_gate" in w else None
     t0 = time.perf_counter()
+    if "w_norm" in w:
+        xs = moe.block_input(xs, to64(w["w_norm"]), 1e-6, dtype="bf16" if wl.act == "bf16" else "f16")
     if kind == "refill":
         out = moe.moe_layer(xs, wr, b, wl.k, ew, shared, extra=1)
         r = out["route"]
@@ -266,7 +274,7 @@ def oracle_tokens_per_s(wl, w, x: torch.Tensor, n_tokens: int, kind: str):
         f, _, _ = nvfp4.routed_outputs_w4a4(xs, perm, ew)
         moe.combine(f, perm["slot_row"], r["w"], moe.swiglu_expert(xs, *shared)[0])
     else:
-        moe.moe_layer(xs, wr, b, wl.k, ew, shared)
+        moe.moe_layer(xs, wr, b, wl.k, ew, shared, shared_gate_w=gate_w)
     dt = time.perf_counter() - t0
     return n_tokens / dt, dt
 
@@ -408,6 +416,12 @@ def bench_workload(args, dist: Dist, workload: str, with_e2e: bool = True, with_
 
         def layer_weights(seed):
             return razor_pruned_weights(wl_full, seed, keep, dev)
+    elif workload in WITH_NORM:
+        def layer_weights(seed):
+            w = synth.make_weights(wl, seed=seed, device=dev)
+            w["w_norm"] = synth.make_norm_weight(wl, seed, device=dev)
+            w["w_sh_gate"] = synth.make_shared_gate(wl, seed, device=dev)
+            return w
     else:
         def layer_weights(seed):
             return synth.make_weights(wl, seed=seed, device=dev)
@@ -442,10 +456,10 @@ def bench_workload(args, dist: Dist, workload: str, with_e2e: bool = True, with_
     stream = torch.cuda.current_stream()
 
     def step(lay, x, ev=None):
-        lay.route(x)
+        xin = lay.route(x)
         if ev:
             ev[0].record()
-        f, sh = lay.experts_and_shared(x)
+        f, sh = lay.experts_and_shared(xin)
         if ev:
             ev[1].record()
         if kind == "refill":

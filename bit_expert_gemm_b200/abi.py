@@ -47,6 +47,8 @@ _SIGS = {
     "moe_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "moe_route_topk": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "moe_route_permute": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_norm_route_permute": (_I, [_P, _I, _I, _P, ctypes.c_float, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                                    _P, _P, _P, _P, _SZ, _P]),
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_grouped_swiglu_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _SZ, _P]),
@@ -210,6 +212,49 @@ def moe_route_permute(x, w_router, bias, k: int, extra: int = 0, topk_idx=None, 
           _p(topk_w), _p(topk_logit), _p(expert_offsets), _p(row_token), _p(slot_row), _p(ws), ws.numel(),
           _stream(stream))
     return topk_idx, topk_w, topk_logit, expert_offsets, row_token, slot_row
+
+
+def moe_norm_route_permute(x, norm_w, w_router, bias, k: int, extra: int = 0, eps: float = 1e-6,
+                           w_shared_gate=None, x_norm=None, shared_gate=None, topk_idx=None, topk_w=None,
+                           topk_logit=None, expert_offsets=None, row_token=None, slot_row=None, ws=None, stream=None):
+    """Pre-MoE RMSNorm (gain 1 + norm_w) into x_norm, the shared-expert gate
+    when w_shared_gate is given, and moe_route_permute of x_norm, in one
+    call.  Returns (x_norm, shared_gate or None, topk_idx, topk_w,
+    topk_logit, expert_offsets, row_token, slot_row)."""
+    T, H = x.shape
+    E = w_router.shape[0]
+    ks = k + extra
+    dev = x.device
+    if norm_w.dtype != x.dtype or tuple(norm_w.shape) != (H,):
+        raise ValueError("moe_norm_route_permute: norm_w must be [H] of x's dtype")
+    if w_shared_gate is not None and (w_shared_gate.dtype != x.dtype or tuple(w_shared_gate.shape) != (H,)):
+        raise ValueError("moe_norm_route_permute: w_shared_gate must be [H] of x's dtype")
+    if x_norm is None:
+        x_norm = torch.empty_like(x)
+    if w_shared_gate is not None and shared_gate is None:
+        shared_gate = torch.empty((T,), dtype=torch.float32, device=dev)
+    if w_shared_gate is None:
+        shared_gate = None
+    if topk_idx is None:
+        topk_idx = torch.empty((T, ks), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if topk_logit is None:
+        topk_logit = torch.empty((T, ks), dtype=torch.float32, device=dev)
+    if expert_offsets is None:
+        expert_offsets = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    if row_token is None:
+        row_token = torch.empty((T * ks,), dtype=torch.int32, device=dev)
+    if slot_row is None:
+        slot_row = torch.empty((T, ks), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(MOE_OP_ROUTE_PERMUTE, T, H, E, ks, 0, dev)
+    if bias is not None:
+        _need(bias, torch.float32, "bias")
+    _call("moe_norm_route_permute", _p(x), T, H, _p(norm_w), float(eps), _p(w_shared_gate), _p(w_router), _p(bias), E,
+          k, extra, _dtype_code(x), _p(x_norm), _p(shared_gate), _p(topk_idx), _p(topk_w), _p(topk_logit),
+          _p(expert_offsets), _p(row_token), _p(slot_row), _p(ws), ws.numel(), _stream(stream))
+    return x_norm, shared_gate, topk_idx, topk_w, topk_logit, expert_offsets, row_token, slot_row
 
 
 def moe_permute(topk_idx, E: int, expert_offsets=None, row_token=None, slot_row=None, ws=None, stream=None):

@@ -20,7 +20,7 @@ size_t permute_ws_bytes(int T, int E);
 size_t route_permute_ws_bytes(int T, int E);
 int route_permute(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
                   int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, int32_t* offsets,
-                  int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes, cudaStream_t stream);
+                  int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes, cudaStream_t stream, const RouteNorm* norm = nullptr);
 int permute(const int32_t* topk_idx, int T, int ks, int E, int32_t* offsets, int32_t* row_token, int32_t* slot_row,
             void* ws, size_t ws_bytes, cudaStream_t stream);
 int gather_rows(const void* x, const int32_t* row_token, int rows, int H, void* out, cudaStream_t stream);
@@ -68,7 +68,8 @@ size_t nvfp4_packed_sf_bytes(int E, int rows_per_expert, int K, int swiglu);
 int nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, int K, int swiglu, uint8_t* out,
                      cudaStream_t stream);
 int shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, float* gate, cudaStream_t stream);
-int rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, cudaStream_t stream);
+int rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, cudaStream_t stream,
+            const void* w_gate = nullptr, float* gate = nullptr);
 size_t dense_gemv_ws_bytes(int T, int I);
 bool dense_gemv_fits(int T, int H, int I);
 int dense_swiglu_gemv(const void* x, const int32_t* offsets, int T, int H, int I, const void* w_gu, const void* w_d,
@@ -347,27 +348,51 @@ int moe_permute(const int32_t* topk_idx, int T, int k_slots, int E, int32_t* exp
                  static_cast<cudaStream_t>(stream));
 }
 
+static int route_permute_entry(const char* fn, const void* x, int T, int H, const void* w_router, const float* bias,
+                               int E, int k, int extra, int dtype, int32_t* topk_idx, float* topk_w,
+                               float* topk_logit, int32_t* expert_offsets, int32_t* row_token, int32_t* slot_row,
+                               void* ws, size_t ws_bytes, void* stream, const RouteNorm* norm) {
+  MOE_REQUIRE(T >= 0 && H > 0 && E > 0, MOE_ERR_INVALID_ARG, "%s: bad sizes T=%d H=%d E=%d", fn, T, H, E);
+  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "%s: dtype %d", fn, dtype);
+  MOE_REQUIRE(extra == 0 || extra == 1, MOE_ERR_INVALID_ARG, "%s: extra must be 0 or 1", fn);
+  MOE_REQUIRE(k >= 1 && k + extra <= 16 && k + extra <= E, MOE_ERR_UNSUPPORTED,
+              "%s: need 1 <= k, k+extra <= 16 and <= E (k=%d extra=%d E=%d)", fn, k, extra, E);
+  MOE_REQUIRE(E <= 1024, MOE_ERR_UNSUPPORTED, "%s: E=%d > 1024", fn, E);
+  MOE_REQUIRE(H % 64 == 0, MOE_ERR_UNSUPPORTED, "%s: H=%d is not a multiple of 64", fn, H);
+  MOE_REQUIRE(long(T) * (k + extra) < (1l << 31), MOE_ERR_UNSUPPORTED, "%s: T*(k+extra) overflows", fn);
+  MOE_REQUIRE(expert_offsets != nullptr, MOE_ERR_INVALID_ARG, "%s: expert_offsets is null", fn);
+  if (norm) {
+    MOE_REQUIRE(norm->w && norm->x_norm, MOE_ERR_INVALID_ARG, "%s: norm_w and x_norm must not be null", fn);
+    MOE_REQUIRE((norm->gate_w == nullptr) == (norm->gate == nullptr), MOE_ERR_INVALID_ARG,
+                "%s: w_shared_gate and shared_gate_out go together", fn);
+    MOE_REQUIRE(norm->eps >= 0.f, MOE_ERR_INVALID_ARG, "%s: eps < 0", fn);
+    MOE_REQUIRE(aligned16(norm->w) && aligned16(norm->x_norm) && (!norm->gate_w || aligned16(norm->gate_w)),
+                MOE_ERR_INVALID_ARG, "%s: norm_w / x_norm / w_shared_gate not 16-byte aligned", fn);
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) return permute(topk_idx, 0, k + extra, E, expert_offsets, row_token, slot_row, ws, ws_bytes, st);
+  MOE_REQUIRE(x && w_router && topk_idx && topk_w && row_token && slot_row, MOE_ERR_INVALID_ARG, "%s: null pointer",
+              fn);
+  MOE_REQUIRE(aligned16(x) && aligned16(w_router), MOE_ERR_INVALID_ARG, "%s: x / w_router not 16-byte aligned", fn);
+  return route_permute(x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w, topk_logit, expert_offsets,
+                       row_token, slot_row, ws, ws_bytes, st, norm);
+}
+
 int moe_route_permute(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
                       int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, int32_t* expert_offsets,
                       int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes, void* stream) {
-  MOE_REQUIRE(T >= 0 && H > 0 && E > 0, MOE_ERR_INVALID_ARG, "moe_route_permute: bad sizes T=%d H=%d E=%d", T, H, E);
-  MOE_REQUIRE(dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_F16, MOE_ERR_INVALID_ARG, "moe_route_permute: dtype %d",
-              dtype);
-  MOE_REQUIRE(extra == 0 || extra == 1, MOE_ERR_INVALID_ARG, "moe_route_permute: extra must be 0 or 1");
-  MOE_REQUIRE(k >= 1 && k + extra <= 16 && k + extra <= E, MOE_ERR_UNSUPPORTED,
-              "moe_route_permute: need 1 <= k, k+extra <= 16 and <= E (k=%d extra=%d E=%d)", k, extra, E);
-  MOE_REQUIRE(E <= 1024, MOE_ERR_UNSUPPORTED, "moe_route_permute: E=%d > 1024", E);
-  MOE_REQUIRE(H % 64 == 0, MOE_ERR_UNSUPPORTED, "moe_route_permute: H=%d is not a multiple of 64", H);
-  MOE_REQUIRE(long(T) * (k + extra) < (1l << 31), MOE_ERR_UNSUPPORTED, "moe_route_permute: T*(k+extra) overflows");
-  MOE_REQUIRE(expert_offsets != nullptr, MOE_ERR_INVALID_ARG, "moe_route_permute: expert_offsets is null");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (T == 0) return permute(topk_idx, 0, k + extra, E, expert_offsets, row_token, slot_row, ws, ws_bytes, st);
-  MOE_REQUIRE(x && w_router && topk_idx && topk_w && row_token && slot_row, MOE_ERR_INVALID_ARG,
-              "moe_route_permute: null pointer");
-  MOE_REQUIRE(aligned16(x) && aligned16(w_router), MOE_ERR_INVALID_ARG,
-              "moe_route_permute: x / w_router not 16-byte aligned");
-  return route_permute(x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w, topk_logit, expert_offsets,
-                       row_token, slot_row, ws, ws_bytes, st);
+  return route_permute_entry("moe_route_permute", x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w,
+                             topk_logit, expert_offsets, row_token, slot_row, ws, ws_bytes, stream, nullptr);
+}
+
+int moe_norm_route_permute(const void* x, int T, int H, const void* norm_w, float eps, const void* w_shared_gate,
+                           const void* w_router, const float* bias, int E, int k, int extra, int dtype, void* x_norm,
+                           float* shared_gate_out, int32_t* topk_idx, float* topk_w, float* topk_logit,
+                           int32_t* expert_offsets, int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes,
+                           void* stream) {
+  RouteNorm n{norm_w, eps, w_shared_gate, x_norm, shared_gate_out};
+  return route_permute_entry("moe_norm_route_permute", x, T, H, w_router, bias, E, k, extra, dtype, topk_idx, topk_w,
+                             topk_logit, expert_offsets, row_token, slot_row, ws, ws_bytes, stream, &n);
 }
 
 int moe_grouped_swiglu_bf16(const void* x, const int32_t* row_token, const int32_t* expert_offsets, int T, int rows,

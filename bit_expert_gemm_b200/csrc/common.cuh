@@ -67,6 +67,17 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
 
+// Optional pre-MoE RMSNorm in front of the routing (moe_norm_route_permute):
+// x_norm = x / sqrt(mean x^2 + eps) * (1 + w) in 16 bits, and with gate_w
+// the shared-expert gate sigmoid(x_norm . gate_w) per token.
+struct RouteNorm {
+  const void* w;
+  float eps;
+  const void* gate_w;  // may be null (no gate)
+  void* x_norm;
+  float* gate;         // null iff gate_w is null
+};
+
 // Carves consecutive 256-byte aligned pieces out of a workspace.
 struct WsCarver {
   char* base;

@@ -22,8 +22,10 @@ constexpr int kRouterEB = 4;  // experts per block of the small-batch logits ker
 // values); warp w then takes tokens w, w + nwarps, ...: its lanes stride over
 // H in 8-value chunks, with up to 8 chunks of the token row in flight at
 // once, keeping one partial sum per expert, reduced across the warp at the
-// end.  Every thread of the block must call this.
-template <typename T16>
+// end.  Every thread of the block must call this.  X_CG: x was written
+// earlier in the same launch by other blocks (read through L2, not the
+// read-only path).
+template <typename T16, bool X_CG = false>
 __device__ void router_block_logits(const T16* __restrict__ x, const T16* __restrict__ wr,
                                     const float* __restrict__ bias, int T, int H, int E, int e0, uint4* w_sh,
                                     float* __restrict__ logits) {
@@ -46,7 +48,7 @@ __device__ void router_block_logits(const T16* __restrict__ x, const T16* __rest
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int c = c0 + 32 * u;
-        xv[u] = c < nchunk ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+        xv[u] = c < nchunk ? (X_CG ? __ldcg(xr + c) : __ldg(xr + c)) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {

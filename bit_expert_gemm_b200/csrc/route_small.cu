@@ -12,6 +12,11 @@
 //      row = offset + popcount of the expert's bits below its token.  Same
 //      order as the standalone permutation: experts ascending, tokens
 //      ascending inside an expert.
+// With a pre-MoE RMSNorm (norm_w not null) a phase 0 comes first: block b
+// normalises tokens b, b + grid, ... into x_norm (16-bit, the block's input
+// activation: x / sqrt(mean x^2 + eps) * (1 + w)) and, with a gate vector,
+// forms the shared-expert gate sigmoid(x_norm . w_gate) from the values it
+// wrote; a grid barrier follows and the logits read x_norm.
 // Values written by other blocks of this launch are read with ld.global.cg
 // (through L2) after the grid barrier.
 #include <cooperative_groups.h>
@@ -55,7 +60,81 @@ struct RouteSmallArgs {
   int32_t* row_token;
   int32_t* slot_row;
   int* status;
+  // optional pre-MoE RMSNorm (phase 0) and shared-expert gate
+  const void* norm_w;
+  float eps;
+  const void* gate_w;
+  void* x_norm;
+  float* gate;
 };
+
+// Phase 0 for token t, by the whole block: the sum of squares in FP32 (each
+// thread over 16-byte pieces, a shuffle tree per warp, then the warps' sums
+// in order), y = x * r * (1 + w) rounded to 16 bits, and the gate from the
+// rounded y.
+template <typename T16>
+__device__ void norm_token(const T16* __restrict__ x, const T16* __restrict__ w, const T16* __restrict__ wg, int t,
+                           int H, float eps, T16* __restrict__ y, float* __restrict__ gate, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + size_t(t) * H);
+  const int nv = H / 8;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < nv; c += blockDim.x) {
+    const uint4 v = __ldg(xr + c);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = Pack2<T16>::unpack(u[j]);
+      ss = fmaf(f.x, f.x, ss);
+      ss = fmaf(f.y, f.y, ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int i = 0; i < nw; ++i) tot += red[i];
+  const float r = 1.0f / sqrtf(tot / float(H) + eps);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  const uint4* gr = reinterpret_cast<const uint4*>(wg);
+  uint4* yr = reinterpret_cast<uint4*>(y + size_t(t) * H);
+  float gacc = 0.f;
+  for (int c = threadIdx.x; c < nv; c += blockDim.x) {
+    const uint4 v = __ldg(xr + c), g = __ldg(wr + c);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w}, gw[4] = {g.x, g.y, g.z, g.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = Pack2<T16>::unpack(u[j]), gg = Pack2<T16>::unpack(gw[j]);
+      o[j] = Pack2<T16>::pack(f.x * r * (1.0f + gg.x), f.y * r * (1.0f + gg.y));
+    }
+    yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    if (gate) {
+      const uint4 q = __ldg(gr + c);
+      const uint32_t qv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 a = Pack2<T16>::unpack(o[j]), b = Pack2<T16>::unpack(qv[j]);
+        gacc = fmaf(a.x, b.x, gacc);
+        gacc = fmaf(a.y, b.y, gacc);
+      }
+    }
+  }
+  if (gate) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) gacc += __shfl_xor_sync(0xffffffffu, gacc, o);
+    __syncthreads();  // every warp has read red[] above
+    if (lane == 0) red[warp] = gacc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float g = 0.f;
+      for (int i = 0; i < nw; ++i) g += red[i];
+      gate[t] = 1.0f / (1.0f + expf(-g));
+    }
+  }
+  __syncthreads();  // red[] is reused by the block's next token
+}
 
 template <typename T16, int NV>
 __global__ void __launch_bounds__(kThreads) k_route_permute_small(const RouteSmallArgs a) {
@@ -64,10 +143,23 @@ __global__ void __launch_bounds__(kThreads) k_route_permute_small(const RouteSma
   // launched after its inputs are complete: a programmatic dependent may start its prologue now
   griddep_launch_dependents();
   const int E = a.E, T = a.T, ks = a.ks;
-  // 1. logits
-  for (int eb = blockIdx.x; eb * kRouterEB < E; eb += gridDim.x)
-    router_block_logits<T16>(static_cast<const T16*>(a.x), static_cast<const T16*>(a.wr), a.bias, T, a.H, E,
-                             eb * kRouterEB, reinterpret_cast<uint4*>(smem), a.logits);
+  // 0. pre-MoE RMSNorm (and the shared-expert gate) into x_norm
+  if (a.norm_w) {
+    __shared__ float red[kThreads / 32];
+    for (int t = blockIdx.x; t < T; t += gridDim.x)
+      norm_token<T16>(static_cast<const T16*>(a.x), static_cast<const T16*>(a.norm_w),
+                      static_cast<const T16*>(a.gate_w), t, a.H, a.eps, static_cast<T16*>(a.x_norm), a.gate, red);
+    grid.sync();
+  }
+  // 1. logits (of x_norm when phase 0 ran: rows other blocks wrote, read through L2)
+  for (int eb = blockIdx.x; eb * kRouterEB < E; eb += gridDim.x) {
+    if (a.norm_w)
+      router_block_logits<T16, true>(static_cast<const T16*>(a.x_norm), static_cast<const T16*>(a.wr), a.bias, T, a.H,
+                                     E, eb * kRouterEB, reinterpret_cast<uint4*>(smem), a.logits);
+    else
+      router_block_logits<T16>(static_cast<const T16*>(a.x), static_cast<const T16*>(a.wr), a.bias, T, a.H, E,
+                               eb * kRouterEB, reinterpret_cast<uint4*>(smem), a.logits);
+  }
   grid.sync();
   // 2. top-k: by block 0 alone when every token has a warp of its own there
   // (then the permutation follows after a block barrier), else by all blocks
@@ -199,10 +291,23 @@ size_t route_permute_ws_bytes(int T, int E) {
   return c.used;
 }
 
+int rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, cudaStream_t stream,
+            const void* w_gate, float* gate);
+
+// norm (optional): the pre-MoE RMSNorm of x into norm->x_norm (and the gate)
+// before the routing, which then reads x_norm.
 int route_permute(const void* x, int T, int H, const void* w_router, const float* bias, int E, int k, int extra,
                   int dtype, int32_t* topk_idx, float* topk_w, float* topk_logit, int32_t* offsets,
-                  int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                  int32_t* row_token, int32_t* slot_row, void* ws, size_t ws_bytes, cudaStream_t stream,
+                  const RouteNorm* norm) {
   const int ks = k + extra;
+  if (norm && T > kRouteSmallMaxT) {
+    // the norm kernel (one read of x; the gate from its output), then the
+    // large-batch routing of x_norm
+    const int rc = rmsnorm(x, T, H, norm->w, norm->eps, dtype, norm->x_norm, stream, norm->gate_w, norm->gate);
+    if (rc) return rc;
+    x = norm->x_norm;
+  }
   if (T > kRouteSmallMaxT) {
     WsCarver carve(ws, ws_bytes);
     void* ws_r = carve.take<uint8_t>(route_ws_bytes(T, E));
@@ -240,6 +345,13 @@ int route_permute(const void* x, int T, int H, const void* w_router, const float
   a.row_token = row_token;
   a.slot_row = slot_row;
   a.status = device_status_ptr();
+  if (norm) {
+    a.norm_w = norm->w;
+    a.eps = norm->eps;
+    a.gate_w = norm->gate_w;
+    a.x_norm = norm->x_norm;
+    a.gate = norm->gate;
+  }
   const size_t w_bytes = size_t(kRouterEB) * H * 2;
   const size_t p_bytes = (size_t(E) * ((T + 31) / 32) + E + 1) * 4;
   const size_t smem = w_bytes > p_bytes ? w_bytes : p_bytes;

@@ -77,14 +77,18 @@ int shared_gate(const void* x, int T, int H, const void* w_gate, int dtype, floa
 // (lane-strided, then a shuffle tree), the scale with an IEEE square root and
 // division, then a second pass over the row (from L1/L2) that scales and
 // writes it in 16 bits; every lane rewrites only the pieces it reads, after
-// the sum is complete, so y may be x.
+// the sum is complete, so y may be x.  With a gate vector (w_gate, not
+// null) the second pass also forms the shared-expert gate of the token from
+// the 16-bit normalised values it writes: gate[t] = sigmoid(y[t] . w_gate),
+// so that the block's input is normalised, and its gate computed, in one
+// read of x.
 // ---------------------------------------------------------------------------
 namespace moe {
 namespace {
 
 template <typename T16>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T16* x, const T16* __restrict__ w, int T, int H, float eps,
-                                                 T16* y) {
+                                                 T16* y, const T16* __restrict__ w_gate, float* __restrict__ gate) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -105,7 +109,9 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T16* x, const T16* __rest
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float r = 1.0f / sqrtf(ss / float(H) + eps);
   const uint4* wr = reinterpret_cast<const uint4*>(w);
+  const uint4* gr = reinterpret_cast<const uint4*>(w_gate);
   uint4* yr = reinterpret_cast<uint4*>(y + size_t(t) * H);
+  float gacc = 0.f;
   for (int c = lane; c < nv; c += 32) {
     const uint4 v = xr[c], g = __ldg(wr + c);
     const uint32_t u[4] = {v.x, v.y, v.z, v.w}, gw[4] = {g.x, g.y, g.z, g.w};
@@ -116,21 +122,37 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T16* x, const T16* __rest
       o[j] = Pack2<T16>::pack(f.x * r * (1.0f + gg.x), f.y * r * (1.0f + gg.y));
     }
     yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    if (gate) {
+      const uint4 q = __ldg(gr + c);
+      const uint32_t qv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 a = Pack2<T16>::unpack(o[j]), b = Pack2<T16>::unpack(qv[j]);
+        gacc = fmaf(a.x, b.x, gacc);
+        gacc = fmaf(a.y, b.y, gacc);
+      }
+    }
+  }
+  if (gate) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) gacc += __shfl_xor_sync(0xffffffffu, gacc, o);
+    if (lane == 0) gate[t] = 1.0f / (1.0f + expf(-gacc));
   }
 }
 
 }  // namespace
 
-int rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, cudaStream_t stream) {
+int rmsnorm(const void* x, int T, int H, const void* w, float eps, int dtype, void* y, cudaStream_t stream,
+            const void* w_gate, float* gate) {
   if (T == 0) return MOE_OK;
   const dim3 grid((T + 7) / 8);
   if (dtype == MOE_DTYPE_BF16)
-    k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x),
-                                                       static_cast<const __nv_bfloat16*>(w), T, H, eps,
-                                                       static_cast<__nv_bfloat16*>(y));
+    k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w), T, H, eps,
+        static_cast<__nv_bfloat16*>(y), static_cast<const __nv_bfloat16*>(w_gate), gate);
   else
     k_rmsnorm<__half><<<grid, 256, 0, stream>>>(static_cast<const __half*>(x), static_cast<const __half*>(w), T, H,
-                                                eps, static_cast<__half*>(y));
+                                                eps, static_cast<__half*>(y), static_cast<const __half*>(w_gate), gate);
   MOE_CHECK_CUDA(cudaGetLastError());
   return MOE_OK;
 }

@@ -6,7 +6,10 @@ launches only the library's kernels (no allocation, no host sync).  The
 weight format is one of "bf16" (16-bit weights, BF16 or FP16 activations),
 "awq_g32" and "nvfp4"; the router and the shared expert are always 16-bit.
 
-forward(x)               x [T, H] on the device -> y [T, H]
+forward(x)               x [T, H] on the device -> y [T, H]; with a pre-MoE
+                         RMSNorm gain in the weights ("w_norm" [H]) the
+                         block's input is the normalised x (one call with
+                         the routing: moe_norm_route_permute)
 forward_host(xh, yh)     pinned host x -> y in pinned host memory (copies in
                          the stream, for end-to-end measurements)
 refill_pass(x, stats)    one Refill-RMS scoring pass (k+1 slots), adds to the
@@ -74,6 +77,8 @@ class MoELayer:
         self.dev = device or weights["w_router"].device
         self.E, self.H = weights["w_router"].shape
         self.adt = weights["w_router"].dtype
+        self.norm = "w_norm" in weights  # pre-MoE RMSNorm, gain 1 + w_norm, eps 1e-6
+        self.norm_eps = 1e-6
         self.I_sh = weights["w_sh_down"].shape[1]
         if fmt in ("bf16",):
             self.I = weights["w_gate_up"].shape[1] // 2
@@ -111,6 +116,8 @@ class MoELayer:
         self.shared = torch.empty((T_max, H), dtype=self.adt, device=d)
         # optional shared-expert gate (weights key "w_sh_gate", [H]): sigmoid(x . w) per token
         self.sh_gate = torch.empty((T_max,), dtype=torch.float32, device=d) if "w_sh_gate" in self.w else None
+        # the normalised block input when the layer carries its pre-MoE RMSNorm
+        self.x_norm = torch.empty((T_max, H), dtype=self.adt, device=d) if self.norm else None
         self.y = torch.empty((T_max, H), dtype=self.adt, device=d)
         op = {"bf16": abi.MOE_OP_SWIGLU_BF16, "awq_g32": abi.MOE_OP_SWIGLU_AWQ_G32,
               "nvfp4": abi.MOE_OP_SWIGLU_NVFP4}[self.fmt]
@@ -142,12 +149,23 @@ class MoELayer:
             self._sh_off[T] = t
         return t
 
-    def route(self, x: torch.Tensor):
+    def route(self, x: torch.Tensor) -> torch.Tensor:
+        """Routing and permutation of the batch; returns the block's input:
+        x, or with a pre-MoE RMSNorm the normalised x (then the shared-expert
+        gate, if the layer has one, is computed by the same call)."""
         T = x.shape[0]
         ks = self.k + self.extra
-        abi.moe_route_permute(x, self.w["w_router"], self.w["bias"], self.k, self.extra, topk_idx=self.topk_idx[:T],
-                              topk_w=self.topk_w[:T], topk_logit=self.topk_logit[:T], expert_offsets=self.offsets,
-                              row_token=self.row_token[:T * ks], slot_row=self.slot_row[:T], ws=self.ws_route)
+        outs = dict(topk_idx=self.topk_idx[:T], topk_w=self.topk_w[:T], topk_logit=self.topk_logit[:T],
+                    expert_offsets=self.offsets, row_token=self.row_token[:T * ks], slot_row=self.slot_row[:T],
+                    ws=self.ws_route)
+        if self.norm:
+            gate = self.sh_gate[:T] if self.sh_gate is not None else None
+            abi.moe_norm_route_permute(x, self.w["w_norm"], self.w["w_router"], self.w["bias"], self.k, self.extra,
+                                       eps=self.norm_eps, w_shared_gate=self.w.get("w_sh_gate"),
+                                       x_norm=self.x_norm[:T], shared_gate=gate, **outs)
+            return self.x_norm[:T]
+        abi.moe_route_permute(x, self.w["w_router"], self.w["bias"], self.k, self.extra, **outs)
+        return x
 
     def experts(self, x: torch.Tensor) -> torch.Tensor:
         T = x.shape[0]
@@ -215,9 +233,9 @@ class MoELayer:
         into the layer's own output buffer (overwritten by the next pass)."""
         T = x.shape[0]
         assert T <= self.T_max and self.extra == 0
-        self.route(x)
-        gate = self.shared_gate(x)
-        f, sh = self.experts_and_shared(x)
+        xin = self.route(x)
+        gate = self.block_gate(xin)
+        f, sh = self.experts_and_shared(xin)
         y = self.y[:T] if y is None else y
         abi.moe_combine(f, self.slot_row[:T], self.topk_w[:T], shared_out=sh, shared_gate=gate, y=y)
         return y
@@ -227,6 +245,16 @@ class MoELayer:
         if self.sh_gate is None:
             return None
         return abi.moe_shared_gate(x, self.w["w_sh_gate"], gate=self.sh_gate[:x.shape[0]])
+
+    def block_gate(self, xin: torch.Tensor) -> Optional[torch.Tensor]:
+        """The shared-expert gate of the block input xin (route's result):
+        already computed by the routing call when the layer normalises its
+        input, else by moe_shared_gate; None without a gate."""
+        if self.sh_gate is None:
+            return None
+        if self.norm:
+            return self.sh_gate[:xin.shape[0]]
+        return self.shared_gate(xin)
 
     def capture(self, x: torch.Tensor, fn=None, warmup: int = 1) -> "torch.cuda.CUDAGraph":
         """CUDA graph of fn(x) (default: forward).  Every launch of the pass
@@ -260,9 +288,9 @@ class MoELayer:
         """One Refill-RMS scoring pass over x; statistics are added in place."""
         T = x.shape[0]
         assert self.extra == 1
-        self.route(x)
-        gate = self.shared_gate(x)
-        f, sh = self.experts_and_shared(x)
+        xin = self.route(x)
+        gate = self.block_gate(xin)
+        f, sh = self.experts_and_shared(xin)
         y = self.y[:T]
         # the shared expert cancels in the score; with a gate, y is combined separately
         abi.razor_refill_rms_accumulate(f, self.slot_row[:T], self.topk_idx[:T], self.topk_logit[:T], self.offsets,

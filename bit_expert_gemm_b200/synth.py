@@ -144,6 +144,13 @@ def make_shared_gate(wl: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
     return _normal(g, (wl.H,), wl.H ** -0.5, _dt(wl.act), device)
 
 
+def make_norm_weight(wl: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
+    """Optional pre-MoE RMSNorm gain offset w [H] ~ N(0, 0.1) (the gain is
+    1 + w) in the activation dtype, from its own generator."""
+    g = _gen(8_888_887 + seed, device)
+    return _normal(g, (wl.H,), 0.1, _dt(wl.act), device)
+
+
 def make_tokens(wl: Workload, T: int, seed: int = 0, batch: int = 0, device="cpu") -> torch.Tensor:
     """x [T, H] ~ N(0, 1) in the workload's activation dtype."""
     g = _gen(1_000_003 * (seed + 1) + 7919 * T + 104_729 * batch, device)

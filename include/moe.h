@@ -176,6 +176,30 @@ MOE_API int moe_route_permute(const void* x, int T, int H, const void* w_router,
                               size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Pre-MoE RMSNorm, the optional shared-expert gate and moe_route_permute in
+ * one call [ARCH] (normalisation entries: RMSNorm before the block, gain
+ * 1 + w, epsilon 1e-6; [AWQ] "Checkpoint": the shared-expert gate tensor).
+ *
+ *   x_norm[t, h] = x[t, h] / sqrt(mean_h x[t, :]^2 + eps) * (1 + norm_w[h])
+ *                  (FP32, rounded to dtype: the block's 16-bit input)
+ *   shared_gate_out[t] = 1 / (1 + exp(-x_norm[t, :] . w_shared_gate))
+ *   then moe_route_permute of x_norm (same outputs and limits).
+ *
+ * x, x_norm [T, H] dtype (x_norm may be x); norm_w [H] dtype; w_shared_gate
+ * [H] dtype or NULL, and shared_gate_out [T] FP32 then NULL too.  The experts
+ * and the shared expert of the layer take x_norm as their input.  For T <=
+ * 128 the normalisation is a first phase of the cooperative routing kernel
+ * (one more grid barrier); larger T run one normalisation kernel (one read
+ * of x, the gate from the values it writes) before the routing of x_norm.
+ * Workspace: MOE_OP_ROUTE_PERMUTE.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_norm_route_permute(const void* x, int T, int H, const void* norm_w, float eps,
+                                   const void* w_shared_gate, const void* w_router, const float* bias, int E, int k,
+                                   int extra, int dtype, void* x_norm, float* shared_gate_out, int32_t* topk_idx,
+                                   float* topk_w, float* topk_logit, int32_t* expert_offsets, int32_t* row_token,
+                                   int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_permute without a workspace argument.  The pages have no counterpart:
  * this exists for callers that only receive input and output buffers from
  * the framework hosting them (a plug-in interface without an allocator, a

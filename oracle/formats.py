@@ -44,6 +44,17 @@ def f32_to_bf16(x: np.ndarray) -> np.ndarray:
     return rounded.astype(np.uint16)
 
 
+def f64_to_bf16_values(x: np.ndarray) -> np.ndarray:
+    """float64 -> the nearest BF16 value (ties to even), as float64, rounded
+    once from the float64 value (not through binary32).  For finite values
+    whose magnitude is inside BF16's normal range, which is all that the
+    oracle rounds: with x = m * 2^e, 0.5 <= |m| < 1, BF16 keeps 8
+    significant bits, so the result is rint(m * 256) / 256 * 2^e."""
+    x = np.asarray(x, np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
 # ----------------------------------------------------------------------------
 # FP16 (IEEE binary16).  numpy's float16 is IEEE binary16 with correctly
 # rounded conversions; the tests pin it against torch.float16.

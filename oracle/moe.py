@@ -31,6 +31,8 @@ from typing import Callable, Optional, Sequence
 
 import numpy as np
 
+from .formats import f64_to_bf16_values
+
 
 def router_logits(x: np.ndarray, w_router: np.ndarray, bias: Optional[np.ndarray]) -> np.ndarray:
     """l = x . Wr^T (+ b).  x [T, H], w_router [E, H], bias [E] -> [T, E]."""
@@ -147,6 +149,20 @@ def rmsnorm(x: np.ndarray, w: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     x = np.asarray(x, np.float64)
     ms = np.mean(x * x, axis=-1, keepdims=True)
     return x / np.sqrt(ms + eps) * (1.0 + np.asarray(w, np.float64))
+
+
+def block_input(x: np.ndarray, w: np.ndarray, eps: float = 1e-6, dtype: str = "bf16") -> np.ndarray:
+    """The MoE block's input when the layer carries its pre-MoE RMSNorm: the
+    normalised activation as the model's 16-bit tensor (BF16, or FP16 for
+    the AWQ card's FP16 compute), rounded once from the exact value.  The
+    router, the experts, the shared expert and its gate all read it.
+    x [T, H], w [H] -> [T, H] float64 holding 16-bit values."""
+    y = rmsnorm(x, w, eps)
+    if dtype == "bf16":
+        return f64_to_bf16_values(y)
+    if dtype == "f16":
+        return np.asarray(y, np.float64).astype(np.float16).astype(np.float64)
+    raise ValueError(dtype)
 
 
 def shared_gate(x: np.ndarray, w_gate: np.ndarray) -> np.ndarray:

@@ -201,3 +201,40 @@ def test_rmsnorm_against_torch_and_closed_forms():
     assert np.allclose(y[0, [0, 1, 2, 4]], 2.0 / np.sqrt(4.0 + 1e-6), rtol=1e-15) and y[0, 3] == 0.0
     # scale invariance away from eps
     assert np.allclose(moe.rmsnorm(1e3 * x, w), got, rtol=1e-6)  # eps / mean(x^2) is about 1e-7 here
+
+
+def test_bf16_rounding_from_float64():
+    """formats.f64_to_bf16_values: one round-to-nearest-even from float64 to
+    BF16.  On values exact in binary32 it equals the pinned binary32
+    converter; every result is a BF16 value; the error is at most half a
+    BF16 ulp; exact midpoints go to the even neighbour."""
+    from oracle import formats
+    rng = np.random.default_rng(8)
+    v32 = (rng.standard_normal(20000) * np.exp(rng.standard_normal(20000) * 3)).astype(np.float32)
+    got = formats.f64_to_bf16_values(v32.astype(np.float64))
+    assert np.array_equal(got, formats.bf16_to_f64(formats.f32_to_bf16(v32)))
+    v = rng.standard_normal(20000) * 5.0
+    r = formats.f64_to_bf16_values(v)
+    assert np.array_equal(formats.bf16_to_f64(formats.f32_to_bf16(r.astype(np.float32))), r)  # representable
+    ulp = np.ldexp(1.0, np.frexp(v)[1] - 8)  # spacing of BF16 values around v
+    assert np.all(np.abs(r - v) <= ulp / 2)
+    mids = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 3.0 + 2.0 ** -7])
+    assert np.array_equal(formats.f64_to_bf16_values(mids), [1.0, 1.0 + 2.0 ** -6, -1.0, 3.0])
+
+
+def test_block_input_is_the_rounded_norm():
+    """moe.block_input: the pinned RMSNorm, rounded once to BF16 (or FP16):
+    within half a 16-bit ulp of torch's rms_norm and exactly a 16-bit value."""
+    from oracle import formats
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((9, 128)) * 2.0
+    w = rng.standard_normal(128) * 0.1
+    exact = torch.nn.functional.rms_norm(torch.from_numpy(x), (128,), weight=torch.from_numpy(1.0 + w),
+                                         eps=1e-6).numpy()
+    b = moe.block_input(x, w)
+    assert np.array_equal(formats.bf16_to_f64(formats.f32_to_bf16(b.astype(np.float32))), b)
+    assert np.all(np.abs(b - exact) <= np.ldexp(1.0, np.frexp(exact)[1] - 8) / 2 * (1 + 1e-12))
+    assert not np.array_equal(b, exact)
+    h = moe.block_input(x, w, dtype="f16")
+    assert np.array_equal(h.astype(np.float16).astype(np.float64), h)
+    assert np.all(np.abs(h - exact) <= np.ldexp(1.0, np.frexp(exact)[1] - 11) / 2 * (1 + 1e-12))

@@ -204,6 +204,14 @@ MUTATIONS = [
     ("NVFP4 one global scale shared by gate and up",
      lambda mp: mp.setattr(nvfp4, "quantize_expert_weights", _nvfp4_shared_gate_up_scale),
      [tq.test_nvfp4_expert_weights_one_global_scale_per_projection]),
+    ("block input not rounded to 16 bits",
+     lambda mp: mp.setattr(moe, "block_input", lambda x, w, eps=1e-6, dtype="bf16": moe.rmsnorm(x, w, eps)),
+     [tm.test_block_input_is_the_rounded_norm]),
+    ("BF16 rounding by truncation", lambda mp: mp.setattr(
+        __import__("oracle.formats", fromlist=["formats"]), "f64_to_bf16_values",
+        lambda x: np.ldexp(np.trunc(np.frexp(np.asarray(x, np.float64))[0] * 256.0) / 256.0,
+                           np.frexp(np.asarray(x, np.float64))[1])),
+     [tm.test_bf16_rounding_from_float64]),
     ("NVFP4 block scale from 4 s_g", lambda mp: mp.setattr(nvfp4, "quantize", _quantize_4sg),
      [tq.test_nvfp4_grid_values_round_trip_exactly, tq.test_nvfp4_error_bound_and_block_max]),
 ]
