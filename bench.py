@@ -543,7 +543,8 @@ def bench_workload(args, dist: Dist, workload: str, with_e2e: bool = True, with_
     roofline["traffic"], src = measured_traffic(workload)
     if src:
         roofline["traffic_source"] = (src + ": dram__bytes_read.sum + dram__bytes_write.sum of the expert call's "
-                                      "launches, bytes per call, cold-cache ncu capture")
+                                      "launches, bytes per call, from a one-pass ncu capture of a single-layer run of "
+                                      "the same shapes (cold-cache)")
 
     # end-to-end through the public API: pinned host x -> y in pinned host memory, every step's upload and
     # download inside the timed region, overlapped with the neighbouring steps' forwards (HostPipeline)
@@ -633,6 +634,7 @@ def decode_summary(line: dict) -> dict:
     return {"tokens_per_s": line["value"], "ms_per_step": line["ms_per_step"],
             "ms_per_step_after_l2_write_flush": line["ms_per_step_after_l2_write_flush"],
             "expert_call_gbs": r["achieved"], "hbm_peak_gbs": r["peak"], "frac": r["frac"],
+            "traffic": r.get("traffic"),
             "frac_of_nominal_8tbs": r["frac_of_nominal"], "work_per_launch": r["work_per_launch"],
             "expert_ffn_ms": line["expert_ffn_ms"], "launches_per_step": line["launches_per_step"],
             "clocks": line["clocks"], "l2": line["config"]["l2"]}
