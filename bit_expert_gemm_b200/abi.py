@@ -50,6 +50,8 @@ _SIGS = {
     "moe_norm_route_permute": (_I, [_P, _I, _I, _P, ctypes.c_float, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                                     _P, _P, _P, _P, _SZ, _P]),
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "moe_ep_plan": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_gather_rows": (_I, [_P, _I, _I, _P, _I, _P, _P]),
     "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_grouped_swiglu_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _SZ, _P]),
     "moe_experts_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -255,6 +257,33 @@ def moe_norm_route_permute(x, norm_w, w_router, bias, k: int, extra: int = 0, ep
           k, extra, _dtype_code(x), _p(x_norm), _p(shared_gate), _p(topk_idx), _p(topk_w), _p(topk_logit),
           _p(expert_offsets), _p(row_token), _p(slot_row), _p(ws), ws.numel(), _stream(stream))
     return x_norm, shared_gate, topk_idx, topk_w, topk_logit, expert_offsets, row_token, slot_row
+
+
+def moe_ep_plan(expert_offsets, world: int, rows: int, row_local_expert=None, send_counts=None, stream=None):
+    """Expert-parallel dispatch plan of `rows` permuted rows: the local
+    expert index of each row at its destination rank and the rows per rank."""
+    _need(expert_offsets, torch.int32, "expert_offsets")
+    E = expert_offsets.numel() - 1
+    dev = expert_offsets.device
+    if row_local_expert is None:
+        row_local_expert = torch.empty((rows,), dtype=torch.int32, device=dev)
+    if send_counts is None:
+        send_counts = torch.empty((world,), dtype=torch.int32, device=dev)
+    _call("moe_ep_plan", _p(expert_offsets), E, world, rows, _p(row_local_expert), _p(send_counts), _stream(stream))
+    return row_local_expert, send_counts
+
+
+def moe_gather_rows(src, index, out=None, stream=None):
+    """out[r] = src[index[r]] for whole 16-bit rows."""
+    _need(index, torch.int32, "index")
+    src_rows, H = src.shape
+    rows = index.numel()
+    if src.element_size() != 2:
+        raise ValueError("moe_gather_rows: 16-bit rows expected")
+    if out is None:
+        out = torch.empty((rows, H), dtype=src.dtype, device=src.device)
+    _call("moe_gather_rows", _p(src), src_rows, H, _p(index), rows, _p(out), _stream(stream))
+    return out
 
 
 def moe_permute(topk_idx, E: int, expert_offsets=None, row_token=None, slot_row=None, ws=None, stream=None):

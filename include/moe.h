@@ -200,6 +200,29 @@ MOE_API int moe_norm_route_permute(const void* x, int T, int H, const void* norm
                                    int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Expert parallelism over `world` ranks ([NVFP4] serving example: expert
+ * parallelism over eight GPUs).  Rank d owns the routed experts
+ * [d * E/world, (d+1) * E/world).  A rank's permuted rows (moe_permute:
+ * experts ascending) are therefore already grouped by destination rank.
+ *
+ * moe_ep_plan: expert_offsets [E+1] (device) -> row_local_expert [rows] int32,
+ * the index of each permuted row's expert among its destination's experts
+ * (e mod E/world), and send_counts [world] int32, the rows each destination
+ * receives (offsets[(d+1) E/world] - offsets[d E/world]).  Limits: E a
+ * multiple of world.
+ *
+ * moe_gather_rows: out[r] = src[index[r]] for whole 16-bit rows of H
+ * elements: src [src_rows, H], index [rows] int32, out [rows, H] (H % 8 == 0,
+ * 16-byte aligned rows).  An index outside [0, src_rows) writes a zero row
+ * and records MOE_ERR_INVALID_ARG in the device status word.  Used for the x
+ * rows of the send order and for the experts' outputs in the received order.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_ep_plan(const int32_t* expert_offsets, int E, int world, int rows, int32_t* row_local_expert,
+                        int32_t* send_counts, void* stream);
+MOE_API int moe_gather_rows(const void* src, int src_rows, int H, const int32_t* index, int rows, void* out,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_permute without a workspace argument.  The pages have no counterpart:
  * this exists for callers that only receive input and output buffers from
  * the framework hosting them (a plug-in interface without an allocator, a
