@@ -198,15 +198,17 @@ __global__ void __launch_bounds__(256) k_refill(const void* __restrict__ f, cons
 
   for (int c = threadIdx.x * 4; c < H; c += blockDim.x * 4) {
     float fv[kRefillMaxSlots][4];
+    // every row load of the token is issued before the first use; a slot
+    // without a row (-1: an out-of-range expert id, recorded by the
+    // permutation) loads row 0 and contributes zeros
 #pragma unroll
     for (int j = 0; j < kRefillMaxSlots; ++j)
-      if (j < ks) {
-        if (row_sh[j] >= 0) {
-          load4<T16, F32>(f, size_t(row_sh[j]), H, c, fv[j]);
-        } else {  // an out-of-range expert id (recorded by the permutation): no row
+      if (j < ks) load4<T16, F32>(f, size_t(max(row_sh[j], 0)), H, c, fv[j]);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) fv[j][i] = 0.f;
-        }
+    for (int j = 0; j < kRefillMaxSlots; ++j)
+      if (j < ks && row_sh[j] < 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) fv[j][i] = 0.f;
       }
     float U[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -608,22 +608,39 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
 
 // out[r] = sum_{j < J} P[j][r] in ascending j; rows r < rows go to f (FP32
 // or 16-bit), the shared rows r >= rows to shared_out (16-bit).  Grid (R,
-// ceil(H / 1024)); launched as a programmatic dependent of k_decode_ffn.
+// ceil(H / 256)) of 64-thread blocks, so that a decode batch's few rows still
+// spread over many SMs; every thread issues its first kMaxJ loads (J = I/64)
+// before the first addition, which then runs in ascending j.  Launched as a
+// programmatic dependent of k_decode_ffn.
+constexpr int kMaxJ = 16;
 template <typename T16>
-__global__ void __launch_bounds__(256) k_sum_partials(const float* __restrict__ P, int J, int R, int rows, int H,
-                                                      void* __restrict__ f, int f_fp32, T16* __restrict__ shared_out) {
+__global__ void __launch_bounds__(64) k_sum_partials(const float* __restrict__ P, int J, int R, int rows, int H,
+                                                     void* __restrict__ f, int f_fp32, T16* __restrict__ shared_out) {
   griddep_wait();
   griddep_launch_dependents();
   const int r = blockIdx.x;
   const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
   if (c >= H) return;
+  float4 p[kMaxJ];
+#pragma unroll
+  for (int j = 0; j < kMaxJ; ++j)
+    p[j] = j < J ? *reinterpret_cast<const float4*>(P + (size_t(j) * R + r) * H + c) : make_float4(0.f, 0.f, 0.f, 0.f);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < J; ++j) {
-    const float4 p = *reinterpret_cast<const float4*>(P + (size_t(j) * R + r) * H + c);
-    acc.x += p.x;
-    acc.y += p.y;
-    acc.z += p.z;
-    acc.w += p.w;
+#pragma unroll
+  for (int j = 0; j < kMaxJ; ++j) {
+    if (j < J) {
+      acc.x += p[j].x;
+      acc.y += p[j].y;
+      acc.z += p[j].z;
+      acc.w += p[j].w;
+    }
+  }
+  for (int j = kMaxJ; j < J; ++j) {  // I > 1024: the rest one by one, still in ascending j
+    const float4 q = *reinterpret_cast<const float4*>(P + (size_t(j) * R + r) * H + c);
+    acc.x += q.x;
+    acc.y += q.y;
+    acc.z += q.z;
+    acc.w += q.w;
   }
   if (r < rows && f_fp32) {
     *reinterpret_cast<float4*>(static_cast<float*>(f) + size_t(r) * H + c) = acc;
@@ -649,13 +666,13 @@ int launch_fused(const Maps& maps, const Args& a, int f_fp32, void* f, void* sha
   MOE_CHECK_CUDA(launch_pdl(k_decode_ffn<WQ>, dim3(num_sms()), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, stream, maps, a));
   const int R = a.rows + a.T;
   if (R == 0) return MOE_OK;
-  const dim3 grid(R, (a.H / 4 + 255) / 256);
+  const dim3 grid(R, (a.H / 4 + 63) / 64);
   if (a.bf16)
-    MOE_CHECK_CUDA(launch_pdl(k_sum_partials<__nv_bfloat16>, grid, dim3(256), 0, stream,
+    MOE_CHECK_CUDA(launch_pdl(k_sum_partials<__nv_bfloat16>, grid, dim3(64), 0, stream,
                               static_cast<const float*>(a.partial), a.I / BK, R, a.rows, a.H, f, f_fp32,
                               static_cast<__nv_bfloat16*>(shared_out)));
   else
-    MOE_CHECK_CUDA(launch_pdl(k_sum_partials<__half>, grid, dim3(256), 0, stream, static_cast<const float*>(a.partial),
+    MOE_CHECK_CUDA(launch_pdl(k_sum_partials<__half>, grid, dim3(64), 0, stream, static_cast<const float*>(a.partial),
                               a.I / BK, R, a.rows, a.H, f, f_fp32, static_cast<__half*>(shared_out)));
   return MOE_OK;
 }
