@@ -619,7 +619,7 @@ def bench_workload(args, dist: Dist, workload: str, with_e2e: bool = True, with_
     roofline["timing"] = ("CUDA events around the expert call, in a second run of the same rotation right after "
                           "the timed region; mean over the units")
     if dist.rank == 0 and with_cpu:
-        n = args.cpu_sample_tokens or (96 if kind == "refill" else 192)
+        n = args.cpu_sample_tokens or (256 if kind == "refill" else 640)
         tps, dt = oracle_tokens_per_s(wl, w, xs[0], min(n, T), kind)
         line["cpu_baseline"] = {"value": round(tps, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"first {min(n, T)} tokens of one batch of the same workload, full layer "
