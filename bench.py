@@ -664,7 +664,7 @@ def run_reference(args, dist: Dist) -> None:
     dev = torch.device("cuda", dist.local) if torch.cuda.is_available() else torch.device("cpu")
     w = synth.make_weights(wl, seed=0, device=dev)
     x = synth.make_tokens(wl, T, seed=1, device=dev)
-    n = args.cpu_sample_tokens or (4 if kind == "refill" else 8)
+    n = args.cpu_sample_tokens or (64 if kind == "refill" else 128)
     for _ in range(args.warmup):
         oracle_tokens_per_s(wl, w, x, n, kind)
     tot_t, tot_n = 0.0, 0

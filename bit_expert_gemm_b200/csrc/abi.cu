@@ -256,10 +256,15 @@ static bool fused_decode_enabled() {
   return on != 0;
 }
 
+// The split-K kernel keeps one 16-column accumulator per 128 down-projection
+// rows in TMEM after 32 phase-A columns: H <= 3584 leaves room for its reads.
+static constexpr int kFusedMaxH = 3584;
+static bool use_fused(int T, int H) { return T <= kFusedMaxT && H <= kFusedMaxH && fused_decode_enabled(); }
+
 // AWQ routed + 16-bit shared experts: the split-K partials for T <= 16, else
 // the grouped AWQ call's workspace, reused afterwards by the shared expert's h.
 static size_t experts_awq_ws_bytes(int T, int rows, int H, int I, int E) {
-  if (T <= kFusedMaxT && fused_decode_enabled()) return decode_fused_ws_bytes(rows, T, H, I);
+  if (use_fused(T, H)) return decode_fused_ws_bytes(rows, T, H, I);
   const size_t a = awq_ws_bytes(rows, H, I, E);
   const size_t b = size_t(T) * I * 2;
   return a > b ? a : b;
@@ -267,7 +272,7 @@ static size_t experts_awq_ws_bytes(int T, int rows, int H, int I, int E) {
 
 static size_t experts_ws_bytes(int T, int rows, int H, int I) {
   (void)H;
-  if (T <= kFusedMaxT && fused_decode_enabled()) return decode_fused_ws_bytes(rows, T, H, I);
+  if (use_fused(T, H)) return decode_fused_ws_bytes(rows, T, H, I);
   if (T <= kDecodeMaxT) return decode_ws_bytes(rows, T, I);
   WsCounter c;
   c.take<uint16_t>(size_t(rows > T ? rows : T) * I);
@@ -438,7 +443,7 @@ int moe_experts_bf16(const void* x, const int32_t* row_token, const int32_t* exp
               "moe_experts_bf16: workspace of %zu bytes is too small (need %zu)", ws_bytes,
               experts_ws_bytes(T, rows, H, I));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (T <= kFusedMaxT && fused_decode_enabled())
+  if (use_fused(T, H))
     return decode_experts_fused(x, row_token, expert_offsets, T, rows, H, I, E, w_gate_up, w_down, w_sh_gate_up,
                                 w_sh_down, dtype, out_fp32, f, shared_out, ws, ws_bytes, st);
   if (T <= kDecodeMaxT)
@@ -476,7 +481,7 @@ static int experts_awq_impl(const void* x, const int32_t* row_token, const int32
               "moe_experts_awq_g32: workspace of %zu bytes is too small (need %zu)", ws_bytes,
               experts_awq_ws_bytes(T, rows, H, I, E));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (T <= kFusedMaxT && fused_decode_enabled())
+  if (use_fused(T, H))
     return decode_experts_fused_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d,
                                     sc_d, w_sh_gate_up, w_sh_down, dtype, out_fp32, f, shared_out, ws, ws_bytes, st,
                                     awq_packed);

@@ -198,6 +198,11 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
     tmem_alloc(&tmem_base_sh, TMEM_COLS);
     tmem_relinquish();
   }
+  // the h tiles start as zeros (their token columns past a group's rows are
+  // never written)
+  for (int i = threadIdx.x; i < 2 * H_BYTES / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(htile)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
   // launched as a programmatic dependent: the routing comes from the kernel before
   griddep_wait();
   griddep_launch_dependents();
@@ -429,17 +434,20 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
       mbar_arrive(&accA_empty[a]);
       // rows 0..63 gate, 64..127 up pre-activations of the block's 64 features
 #pragma unroll
-      for (int c = 0; c < NT; ++c) xchg[(q * 32 + lane) * XS + c] = v[c];
+      for (int c = 0; c < NT; ++c)
+        if (c < nn) xchg[(q * 32 + lane) * XS + c] = v[c];
       epilogue_sync();
       {
         // h[c][f] = silu(gate[f][c]) * up[f][c], 16-bit, K-major 128-byte
         // swizzled: row c at c*128 bytes, 16-byte chunk (f/8) xor (c%8),
-        // element f%8.  1024 values over the 128 threads, in a rolled loop
-        // (this code runs once per item: compact code stays cached).
+        // element f%8.  64 * nn values over the 128 threads, in a rolled loop
+        // (this code runs once per item: compact code stays cached).  Token
+        // columns c >= nn keep zeros or an earlier item's values: they feed
+        // only accumulator columns that are never read.
         const int et = threadIdx.x - 64;
         uint8_t* ht = htile + a * H_BYTES;
 #pragma unroll 1
-        for (int idx = et; idx < 64 * NT; idx += 128) {
+        for (int idx = et; idx < 64 * nn; idx += 128) {
           const int f = idx & 63, c = idx >> 6;
           const float h = silu_f(xchg[f * XS + c]) * xchg[(64 + f) * XS + c];
           const uint32_t off = uint32_t(c * 128 + (((f >> 3) ^ (c & 7)) << 4) + (f & 7) * 2);
@@ -455,18 +463,66 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
       // phase B: FP32 partials of the group's rows
       if (!epilogue_all(mbar_wait(&accB_full, uint32_t(n & 1), &abort_flag, status, lim))) break;
       tc_fence_after();
-      float* P = args.partial + (size_t(j) * R + r0) * args.H;
-      // two blocks' accumulators (32 consecutive columns) per TMEM load wait
-      for (int m0 = 0; m0 < MB2; m0 += 2) {
-        float w0[32];
-        tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + ACCB_COL + uint32_t(m0 * NT), w0);
+      float* P = args.partial + (size_t(j) * R + r0) * args.H + q * 32 + lane;
+      const size_t H = size_t(args.H);
+      const uint32_t tq = tmem_base + (uint32_t(q * 32) << 16) + ACCB_COL;
+      // the accumulators' first nn columns, many blocks per TMEM load wait
+      // (a load's latency is paid once per batch): 16 blocks x 4 columns, 8 x
+      // 8, or 4 x 16 (addresses of blocks past the last clamped to it); the
+      // AWQ kernels (fewer registers per thread) 8 x 4 or 2 x 16
+      if (nn <= 4) {
+        // 16 blocks per wait; 8 in the AWQ kernels, whose 576 threads have
+        // fewer registers each
+        constexpr int NB = WQ ? 8 : 16;
+        for (int m0 = 0; m0 < MB2; m0 += NB) {
+          uint32_t ta[NB], v[NB * 4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (m0 + u < MB2) {
-            const int feat = (m0 + u) * BM + q * 32 + lane;
+          for (int b = 0; b < NB; ++b) ta[b] = tq + uint32_t(min(m0 + b, MB2 - 1) * NT);
+          if constexpr (WQ) tmem_ld_8x4(ta, v); else tmem_ld_16x4(ta, v);
 #pragma unroll
-            for (int c = 0; c < NT; ++c)
-              if (c < nn) P[size_t(c) * args.H + feat] = w0[u * NT + c];
+          for (int b = 0; b < NB; ++b)
+            if (m0 + b < MB2)
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                if (c < nn) P[size_t(c) * H + size_t(m0 + b) * BM] = __uint_as_float(v[b * 4 + c]);
+        }
+      } else if (WQ) {
+        for (int m0 = 0; m0 < MB2; m0 += 2) {
+          float w0[32];
+          tmem_ld32(tq + uint32_t(m0 * NT), w0);
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            if (m0 + u < MB2)
+#pragma unroll
+              for (int c = 0; c < NT; ++c)
+                if (c < nn) P[size_t(c) * H + size_t(m0 + u) * BM] = w0[u * NT + c];
+        }
+      } else if (nn <= 8) {
+        for (int m0 = 0; m0 < MB2; m0 += 8) {
+          uint32_t ta[8], v[64];
+#pragma unroll
+          for (int b = 0; b < 8; ++b) ta[b] = tq + uint32_t(min(m0 + b, MB2 - 1) * NT);
+          tmem_ld_8x8(ta, v);
+#pragma unroll
+          for (int b = 0; b < 8; ++b)
+            if (m0 + b < MB2)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                if (c < nn) P[size_t(c) * H + size_t(m0 + b) * BM] = __uint_as_float(v[b * 8 + c]);
+        }
+      } else {
+        for (int m0 = 0; m0 < MB2; m0 += 4) {
+          float w0[32], w1[32];
+          // blocks m0, m0+1 and m0+2, m0+3 (32 columns each); MB2 <= 28 keeps
+          // the reads past an odd last block inside the allocation
+          tmem_ld32x2(tq + uint32_t(m0 * NT), tq + uint32_t(min(m0 + 2, MB2 - 1) * NT), w0, w1);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (m0 + u < MB2) {
+#pragma unroll
+              for (int c = 0; c < NT; ++c)
+                if (c < nn) P[size_t(c) * H + size_t(m0 + u) * BM] = u < 2 ? w0[u * NT + c] : w1[(u - 2) * NT + c];
+            }
           }
         }
       }
@@ -680,8 +736,8 @@ int launch_fused(const Maps& maps, const Args& a, int f_fp32, void* f, void* sha
 int fill_args(Args& a, const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
               int E, int dtype, void* ws, size_t ws_bytes) {
   MOE_REQUIRE(T <= kFusedMaxT, MOE_ERR_UNSUPPORTED, "fused decode experts: T=%d > %d", T, kFusedMaxT);
-  MOE_REQUIRE(H % BM == 0 && I % BK == 0, MOE_ERR_UNSUPPORTED,
-              "fused decode experts: need H %% 128 == 0 and I %% 64 == 0 (H=%d I=%d)", H, I);
+  MOE_REQUIRE(H % BM == 0 && I % BK == 0 && H / BM <= 28, MOE_ERR_UNSUPPORTED,
+              "fused decode experts: need H %% 128 == 0, H <= 3584 and I %% 64 == 0 (H=%d I=%d)", H, I);
   MOE_REQUIRE(E <= kGemmMaxGroups, MOE_ERR_UNSUPPORTED, "fused decode experts: E=%d > %d", E, kGemmMaxGroups);
   WsCarver carve(ws, ws_bytes);
   float* P = carve.take<float>(size_t(I / BK) * (rows + T) * H);
