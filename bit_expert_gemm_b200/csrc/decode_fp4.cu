@@ -15,7 +15,8 @@
 // compute the same function; a decode batch streams each touched expert's
 // 2.2 MB once, which is HBM-bound work with no use for a 128-row MMA tile.
 //
-// Three launches:
+// Three launches, each a programmatic dependent of the one before (its
+// launch and block scheduling overlap the previous kernel's tail):
 //   k_fp4_prep    one block: amax of x, each token quantised once (the
 //                 library's group-16 recipe), the list of experts with
 //                 routed rows, and the h amax word cleared;
@@ -98,6 +99,9 @@ struct Fp4DecArgs {
 template <typename T16>
 __global__ void __launch_bounds__(1024) k_fp4_prep(const T16* __restrict__ x, Fp4DecArgs a, uint8_t* xq, uint8_t* xsf,
                                                    int32_t* active) {
+  // launched as a programmatic dependent: inputs from the kernels before
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ float red[32];
   __shared__ int scan[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -261,6 +265,8 @@ __device__ __forceinline__ void fp4_rows(int K, int n_e, const uint8_t* wbase, c
 template <int SWIGLU>
 __global__ void __launch_bounds__(256, 3) k_fp4_gemv(Fp4DecArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
+  griddep_wait();
+  griddep_launch_dependents();
   const int K = SWIGLU ? a.H : a.I;
   const int nb = K / 16;
   int8_t* act = reinterpret_cast<int8_t*>(smem);
@@ -399,8 +405,8 @@ int nvfp4_decode(const void* x, const int32_t* row_token, const int32_t* offsets
   a.amax = amax;
   a.gs_in = act_gs_in;
   a.h = reinterpret_cast<__nv_bfloat16*>(h);
-  k_fp4_prep<__nv_bfloat16><<<1, 1024, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), a, xq, xsf, active);
-  MOE_CHECK_CUDA(cudaGetLastError());
+  MOE_CHECK_CUDA(launch_pdl(k_fp4_prep<__nv_bfloat16>, dim3(1), dim3(1024), 0, stream,
+                            static_cast<const __nv_bfloat16*>(x), a, xq, xsf, active));
   // work items: at most min(E, rows) experts x tiles x 4 slices; up to 8
   // blocks of 8 warps per SM
   const int max_active = std::min(E, rows);
@@ -416,16 +422,14 @@ int nvfp4_decode(const void* x, const int32_t* row_token, const int32_t* offsets
   a.wsf = w1sf;
   a.gsw = gs_gu;
   const int g1 = std::max(1, std::min(cap, max_active * (I / 64) * 4));
-  k_fp4_gemv<1><<<g1, 256, smem1, stream>>>(a);
-  MOE_CHECK_CUDA(cudaGetLastError());
+  MOE_CHECK_CUDA(launch_pdl(k_fp4_gemv<1>, dim3(g1), dim3(256), smem1, stream, a));
   a.w = w_d;
   a.wsf = w2sf;
   a.gsw = gs_d;
   a.f = f;
   a.f_fp32 = out_fp32;
   const int g2 = std::max(1, std::min(cap, max_active * (H / 128) * 4));
-  k_fp4_gemv<0><<<g2, 256, smem2, stream>>>(a);
-  MOE_CHECK_CUDA(cudaGetLastError());
+  MOE_CHECK_CUDA(launch_pdl(k_fp4_gemv<0>, dim3(g2), dim3(256), smem2, stream, a));
   return MOE_OK;
 }
 

@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(256) k_dense_gemv1(const T16* __restrict__ x, 
                                                      int T, const T16* __restrict__ w_gu, int H, int I,
                                                      float* __restrict__ P) {
   extern __shared__ __align__(16) uint8_t smem[];
+  griddep_wait();
+  griddep_launch_dependents();
   T16* xs = reinterpret_cast<T16*>(smem);  // [NT][H/4]
   // the expert's rows, clamped to the batch
   const int r0 = max(0, offsets[0]);
@@ -111,6 +113,8 @@ __global__ void __launch_bounds__(256) k_dense_gemv2(const float* __restrict__ P
                                                      int T, const T16* __restrict__ w_d, int H, int I, int out_fp32,
                                                      void* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem[];
+  griddep_wait();
+  griddep_launch_dependents();
   T16* hs = reinterpret_cast<T16*>(smem);  // [NT][I]
   // the expert's rows, clamped to the batch
   const int r0 = max(0, offsets[0]);
@@ -179,12 +183,11 @@ int launch_dense(const void* x, const int32_t* offsets, int T, int H, int I, con
     MOE_CHECK_CUDA(cudaFuncSetAttribute(k_dense_gemv1<T16, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(s1)));
   if (s2 > 48 * 1024)
     MOE_CHECK_CUDA(cudaFuncSetAttribute(k_dense_gemv2<T16, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(s2)));
-  k_dense_gemv1<T16, NT><<<dim3(I / 16, 4), 256, s1, stream>>>(static_cast<const T16*>(x), offsets, T,
-                                                                static_cast<const T16*>(w_gu), H, I, P);
-  MOE_CHECK_CUDA(cudaGetLastError());
-  k_dense_gemv2<T16, NT><<<H / 32, 256, s2, stream>>>(P, offsets, T, static_cast<const T16*>(w_d), H, I, out_fp32,
-                                                       out);
-  MOE_CHECK_CUDA(cudaGetLastError());
+  // programmatic dependents: launch and block scheduling overlap the kernel before
+  MOE_CHECK_CUDA(launch_pdl(k_dense_gemv1<T16, NT>, dim3(I / 16, 4), dim3(256), s1, stream, static_cast<const T16*>(x),
+                            offsets, T, static_cast<const T16*>(w_gu), H, I, P));
+  MOE_CHECK_CUDA(launch_pdl(k_dense_gemv2<T16, NT>, dim3(H / 32), dim3(256), s2, stream, static_cast<const float*>(P),
+                            offsets, T, static_cast<const T16*>(w_d), H, I, out_fp32, out));
   return MOE_OK;
 }
 

@@ -137,7 +137,7 @@ __device__ void norm_token(const T16* __restrict__ x, const T16* __restrict__ w,
 }
 
 template <typename T16, int NV>
-__global__ void __launch_bounds__(kThreads) k_route_permute_small(const RouteSmallArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) k_route_permute_small(const RouteSmallArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   cg::grid_group grid = cg::this_grid();
   // launched after its inputs are complete: a programmatic dependent may start its prologue now
