@@ -338,6 +338,24 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ, AG>::THREADS, 1)
           }
           warp_store_rows<64>(stg, pk, nvalid, gtile + size_t(t.n * BNH + c * 32) * 2, pitch, lane);
         }
+      } else if (!args.out_fp32 && !args.bias) {
+        // 16-bit output: 64 columns per TMEM load wait, stored as whole
+        // 128-byte segments of each row
+        static_assert(BN % 64 == 0, "tile widths are 64, 128 or 256");
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; c += 2) {
+          float v0[32], v1[32];
+          tmem_ld32x2(tb + c * 32, tb + (c + 1) * 32, v0, v1);
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = args.bf16 ? Pack2<__nv_bfloat16>::pack(v0[2 * i], v0[2 * i + 1])
+                              : Pack2<__half>::pack(v0[2 * i], v0[2 * i + 1]);
+            pk[16 + i] = args.bf16 ? Pack2<__nv_bfloat16>::pack(v1[2 * i], v1[2 * i + 1])
+                                   : Pack2<__half>::pack(v1[2 * i], v1[2 * i + 1]);
+          }
+          warp_store_rows<128>(stg, pk, nvalid, gtile + size_t(t.n * BN + c * 32) * 2, pitch, lane);
+        }
       } else {
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
