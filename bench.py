@@ -626,9 +626,10 @@ def bench_workload(args, dist: Dist, workload: str, with_e2e: bool = True, with_
                           "the timed region; mean over the units")
     if dist.rank == 0 and with_cpu:
         # the same per-call sample as the reference arm's steps (so the two
-        # rates compare), called on consecutive slices of one batch until
-        # about 10 s of CPU work
+        # rates compare): one untimed call, then calls on consecutive slices
+        # of one batch until about 10 s of CPU work
         n = min(args.cpu_sample_tokens or CPU_SAMPLE_TOKENS[kind], T)
+        oracle_tokens_per_s(wl, w, xs[0][T - n:], n, kind)  # untimed warm-up call, as the reference arm has
         tot_t, tot_n, calls = 0.0, 0, 0
         while calls < 4 and (calls == 0 or tot_t < 10.0) and (calls + 1) * n <= T:
             _, dt = oracle_tokens_per_s(wl, w, xs[0][calls * n:], n, kind)
