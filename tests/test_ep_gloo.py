@@ -3,7 +3,8 @@ orchestration of ep.py (routing, plan, the two all-to-all exchanges with
 their split sizes, the local permutation, the return to the source ranks'
 permuted order, the combine) with the steps taken by the oracle instead of
 the kernels.  Every rank's output must equal the oracle's whole layer on that
-rank's tokens."""
+rank's tokens; with extra = 1 (Refill-RMS scoring) every rank's statistics,
+after the all-reduce, must equal the oracle's over all ranks' tokens."""
 
 import os
 import socket
@@ -26,12 +27,14 @@ class OracleOps:
     """The steps of ep.ExpertParallelLayer computed by the oracle in float64
     on CPU tensors (the layer's buffers), for testing the orchestration."""
 
-    def route_permute(self, x, w_router, bias, k, bufs):
+    def route_permute(self, x, w_router, bias, k, extra, bufs):
         from oracle import moe
-        r = moe.route(x.numpy(), w_router.numpy(), bias.numpy(), k)
+        r = moe.route(x.numpy(), w_router.numpy(), bias.numpy(), k, extra)
         p = moe.permute(r["idx"], w_router.shape[0])
+        self.p = r["p"]
         bufs["topk_idx"].copy_(torch.from_numpy(r["idx"]))
         bufs["topk_w"].copy_(torch.from_numpy(r["w"]))
+        bufs["topk_logit"].copy_(torch.from_numpy(np.take_along_axis(r["logits"], r["idx"], axis=1)))
         bufs["offsets"].copy_(torch.from_numpy(p["offsets"]))
         bufs["row_token"].copy_(torch.from_numpy(p["row_token"]))
         bufs["slot_row"].copy_(torch.from_numpy(p["slot_row"]))
@@ -75,6 +78,16 @@ class OracleOps:
     def combine(self, f_home, slot_row, topk_w, shared, y):
         from oracle import moe
         y.copy_(torch.from_numpy(moe.combine(f_home.numpy(), slot_row.numpy(), topk_w.numpy(), shared.numpy())))
+
+    def refill(self, f_home, slot_row, topk_idx, topk_logit, offsets, sum_sq, count, shared, y, ws):
+        from oracle import moe, razor
+        k = slot_row.shape[1] - 1
+        idx, sr = topk_idx.numpy().astype(np.int64), slot_row.numpy().astype(np.int64)
+        d = razor.refill_deltas_closed_form(f_home.numpy(), sr, idx, self.p, k)
+        razor.accumulate(sum_sq.numpy(), count.numpy(), d, idx, k)  # in place (shared storage)
+        pk = np.take_along_axis(self.p, idx[:, :k], axis=1)
+        y.copy_(torch.from_numpy(moe.combine(f_home.numpy(), sr[:, :k], pk / pk.sum(1, keepdims=True),
+                                             shared.numpy())))
 
 
 def _weights(E, H, I, seed):
@@ -138,3 +151,68 @@ def test_expert_parallel_matches_whole_layer(world):
                                 lambda e: (w["w_gate_up"][e, :I], w["w_gate_up"][e, I:], w["w_down"][e]),
                                 (w["w_sh_gate_up"][:I], w["w_sh_gate_up"][I:], w["w_sh_down"]))
             assert np.allclose(res[f"y{rank}_{step}"], ref["y"], rtol=1e-12, atol=1e-12), (rank, step)
+
+
+def _refill_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import datetime
+
+    import torch.distributed as dist
+
+    from bit_expert_gemm_b200 import ep
+    from bit_expert_gemm_b200.layer import refill_allreduce
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = _weights(E, H, I, 7)
+        T = 20 + 7 * rank
+        layer = ep.ExpertParallelLayer(w, K, rank, world, T_max=48, ops=OracleOps(), device=torch.device("cpu"),
+                                       extra=1)
+        sum_sq = torch.zeros(E, dtype=torch.float64)
+        count = torch.zeros(E, dtype=torch.int64)
+        for step in range(2):
+            x = _tokens(rank + 10 * step, T, H)
+            y = ep.refill_pass(layer, x, sum_sq, count)
+            out[f"y{rank}_{step}"] = y.numpy().copy()
+        refill_allreduce(sum_sq, count)
+        out[f"s{rank}"] = sum_sq.numpy().copy()
+        out[f"c{rank}"] = count.numpy().copy()
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", WORLDS)
+def test_expert_parallel_refill_statistics(world):
+    """Refill-RMS scoring with the experts split over the ranks: each rank's
+    k + 1 routed rows per token travel and come back, the statistics are added
+    at the tokens' home, and after the all-reduce every rank holds the sums and
+    counts of all ranks' tokens, as the oracle's single-process pass gives."""
+    from oracle import moe, razor
+
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_refill_worker, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
+        res = dict(out)
+    w = {n: t.numpy() for n, t in _weights(E, H, I, 7).items()}
+    ew = lambda e: (w["w_gate_up"][e, :I], w["w_gate_up"][e, I:], w["w_down"][e])
+    sh = (w["w_sh_gate_up"][:I], w["w_sh_gate_up"][I:], w["w_sh_down"])
+    s_ref, c_ref = np.zeros(E), np.zeros(E, np.int64)
+    for rank in range(world):
+        T = 20 + 7 * rank
+        for step in range(2):
+            x = _tokens(rank + 10 * step, T, H).numpy()
+            ref = moe.moe_layer(x, w["w_router"], w["bias"], K, ew, sh, extra=1)
+            r = ref["route"]
+            d = razor.refill_deltas_closed_form(ref["f"], ref["perm"]["slot_row"], r["idx"], r["p"], K)
+            razor.accumulate(s_ref, c_ref, d, r["idx"], K)
+            assert np.allclose(res[f"y{rank}_{step}"], ref["y"], rtol=1e-12, atol=1e-12), (rank, step)
+    assert c_ref.sum() > 0
+    for rank in range(world):
+        assert np.array_equal(res[f"c{rank}"], c_ref), rank
+        assert np.allclose(res[f"s{rank}"], s_ref, rtol=1e-12, atol=0), rank

@@ -4,7 +4,8 @@ device, the two exchanges as copies between their buffers, in the order a
 real exchange imposes; no kernel waits for another).  Prefill-sized batches
 run the same GEMM kernels as MoELayer on the same rows, so every rank's
 output must equal MoELayer's on its tokens bit for bit; a decode-sized batch
-(MoELayer then takes the decode kernels) is compared with the oracle."""
+(MoELayer then takes the decode kernels) is compared with the oracle; the
+Refill scoring pass (extra = 1) is compared with MoELayer.refill_pass."""
 
 import numpy as np
 import pytest
@@ -38,6 +39,38 @@ def test_expert_parallel_equals_layer(bf16_weights, world, T):
         assert torch.equal(ys[r], ref), r
         # the exchange moved every routed row: the ranks together received T*k rows per rank
         assert int(layers[r].send_counts.sum()) == xs[r].shape[0] * wl.k
+    del layers
+
+
+def test_expert_parallel_refill_equals_layer(bf16_weights):
+    """Refill-RMS scoring with the experts split over two emulated ranks: each
+    rank's statistics and outputs equal MoELayer.refill_pass on its tokens bit
+    for bit (the same FP32 rows, permuted order and fixed-order sums), and the
+    ranks' statistics added equal one pass over all their tokens."""
+    wl, w = bf16_weights
+    world, T = 2, 512
+    layers = [ep.ExpertParallelLayer(w, wl.k, r, world, T_max=T, extra=1) for r in range(world)]
+    xs = [synth.make_tokens(wl, T - 16 * r, seed=60 + r, device=DEV) for r in range(world)]
+    stats = [(torch.zeros(wl.E, dtype=torch.float64, device=DEV), torch.zeros(wl.E, dtype=torch.int64, device=DEV))
+             for _ in range(world)]
+    ys = [y.clone() for y in ep.forward_emulated(layers, xs, stats=stats)]
+    torch.cuda.synchronize()
+    assert abi.moe_device_status() == 0
+    ref_layer = MoELayer(w, wl.k, "bf16", T_max=2 * T, extra=1)
+    for r in range(world):
+        ss = torch.zeros_like(stats[r][0])
+        cc = torch.zeros_like(stats[r][1])
+        y_ref = ref_layer.refill_pass(xs[r], ss, cc).clone()
+        assert torch.equal(ys[r], y_ref), r
+        assert torch.equal(stats[r][1], cc), r
+        assert torch.equal(stats[r][0], ss), r
+        assert int(cc.sum()) == xs[r].shape[0] * wl.k
+    ss = torch.zeros_like(stats[0][0])
+    cc = torch.zeros_like(stats[0][1])
+    ref_layer.refill_pass(torch.cat(xs), ss, cc)
+    torch.cuda.synchronize()
+    assert torch.equal(stats[0][1] + stats[1][1], cc)
+    assert rel_err((stats[0][0] + stats[1][0]).cpu().numpy(), ss.cpu().numpy()) < 1e-9
     del layers
 
 
