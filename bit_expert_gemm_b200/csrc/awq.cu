@@ -103,12 +103,28 @@ int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scale
 // Gate/up unit (j, kt): K rows 64 kt.., output words 8j..8j+7 of the gate
 // half (wc < 8) and I/8 + 8j.. of the up half (wc >= 8); down unit (j, m):
 // K rows 64 j.. (the down projection's input features), output words
-// 16 m..16 m + 15.  Values are copied, not changed.
+// 16 m..16 m + 15.  Codes and zero points are stored in pair order: the
+// value of a word's output column 2m goes to nibble m, that of column 2m + 1
+// to nibble m + 4 (the checkpoint has column c in nibble c), so that the
+// dequantisation forms consecutive column pairs; scales are copied as they
+// are.
 // ---------------------------------------------------------------------------
 constexpr int kAwqUnitBytes = 4736;
 
 size_t awq_packed_bytes(int E, int H, int I) {
   return size_t(E) * size_t(I / 64) * size_t(H / 64 + H / 128) * kAwqUnitBytes;
+}
+
+// Column c of a checkpoint word (nibble c) to pair order: columns 2m, 2m + 1
+// in nibbles m, m + 4.
+__device__ __forceinline__ uint32_t awq_pair_order(uint32_t w) {
+  uint32_t o = 0;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    o |= ((w >> (8 * m)) & 0xFu) << (4 * m);           // column 2m
+    o |= ((w >> (8 * m + 4)) & 0xFu) << (4 * m + 16);  // column 2m + 1
+  }
+  return o;
 }
 
 // grid (units per expert, E), 256 threads
@@ -146,10 +162,10 @@ __global__ void __launch_bounds__(256) k_awq_pack(const uint32_t* __restrict__ q
   {  // codes: thread t = (r0, wc) copies rows r0, r0 + 16, r0 + 32, r0 + 48 of word wc
     const int r0 = t >> 4, wc = t & 15;
     uint4 c;
-    c.x = qw[size_t(k0 + r0) * W + word(wc)];
-    c.y = qw[size_t(k0 + r0 + 16) * W + word(wc)];
-    c.z = qw[size_t(k0 + r0 + 32) * W + word(wc)];
-    c.w = qw[size_t(k0 + r0 + 48) * W + word(wc)];
+    c.x = awq_pair_order(qw[size_t(k0 + r0) * W + word(wc)]);
+    c.y = awq_pair_order(qw[size_t(k0 + r0 + 16) * W + word(wc)]);
+    c.z = awq_pair_order(qw[size_t(k0 + r0 + 32) * W + word(wc)]);
+    c.w = awq_pair_order(qw[size_t(k0 + r0 + 48) * W + word(wc)]);
     reinterpret_cast<uint4*>(dst)[t] = c;
   }
   {  // scales: thread t = (group, column)
@@ -158,7 +174,7 @@ __global__ void __launch_bounds__(256) k_awq_pack(const uint32_t* __restrict__ q
   }
   if (t < 32) {  // zero points
     const int gi = t >> 4, wc = t & 15;
-    reinterpret_cast<uint32_t*>(dst + 4608)[t] = qz[size_t(g0 + gi) * W + word(wc)];
+    reinterpret_cast<uint32_t*>(dst + 4608)[t] = awq_pair_order(qz[size_t(g0 + gi) * W + word(wc)]);
   }
 }
 

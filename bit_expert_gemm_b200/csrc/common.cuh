@@ -505,6 +505,45 @@ __device__ __forceinline__ uint4 awq_dequant8(uint32_t W, const AwqGroup& g) {
   return make_uint4(__byte_perm(d[0], d[1], 0x5410), __byte_perm(d[2], d[3], 0x5410), __byte_perm(d[0], d[1], 0x7632),
                     __byte_perm(d[2], d[3], 0x7632));
 }
+// The same for words in pair order (the tile-packed copy: output columns 2m
+// and 2m + 1 in nibbles m and m + 4, zero points likewise): the pairs come
+// out as consecutive columns, so the scales are the 16-bit pairs of S as
+// they are and the eight values need no reordering.
+template <bool BF = false>
+__device__ __forceinline__ AwqGroup awq_group_paired(uint32_t Z, uint4 S) {
+  constexpr uint32_t magic = BF ? 0x43004300u : 0x64006400u;
+  AwqGroup g;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) g.z[m] = ((Z >> (4 * m)) & 0x000F000Fu) | magic;
+  g.s[0] = S.x;
+  g.s[1] = S.y;
+  g.s[2] = S.z;
+  g.s[3] = S.w;
+  if (BF) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) g.s[m] = f16x2_to_bf16x2_rn(g.s[m]);
+  }
+  return g;
+}
+template <bool BF = false>
+__device__ __forceinline__ uint4 awq_dequant8_paired(uint32_t W, const AwqGroup& g) {
+  constexpr uint32_t magic = BF ? 0x43004300u : 0x64006400u;
+  uint32_t d[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const uint32_t q = ((W >> (4 * m)) & 0x000F000Fu) | magic;
+    if (BF) {
+      uint32_t t;
+      asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(q), "r"(g.z[m]));
+      asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d[m]) : "r"(t), "r"(g.s[m]));
+    } else {
+      __half2 t = __hsub2(*reinterpret_cast<const __half2*>(&q), *reinterpret_cast<const __half2*>(&g.z[m]));
+      __half2 v = __hmul2(t, *reinterpret_cast<const __half2*>(&g.s[m]));
+      d[m] = *reinterpret_cast<uint32_t*>(&v);  // (c_2m, c_2m+1)
+    }
+  }
+  return make_uint4(d[0], d[1], d[2], d[3]);
+}
 template <bool BF = false>
 __device__ __forceinline__ uint4 awq_dequant8(uint32_t W, uint32_t Z, uint4 S) {
   return awq_dequant8<BF>(W, awq_group<BF>(Z, S));

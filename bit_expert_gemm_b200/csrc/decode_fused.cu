@@ -632,20 +632,30 @@ __global__ void __launch_bounds__(FusedCfg<WQ>::THREADS, 1)
               }
             }
           }
+          // the packed copy holds codes and zero points in pair order
+          auto convert = [&](auto group, auto dequant) {
 #pragma unroll
-          for (int u = 0; u < KSUB; ++u) {
-            if (u < nsub) {
-              uint8_t* at = sub(stage, u) + atom_off;
-              const AwqGroup g0 = awq_group<WQ == 2>(z[u][0], sv[u][0]), g1 = awq_group<WQ == 2>(z[u][1], sv[u][1]);
+            for (int u = 0; u < KSUB; ++u) {
+              if (u < nsub) {
+                uint8_t* at = sub(stage, u) + atom_off;
+                const AwqGroup g0 = group(z[u][0], sv[u][0]), g1 = group(z[u][1], sv[u][1]);
 #pragma unroll
-              for (int i = 0; i < NRW; ++i) {
-                const int r = r0 + 16 * i;  // rows 0..31 use group 0, 32..63 group 1
-                const uint4 v = awq_dequant8<WQ == 2>(cv[u][i], i < NRW / 2 ? g0 : g1);
-                const uint32_t off = uint32_t(r >> 3) * AQ_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
-                *reinterpret_cast<uint4*>(at + off) = v;
+                for (int i = 0; i < NRW; ++i) {
+                  const int r = r0 + 16 * i;  // rows 0..31 use group 0, 32..63 group 1
+                  const uint4 v = dequant(cv[u][i], i < NRW / 2 ? g0 : g1);
+                  const uint32_t off =
+                      uint32_t(r >> 3) * AQ_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
+                  *reinterpret_cast<uint4*>(at + off) = v;
+                }
               }
             }
-          }
+          };
+          if (packed)
+            convert([](uint32_t zz, uint4 ss) { return awq_group_paired<WQ == 2>(zz, ss); },
+                    [](uint32_t w, const AwqGroup& g) { return awq_dequant8_paired<WQ == 2>(w, g); });
+          else
+            convert([](uint32_t zz, uint4 ss) { return awq_group<WQ == 2>(zz, ss); },
+                    [](uint32_t w, const AwqGroup& g) { return awq_dequant8<WQ == 2>(w, g); });
           fence_proxy_async_smem();  // the FP16 tile is read by the tensor cores
         }
         mbar_arrive(&aready_bar[stage]);

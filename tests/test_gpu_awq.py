@@ -91,7 +91,8 @@ def test_awq_prepack_layout():
     """Every byte of the tile-packed copy against the layout spelled out in
     numpy: per expert the gate/up units (j, kt), then the down units (j, m);
     per unit codes [r0][wc][i] (K row r0 + 16 i, code word wc), scales
-    [2 groups][128 columns], zeros [2 groups][16 words]."""
+    [2 groups][128 columns], zeros [2 groups][16 words]; code and zero words
+    in pair order (column 2m in nibble m, column 2m + 1 in nibble m + 4)."""
     E, H, I = 3, 256, 128
     wl = dataclasses.replace(synth.WORKLOADS["awq_g32"], H=H, I=I, I_sh=I, E=E, k=2)
     w = synth.make_weights(wl, seed=7, device=DEV)
@@ -109,6 +110,14 @@ def test_awq_prepack_layout():
         for j in range(J):
             for m in range(nkb):
                 units.append((h["qw_d"][e], h["qz_d"][e], h["sc_d"][e], 64 * j, [16 * m + c for c in range(16)]))
+    def pair_order(a):
+        u = a.astype(np.int64) & 0xFFFFFFFF
+        o = np.zeros_like(u)
+        for m in range(4):
+            o |= ((u >> (8 * m)) & 0xF) << (4 * m)
+            o |= ((u >> (8 * m + 4)) & 0xF) << (4 * m + 16)
+        return o.astype(np.uint32).view(np.int32)
+
     want = []
     for qw, qz, sc, k0, words in units:
         codes = np.array([[[qw[k0 + r0 + 16 * i, words[wc]] for i in range(4)] for wc in range(16)]
@@ -116,8 +125,8 @@ def test_awq_prepack_layout():
         cols = np.array([8 * words[c // 8] + c % 8 for c in range(128)])
         scales = np.stack([sc[k0 // 32 + gi, cols] for gi in range(2)]).astype(np.float16)
         zeros = np.stack([qz[k0 // 32 + gi, words] for gi in range(2)]).astype(np.int32)
-        want.append(np.concatenate([codes.view(np.uint8).ravel(), scales.view(np.uint8).ravel(),
-                                    zeros.view(np.uint8).ravel()]))
+        want.append(np.concatenate([pair_order(codes).view(np.uint8).ravel(), scales.view(np.uint8).ravel(),
+                                    pair_order(zeros).view(np.uint8).ravel()]))
     want = np.concatenate(want)
     assert got.size == abi.load().moe_awq_packed_bytes(E, H, I) == want.size
     assert np.array_equal(got, want)
