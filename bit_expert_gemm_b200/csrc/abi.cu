@@ -36,7 +36,7 @@ size_t awq_ws_bytes(int rows, int H, int I, int E);
 int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
                        int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
                        const int32_t* qz_d, const void* sc_d, int dtype, int out_fp32, void* f, void* ws,
-                       size_t ws_bytes, cudaStream_t stream);
+                       size_t ws_bytes, cudaStream_t stream, const void* awq_packed);
 int awq_dequant(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N, int dtype,
                 void* out, cudaStream_t stream);
 size_t nvfp4_quant_ws_bytes(int batch, int rows, int K);
@@ -488,7 +488,7 @@ static int experts_awq_impl(const void* x, const int32_t* row_token, const int32
   int rc = MOE_OK;
   if (rows > 0) {
     rc = grouped_swiglu_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
-                            dtype, out_fp32, f, ws, ws_bytes, st);
+                            dtype, out_fp32, f, ws, ws_bytes, st, awq_packed);
     if (rc) return rc;
   }
   return dense_swiglu(x, T, H, I, w_sh_gate_up, w_sh_down, dtype, shared_out, static_cast<uint16_t*>(ws), st);
@@ -550,7 +550,7 @@ int moe_grouped_swiglu_awq_g32(const void* x, const int32_t* row_token, const in
   MOE_REQUIRE(x && expert_offsets && qw_gu && qz_gu && sc_gu && qw_d && qz_d && sc_d && f, MOE_ERR_INVALID_ARG,
               "moe_grouped_swiglu_awq_g32: null pointer");
   return grouped_swiglu_awq(x, row_token, expert_offsets, T, rows, H, I, E, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
-                            dtype, out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+                            dtype, out_fp32, f, ws, ws_bytes, static_cast<cudaStream_t>(stream), nullptr);
 }
 
 int moe_awq_dequant_g32(const int32_t* qweight, const int32_t* qzeros, const void* scales, int batch, int K, int N,

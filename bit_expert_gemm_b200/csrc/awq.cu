@@ -21,7 +21,7 @@ size_t awq_ws_bytes(int rows, int H, int I, int E) {
 int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* offsets, int T, int rows, int H, int I,
                        int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
                        const int32_t* qz_d, const void* sc_d, int dtype, int out_fp32, void* f, void* ws,
-                       size_t ws_bytes, cudaStream_t stream) {
+                       size_t ws_bytes, cudaStream_t stream, const void* awq_packed) {
   (void)T;
   WsCarver carve(ws, ws_bytes);
   void* xp = row_token ? carve.take<uint16_t>(size_t(rows) * H) : nullptr;
@@ -51,7 +51,7 @@ int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* o
   g1.status = device_status_ptr();
   g1.limit_ns = wait_limit_ns();
   int rc = launch_grouped_gemm_awq(a, rows, qw_gu, qz_gu, sc_gu, 2 * I, g1, EPI_SWIGLU, pick_bn(rows, E, I, true),
-                                   stream);
+                                   stream, awq_packed);
   if (rc) return rc;
   GemmArgs g2 = g1;
   g2.K = I;
@@ -60,7 +60,8 @@ int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* o
   g2.out = f;
   g2.ldo = H;
   g2.out_fp32 = out_fp32;
-  return launch_grouped_gemm_awq(h, rows, qw_d, qz_d, sc_d, H, g2, EPI_STORE, pick_bn(rows, E, H, false), stream);
+  return launch_grouped_gemm_awq(h, rows, qw_d, qz_d, sc_d, H, g2, EPI_STORE, pick_bn(rows, E, H, false), stream,
+                                 awq_packed);
 }
 
 // out[b, k, 8w .. 8w+7] = dequantised word (b, k, w); one thread per word.

@@ -15,6 +15,9 @@ constexpr int kDequantThreads = 256;  // 8 AWQ dequantisation warps
 constexpr int kGatherThreads = 128;   // 4 row-gather warps (A rows loaded through row_token)
 constexpr int kStoreStride = 128 + 16;  // epilogue staging: bytes per row of a 32-column chunk, padded
 constexpr int kSmemBudget = 196 * 1024;
+// one unit of the tile-packed AWQ copy (awq.cu): codes, scales and zero
+// points of 64 K rows x 128 output columns
+constexpr int kAwqUnit = 4736;
 
 enum { W_DENSE = 0, W_AWQ = 1, W_AWQ_BF16 = 2 };  // AWQ_BF16: the BF16 mode of the AWQ dequantisation
 
@@ -53,6 +56,10 @@ struct GemmCfg {
                     SCALE_OFF % 128 == 0 && ZERO_OFF % 128 == 0,
                 "every TMA destination must be 128-byte aligned");
   static_assert(W2 * 4 >= 16, "TMA boxes need at least 16 bytes per row");
+  // the tile-packed AWQ path brings BN / 128 units of 4736 bytes into the same staging area
+  static_assert(!WQ || BN < 128 || (TX_BYTES - (AG ? 0 : A_TILE_BYTES) == BN / 128 * 4736 &&
+                                    RAW_BYTES - CODE_OFF >= BN / 128 * 4736),
+                "packed AWQ units must match the staging area");
 };
 
 struct TileMap {
@@ -233,7 +240,25 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ, AG>::THREADS, 1)
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
           if (!AG) tma_load_2d(smA(stage), &tmA, &full_bar[stage], kb * BK, a_row);
-          if (WQ) {
+          if (WQ && args.awq_packed) {
+            // the stage's BN / 128 packed units, contiguous in the staging
+            // area: gate/up unit (j, kb) of column block j, or down unit
+            // (kb, m) of column block m (per expert: J = I/64 column blocks
+            // of H/64 gate/up units, then J K-blocks of H/128 down units)
+            const int Hd = EPI == EPI_SWIGLU ? args.K : args.n_out;
+            const int Iw = EPI == EPI_SWIGLU ? args.n_out : args.K;
+            const int nka = Hd / 64, nkb = Hd / 128, J = Iw / 64;
+            const size_t base = size_t(t.g) * J * (nka + nkb);
+            constexpr int NU = BN / 128;
+#pragma unroll
+            for (int u = 0; u < NU; ++u) {
+              const int c = t.n * NU + u;
+              const size_t unit = base + (EPI == EPI_SWIGLU ? size_t(c) * nka + kb
+                                                            : size_t(J) * nka + size_t(kb) * nkb + c);
+              bulk_load(reinterpret_cast<uint8_t*>(smCodes(stage, 0)) + u * kAwqUnit,
+                        args.awq_packed + unit * kAwqUnit, uint32_t(kAwqUnit), &full_bar[stage]);
+            }
+          } else if (WQ) {
             const int crow = t.g * args.K + kb * BK;          // code rows (input dim)
             const int grow = t.g * (args.K / 32) + kb * (BK / 32);  // scale / zero rows (groups)
             tma_load_2d(smCodes(stage, 0), &bm.codes, &full_bar[stage], col0 / 8, crow);
@@ -438,11 +463,67 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ, AG>::THREADS, 1)
     const int wl = wc - half * W2;
     const uint32_t chunk = uint32_t(wc & 7);
     const uint32_t atom_off = uint32_t(wc >> 3) * Cfg::B_LBO;
+    // packed copy: the unit and its word holding the thread's word column
+    // (a gate/up unit holds 8 gate then 8 up words of one 64-column block)
+    const bool packed = args.awq_packed != nullptr;
+    const int pu = EPI == EPI_SWIGLU ? wl >> 3 : wc >> 4;
+    const int pw = EPI == EPI_SWIGLU ? (wl & 7) + 8 * half : wc & 15;
     int stage = 0;
     uint32_t phase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, lim)) { L = total; break; }
+        constexpr int NR = BK / RP;
+        if constexpr (BN >= 128) {  // the packed copy serves 128- and 256-column tiles
+        if (packed) {
+          // unit layout: codes [r % 16][word][r / 16], scales [group][128], zeros [group][16 words]
+          const uint8_t* ub = reinterpret_cast<const uint8_t*>(smCodes(stage, 0)) + pu * kAwqUnit;
+          const uint4 s0 = *reinterpret_cast<const uint4*>(ub + 4096 + (8 * pw) * 2);
+          const uint4 s1 = *reinterpret_cast<const uint4*>(ub + 4096 + (128 + 8 * pw) * 2);
+          const uint32_t z0 = *reinterpret_cast<const uint32_t*>(ub + 4608 + pw * 4);
+          const uint32_t z1 = *reinterpret_cast<const uint32_t*>(ub + 4608 + (16 + pw) * 4);
+          uint8_t* btile = smB(stage) + atom_off;
+          // rows r0 + 16 i' of the word are one 16-byte piece of the unit:
+          // RP = 16 -> one piece (rows r0 + 16 i), RP = 8 -> two (rows r0 and
+          // r0 + 8 onwards, interleaved); a warp's pieces are consecutive
+          static_assert(RP == 8 || RP == 16, "packed rows per pass: 256- or 128-column tiles");
+          uint32_t cw[NR];
+          {
+            const uint4 a = *reinterpret_cast<const uint4*>(ub + (r0 * 16 + pw) * 16);
+            if constexpr (RP == 16) {
+              cw[0] = a.x;
+              cw[1] = a.y;
+              cw[2] = a.z;
+              cw[3] = a.w;
+            } else {
+              const uint4 b = *reinterpret_cast<const uint4*>(ub + ((r0 + 8) * 16 + pw) * 16);
+              cw[0] = a.x;
+              cw[1] = b.x;
+              cw[2] = a.y;
+              cw[3] = b.y;
+              cw[4] = a.z;
+              cw[5] = b.z;
+              cw[6] = a.w;
+              cw[7] = b.w;
+            }
+          }
+          const AwqGroup g0 = awq_group_paired<WQ == W_AWQ_BF16>(z0, s0),
+                         g1 = awq_group_paired<WQ == W_AWQ_BF16>(z1, s1);
+#pragma unroll
+          for (int i = 0; i < NR; ++i) {
+            const int r = r0 + i * RP;
+            const uint4 v = awq_dequant8_paired<WQ == W_AWQ_BF16>(cw[i], r < 32 ? g0 : g1);
+            const uint32_t off =
+                uint32_t(r >> 3) * Cfg::B_SBO + uint32_t(r & 7) * 128 + ((chunk ^ uint32_t(r & 7)) << 4);
+            *reinterpret_cast<uint4*>(btile + off) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bready_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          continue;
+        }
+        }
         const uint32_t* codes = smCodes(stage, half) + wl;
         const uint16_t* sc = smScales(stage, half) + wl * 8;
         const uint32_t* zr = smZeros(stage, half) + wl;
@@ -452,7 +533,6 @@ __global__ void __launch_bounds__(GemmCfg<BN, EPI, WQ, AG>::THREADS, 1)
         uint8_t* btile = smB(stage) + atom_off;
         // the thread's code words first (loads before any store, so that the
         // rows' conversions overlap), then convert and store
-        constexpr int NR = BK / RP;
         uint32_t cw[NR];
 #pragma unroll
         for (int i = 0; i < NR; ++i) cw[i] = codes[(r0 + i * RP) * W2];
@@ -603,8 +683,11 @@ int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_tot
 }
 
 int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, const int32_t* qzeros,
-                            const void* scales, int n_total, const GemmArgs& args, int epi, int bn,
-                            cudaStream_t stream) {
+                            const void* scales, int n_total, const GemmArgs& args_in, int epi, int bn,
+                            cudaStream_t stream, const void* awq_packed) {
+  GemmArgs args = args_in;
+  // the packed units are 128 columns wide: tile widths 128 and 256 read them
+  args.awq_packed = (awq_packed && bn >= 128) ? static_cast<const uint8_t*>(awq_packed) : nullptr;
   int rc = check_common(args, epi, bn);
   if (rc) return rc;
   MOE_REQUIRE(args.K % 32 == 0, MOE_ERR_UNSUPPORTED, "AWQ K=%d is not a multiple of the group size 32", args.K);

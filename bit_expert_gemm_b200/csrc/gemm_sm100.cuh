@@ -40,6 +40,10 @@ struct GemmArgs {
   const int* row_token;
   const void* a_src;
   int a_src_rows;
+  // AWQ only (optional): the tile-packed copy of the weights (awq.cu
+  // awq_prepack, codes and zero points in pair order); the kernel then reads
+  // it, one bulk copy per 128-column unit, instead of the checkpoint arrays.
+  const uint8_t* awq_packed;
 };
 
 // Host launcher (gemm_sm100.cu).  A [a_rows, K] and B [b_rows_total, K] are
@@ -55,8 +59,10 @@ int launch_grouped_gemm(const void* A, int a_rows, const void* B, int b_rows_tot
 // exactly fp16_rn((q-z)*s) with FP16 operands (args.bf16 = 0), or
 // bf16_rn((q-z)*bf16_rn(s)) in the BF16 mode (args.bf16 = 1).  args.up_offset is the column of the up
 // half (SwiGLU); args.b_rows_per_group is unused.
+// awq_packed (may be NULL): the tile-packed copy of the same weights, read
+// instead of them for tile widths 128 and 256.
 int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, const int32_t* qzeros,
                             const void* scales, int n_total, const GemmArgs& args, int epi, int bn,
-                            cudaStream_t stream);
+                            cudaStream_t stream, const void* awq_packed = nullptr);
 
 }  // namespace moe

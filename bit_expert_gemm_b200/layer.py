@@ -84,9 +84,10 @@ class MoELayer:
             self.I = weights["w_gate_up"].shape[1] // 2
         elif fmt == "awq_g32":
             self.I = weights["qw_gu"].shape[2] * 8 // 2
-            if T_max <= 16 and "awq_packed" not in weights:
-                # decode-sized layer: the routed weights also tile-packed, so that the
-                # weight-streaming kernel fetches each sub-tile with one bulk copy
+            if "awq_packed" not in weights:
+                # the routed weights also tile-packed: the decode kernel fetches each
+                # sub-tile, the grouped GEMMs each 128-column unit, with one bulk copy,
+                # and both dequantise the pair-ordered codes without byte permutes
                 self.w = weights = dict(weights)
                 weights["awq_packed"] = abi.moe_awq_prepack_g32(weights["qw_gu"], weights["qz_gu"], weights["sc_gu"],
                                                                 weights["qw_d"], weights["qz_d"], weights["sc_d"])

@@ -357,7 +357,9 @@ MOE_API int moe_awq_prepack_g32(const int32_t* qw_gu, const int32_t* qz_gu, cons
  * moe_experts_awq_g32 with the routed weights also given tile-packed
  * (awq_packed, from moe_awq_prepack_g32 on the same qw/qz/sc): for T <= 16
  * the decode kernel reads only awq_packed (one bulk copy per sub-tile
- * instead of six tensor-map boxes); larger T reads qw/qz/sc as before.
+ * instead of six tensor-map boxes); larger T reads awq_packed too in the
+ * grouped GEMMs whose tiles are 128 or 256 columns wide (one bulk copy per
+ * 128-column unit), qw/qz/sc otherwise.
  * Results are identical to moe_experts_awq_g32's.  All other arguments,
  * limits and the workspace as there; awq_packed must not be NULL.
  * ------------------------------------------------------------------------- */
