@@ -22,20 +22,27 @@ int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* o
                        int E, const int32_t* qw_gu, const int32_t* qz_gu, const void* sc_gu, const int32_t* qw_d,
                        const int32_t* qz_d, const void* sc_d, int dtype, int out_fp32, void* f, void* ws,
                        size_t ws_bytes, cudaStream_t stream, const void* awq_packed) {
-  (void)T;
   WsCarver carve(ws, ws_bytes);
   void* xp = row_token ? carve.take<uint16_t>(size_t(rows) * H) : nullptr;
   uint16_t* h = carve.take<uint16_t>(size_t(rows) * I);
   MOE_REQUIRE(carve.ok, MOE_ERR_WORKSPACE, "moe_grouped_swiglu_awq_g32: workspace of %zu bytes is too small",
               ws_bytes);
   if (rows == 0) return MOE_OK;
+  // with the packed copy GEMM1 gathers its A rows (x[row_token[r]]) itself;
+  // otherwise they are gathered into xp first
   const void* a = x;
-  if (row_token) {
+  const bool gather_in_gemm = row_token && awq_packed;
+  if (row_token && !gather_in_gemm) {
     int rc = gather_rows(x, row_token, rows, H, xp, stream);
     if (rc) return rc;
     a = xp;
   }
   GemmArgs g1{};
+  if (gather_in_gemm) {
+    g1.row_token = row_token;
+    g1.a_src = x;
+    g1.a_src_rows = T;
+  }
   g1.group_offsets = offsets;
   g1.G = E;
   g1.rows = rows;
@@ -54,6 +61,9 @@ int grouped_swiglu_awq(const void* x, const int32_t* row_token, const int32_t* o
                                    stream, awq_packed);
   if (rc) return rc;
   GemmArgs g2 = g1;
+  g2.row_token = nullptr;  // GEMM2 reads h in the permuted order
+  g2.a_src = nullptr;
+  g2.a_src_rows = 0;
   g2.K = I;
   g2.n_out = H;
   g2.up_offset = 0;

@@ -697,7 +697,15 @@ int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, c
   CUtensorMap ta;
   BMaps bm;
   memset(&bm, 0, sizeof(bm));
-  rc = make_tmap_16bit_sw128(&ta, A, a_rows, args.K, BM);
+  if (args.row_token) {
+    // A rows gathered in the kernel (x[row_token[r]]); the map over the source only keeps the parameter valid
+    MOE_REQUIRE(args.a_src != nullptr && args.a_src_rows > 0, MOE_ERR_INVALID_ARG, "gathered GEMM without a source");
+    MOE_REQUIRE((reinterpret_cast<uintptr_t>(args.a_src) & 15) == 0, MOE_ERR_INVALID_ARG,
+                "gathered rows are not 16-byte aligned");
+    rc = make_tmap_16bit_sw128(&ta, args.a_src, args.a_src_rows, args.K, BM);
+  } else {
+    rc = make_tmap_16bit_sw128(&ta, A, a_rows, args.K, BM);
+  }
   if (rc) return rc;
   const int G = args.G;
   rc = make_tmap_2d(&bm.codes, qweight, G * args.K, n_total / 8, 4, BK, bnh / 8, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -706,7 +714,10 @@ int launch_grouped_gemm_awq(const void* A, int a_rows, const int32_t* qweight, c
   if (rc) return rc;
   rc = make_tmap_2d(&bm.zeros, qzeros, G * (args.K / 32), n_total / 8, 4, 2, bnh / 8, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
-  MOE_REQUIRE(args.row_token == nullptr, MOE_ERR_UNSUPPORTED, "AWQ GEMM reads pre-gathered rows");
+  if (args.row_token) {
+    if (args.bf16) return dispatch<W_AWQ_BF16, 1>(ta, bm, args, epi, bn, stream);
+    return dispatch<W_AWQ, 1>(ta, bm, args, epi, bn, stream);
+  }
   if (args.bf16) return dispatch<W_AWQ_BF16, 0>(ta, bm, args, epi, bn, stream);
   return dispatch<W_AWQ, 0>(ta, bm, args, epi, bn, stream);
 }
