@@ -338,7 +338,7 @@ MOE_API int moe_experts_awq_g32(const void* x, const int32_t* row_token, const i
 
 /* ---------------------------------------------------------------------------
  * Tile-packed copy of one layer's routed AWQ weights [AWQ], made once, for
- * the T <= 16 path of moe_experts_awq_g32_prepacked: the same codes, zero
+ * moe_experts_awq_g32_prepacked (decode and prefill): the same codes, zero
  * points and scales (no value changes, same total size) regrouped so that
  * every 64-input-row sub-tile the decode kernel streams is one contiguous
  * 4736-byte unit.  Inputs as in moe_grouped_swiglu_awq_g32; out: device
@@ -359,7 +359,8 @@ MOE_API int moe_awq_prepack_g32(const int32_t* qw_gu, const int32_t* qz_gu, cons
  * the decode kernel reads only awq_packed (one bulk copy per sub-tile
  * instead of six tensor-map boxes); larger T reads awq_packed too in the
  * grouped GEMMs whose tiles are 128 or 256 columns wide (one bulk copy per
- * 128-column unit), qw/qz/sc otherwise.
+ * 128-column unit), qw/qz/sc otherwise, and its GEMM1 gathers the x rows
+ * through row_token itself (no separate gather launch).
  * Results are identical to moe_experts_awq_g32's.  All other arguments,
  * limits and the workspace as there; awq_packed must not be NULL.
  * ------------------------------------------------------------------------- */
