@@ -13,7 +13,7 @@ import torch
 from bit_expert_gemm_b200 import MoELayer, abi, synth
 from bit_expert_gemm_b200.layer import prepare_nvfp4_weights, slice_layer_weights
 from oracle import moe, razor
-from tests.helpers import expert_fn_bf16, f64, rel_err, shared_fn
+from tests.helpers import f64, rel_err, shared_fn
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
