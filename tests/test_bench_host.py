@@ -33,3 +33,18 @@ def test_expert_flops_and_default_traffic():
     assert src is not None and "moe_layer_bf16_prefill_t8192.md" in src
     assert traffic is None or traffic > 2e9  # the expert call moves at least the touched experts' 2.1 GB
     assert bench.measured_traffic("no_such_workload") == (None, None)
+
+
+def test_clock_record_rules():
+    # hardware or thermal slowdowns reject the timed region; a power cap alone is kept
+    ok = {"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": []}
+    assert not bench.clocks_rejected(ok)
+    assert not bench.clocks_rejected({**ok, "sm_mhz": 1335.0, "reasons": ["sw_power_cap"]})
+    for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clocks_rejected({**ok, "reasons": [r]})
+        assert bench.clocks_rejected({**ok, "reasons": ["sw_power_cap", r]})
+    # clocks well below the maximum with no reason: a clock lock left on the GPU
+    assert bench.clocks_rejected({**ok, "sm_mhz": 1200.0})
+    assert not bench.clocks_rejected({**ok, "sm_mhz": 1900.0})
+    # no NVML: nothing to judge
+    assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["NVML unavailable: x"]})
