@@ -144,8 +144,10 @@ MOE_API int moe_route_topk(const void* x, int T, int H, const void* w_router, co
                    size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Permutation of the (token, slot) assignments by expert: histogram,
- * exclusive scan, scatter.  The order is deterministic: expert blocks in
+ * Permutation of the (token, slot) assignments by expert, so that each
+ * routed expert [ARCH] ("Routed experts selected per token") runs once over
+ * the rows of all tokens that selected it: histogram, exclusive scan,
+ * scatter.  The pages fix no order; this one is deterministic: expert blocks in
  * ascending expert id, and inside one expert ascending token index (every
  * token selects an expert at most once).
  *
@@ -162,7 +164,8 @@ MOE_API int moe_permute(const int32_t* topk_idx, int T, int k_slots, int E, int3
 
 /* ---------------------------------------------------------------------------
  * moe_route_topk followed by moe_permute of its topk_idx (k_slots = k +
- * extra), in one call, with the arguments and outputs of both.  For T <= 128
+ * extra), in one call, with the arguments and outputs of both ([ARCH]
+ * gating and selection; [RAZOR] rank k + 1 when extra = 1).  For T <= 128
  * (decode) everything runs in one cooperative kernel (grid-wide barriers
  * between the logits, the top-k and the permutation); larger T takes the two
  * calls' kernels in sequence.  Outputs equal those of the two calls, except
@@ -439,8 +442,8 @@ MOE_API int moe_nvfp4_prepack_sf(const uint8_t* sf, int E, int rows_per_expert, 
                                  size_t out_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
- * moe_grouped_swiglu_nvfp4 with the weight scales given already rearranged
- * by moe_nvfp4_prepack_sf (sf_gu_packed from sf_gu with swiglu = 1,
+ * moe_grouped_swiglu_nvfp4 [NVFP4] with the weight scales given already
+ * rearranged by moe_nvfp4_prepack_sf (sf_gu_packed from sf_gu with swiglu = 1,
  * rows_per_expert = 2I, K = H; sf_d_packed from sf_d with swiglu = 0,
  * rows_per_expert = H, K = I).  Results are identical to
  * moe_grouped_swiglu_nvfp4's; all other arguments, limits and the workspace
