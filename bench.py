@@ -309,8 +309,9 @@ EXPERT_KEYS = {"bf16": ("w_gate_up", "w_down"), "awq_g32": ("qw_gu", "qz_gu", "s
                "nvfp4": ("w_gu", "sf_gu", "gs_gu", "w_d", "sf_d", "gs_d")}
 KERNEL_NAMES = {"bf16": "moe_experts_bf16 (routed + shared experts: GEMM1/SwiGLU + GEMM2, tcgen05 kind::f16; "
                         "decode-sized batches stream the weights as the M operand)",
-                "awq_g32": "moe_grouped_swiglu_awq_g32 (row gather + dequantising GEMM1/SwiGLU + GEMM2, tcgen05 "
-                           "kind::f16)",
+                "awq_g32": "moe_experts_awq_g32_prepacked (routed AWQ experts from the tile-packed copy: "
+                           "dequantising GEMM1/SwiGLU gathering its x rows + dequantising GEMM2, tcgen05 kind::f16; "
+                           "T <= 16: the split-K weight-streaming kernel; + the FP16 shared expert)",
                 "nvfp4": "moe_grouped_swiglu_nvfp4_prepacked (activation quantisation + GEMM1/SwiGLU + h "
                          "quantisation + GEMM2: tcgen05 kind::mxf4nvf4; T <= 16: CUDA-core GEMVs with exact dp4a "
                          "group products) + the BF16 shared expert (T <= 16: weight-streaming GEMVs on a second "

@@ -48,3 +48,27 @@ def test_clock_record_rules():
     assert not bench.clocks_rejected({**ok, "sm_mhz": 1900.0})
     # no NVML: nothing to judge
     assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["NVML unavailable: x"]})
+
+
+def test_every_traffic_line_names_existing_sources():
+    # each committed traffic line parses, names kernel sources that exist, and
+    # is found by measured_traffic for its workload (a renamed source would
+    # otherwise turn the figure into a silent null)
+    import glob
+    import re
+    pat = re.compile(r"traffic: workload=(\S+) bytes_per_launch=(\d+) sources=(\S+) sha256=([0-9a-f]+)")
+    seen = set()
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        for line in open(path):
+            m = pat.search(line)
+            if not m:
+                continue
+            wk, nbytes, srcs = m.group(1), int(m.group(2)), m.group(3).split(",")
+            assert wk in bench.WORKLOADS, wk
+            assert nbytes > 0
+            for f in srcs:
+                assert os.path.isfile(os.path.join(ROOT, "bit_expert_gemm_b200", "csrc", f)), (path, f)
+            assert bench.measured_traffic(wk)[1] is not None
+            seen.add(wk)
+    assert {"bf16_prefill", "bf16_decode_t1", "awq_decode_t1", "awq_prefill", "nvfp4_prefill",
+            "nvfp4_decode_t1"} <= seen
