@@ -393,7 +393,9 @@ def moe_awq_prepack_g32(qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d, out=None, stream=
 def moe_experts_awq_g32_prepacked(x, row_token, expert_offsets, rows: int, qw_gu, qz_gu, sc_gu, qw_d, qz_d, sc_d,
                                   awq_packed, w_sh_gate_up, w_sh_down, out_fp32: bool = False, f=None,
                                   shared_out=None, ws=None, stream=None):
-    """moe_experts_awq_g32 with the routed weights also tile-packed (read by the T <= 16 path)."""
+    """moe_experts_awq_g32 with the routed weights also tile-packed: the decode kernel reads only the packed
+    copy, the grouped prefill GEMMs read it for 128- and 256-column tiles and then gather the x rows
+    themselves."""
     T, H = x.shape
     E = qw_gu.shape[0]
     I = qw_gu.shape[2] * 8 // 2

@@ -64,7 +64,7 @@ def main(argv=None) -> None:
             abi.moe_grouped_swiglu_nvfp4_prepacked(xb, rt, off, rows, w["w_gu"], w["sfp_gu"], w["gs_gu"], w["w_d"],
                                                    w["sfp_d"], w["gs_d"])
     elif a.fmt == "awq_g32":
-        # as MoELayer does: decode-sized calls read the tile-packed copy of the routed weights
+        # as MoELayer does: the expert call reads the tile-packed copy of the routed weights
         packed = abi.moe_awq_prepack_g32(w["qw_gu"], w["qz_gu"], w["sc_gu"], w["qw_d"], w["qz_d"], w["sc_d"])
 
         def call():
