@@ -185,6 +185,9 @@ def test_select_bit_exact(E):
     (1, 2048, 640, 512, 10, False, "bf16"), (2, 512, 128, 16, 4, True, "bf16"), (4, 256, 256, 16, 3, False, "f16"),
     (3, 512, 384, 32, 2, False, "bf16"), (8, 512, 128, 16, 4, False, "bf16"), (3, 256, 64, 16, 2, False, "bf16"),
     (16, 1024, 192, 64, 6, True, "bf16"), (5, 384, 128, 32, 4, False, "f16"),
+    # the split-K kernel at its widest H (28 blocks of 128 rows in TMEM) and at the fact sheet's 2560;
+    # above 3584 the two weight-streaming GEMMs serve T <= 16 too
+    (4, 3584, 256, 16, 4, True, "bf16"), (1, 2560, 640, 64, 10, False, "bf16"), (2, 4096, 128, 16, 3, False, "f16"),
     # 16 < T <= 128: two weight-streaming GEMMs
     (17, 512, 128, 16, 3, False, "bf16"), (64, 2048, 640, 64, 10, True, "bf16"), (128, 256, 64, 16, 2, False, "bf16"),
     # T > 128: the grouped prefill GEMMs
