@@ -216,3 +216,22 @@ def test_expert_parallel_refill_statistics(world):
     for rank in range(world):
         assert np.array_equal(res[f"c{rank}"], c_ref), rank
         assert np.allclose(res[f"s{rank}"], s_ref, rtol=1e-12, atol=0), rank
+
+
+def test_expert_parallel_rejects_bad_splits():
+    # the contiguous expert ranges need E % world == 0; extra is 0 or 1; a
+    # rank's slice of the expert weights must hold E / world experts
+    from bit_expert_gemm_b200 import ep
+
+    w = _weights(E, H, I, 7)
+    with pytest.raises(ValueError, match="multiple"):
+        ep.ExpertParallelLayer(w, K, 0, 3, T_max=8, ops=OracleOps(), device=torch.device("cpu"))
+    with pytest.raises(ValueError, match="extra"):
+        ep.ExpertParallelLayer(w, K, 0, 2, T_max=8, ops=OracleOps(), device=torch.device("cpu"), extra=2)
+    part = dict(w, w_gate_up=w["w_gate_up"][:3], w_down=w["w_down"][:3])
+    with pytest.raises(ValueError, match="E/world"):
+        ep.ExpertParallelLayer(part, K, 0, 2, T_max=8, ops=OracleOps(), device=torch.device("cpu"))
+    # a rank given only its own slice keeps it as is
+    own = dict(w, w_gate_up=w["w_gate_up"][8:16], w_down=w["w_down"][8:16])
+    layer = ep.ExpertParallelLayer(own, K, 1, 2, T_max=8, ops=OracleOps(), device=torch.device("cpu"))
+    assert torch.equal(layer.w["w_gate_up"], w["w_gate_up"][8:16])
