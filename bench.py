@@ -629,11 +629,7 @@ def bench_workload(args, dist: Dist, workload: str, with_e2e: bool = True, with_
                                                                  "(AWQ g32)",
                                        "nvfp4": "fp4 e2m1 x fp4 e2m1 (NVFP4)"}[wl.fmt],
         "data": "synthetic (seeded N(0,1) tokens, N(0,1/sqrt(fan_in)) weights)",
-        "config": {"workload": f"{workload}: T={T} H={wl.H} E={wl.E} k={wl.k} I={wl.I} shared={wl.I_sh} "
-                               f"fmt={wl.fmt}" + (" +Refill-RMS accumulate/select" if kind == "refill" else "")
-                               + (f" (RAZOR-pruned from {wl_full.E} experts: Refill-RMS over one {CALIBRATION_T}-token "
-                                  f"calibration row, top {keep} kept, sliced on the device)" if keep else ""),
-                   "tokens_per_step_per_gpu": T, "parallelism": f"dp{dist.world} (replicas, no collective)",
+        "config": {"workload": workload_label(workload), "tokens_per_step_per_gpu": T, "parallelism": f"dp{dist.world} (replicas, no collective)",
                    "launch": "eager C-ABI calls" if args.no_graph else "one CUDA graph per step (the C-ABI calls)",
                    "l2": (f"{n_units} layers with distinct weights in rotation ({layer_bytes / 2**30:.2f} GiB each); "
                           "between two uses of a layer the others stream >= 3x the 126 MB L2 of expert weights, "
@@ -695,12 +691,28 @@ def run_native(args, dist: Dist) -> None:
         print(json.dumps(line), flush=True)
 
 
+def workload_label(workload: str) -> str:
+    """The workload as both arms name it in their JSON line's config."""
+    wname, T, kind = WORKLOADS[workload]
+    wl = synth.WORKLOADS[wname]
+    keep = PRUNED.get(workload, 0)
+    label = (f"{workload}: T={T} H={wl.H} E={keep or wl.E} k={wl.k} I={wl.I} shared={wl.I_sh} fmt={wl.fmt}"
+             + (" +Refill-RMS accumulate/select" if kind == "refill" else ""))
+    if keep:
+        label += (f" (RAZOR-pruned from {wl.E} experts: Refill-RMS over one {CALIBRATION_T}-token calibration row, "
+                  f"top {keep} kept, sliced on the device)")
+    return label
+
+
 def run_reference(args, dist: Dist) -> None:
     """The CPU oracle as the reference arm, rank 0 only."""
     if dist.rank != 0:
         return
     wname, T, kind = WORKLOADS[args.workload]
     wl = synth.WORKLOADS[wname]
+    keep = PRUNED.get(args.workload, 0)
+    if keep:  # a layer of the pruned shape, seeded weights (the selection itself is not timed)
+        wl = dataclasses.replace(wl, E=keep)
     dev = torch.device("cuda", dist.local) if torch.cuda.is_available() else torch.device("cpu")
     w = synth.make_weights(wl, seed=0, device=dev)
     x = synth.make_tokens(wl, T, seed=1, device=dev)
@@ -718,10 +730,10 @@ def run_reference(args, dist: Dist) -> None:
         "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"{args.workload}: T={T} H={wl.H} E={wl.E} k={wl.k} I={wl.I} shared={wl.I_sh} "
-                               f"fmt={wl.fmt}", "tokens_per_step_per_gpu": n},
+        "config": {"workload": workload_label(args.workload), "tokens_per_step_per_gpu": n},
         "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                         "sample": f"{n} tokens per step of the same workload, float64 NumPy"},
+                         "sample": f"{n} tokens per step of the same workload, float64 NumPy"
+                                   + (f" (a layer of the pruned shape, E={keep}, seeded weights)" if keep else "")},
         "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -72,3 +72,14 @@ def test_every_traffic_line_names_existing_sources():
             seen.add(wk)
     assert {"bf16_prefill", "bf16_decode_t1", "awq_decode_t1", "awq_prefill", "nvfp4_prefill",
             "nvfp4_decode_t1"} <= seen
+
+
+def test_workload_labels():
+    # both arms name a workload with the same label; pruned workloads state the kept expert count
+    for name, (wname, T, kind) in bench.WORKLOADS.items():
+        label = bench.workload_label(name)
+        assert label.startswith(f"{name}: T={T} ")
+        assert ("Refill-RMS accumulate" in label) == (kind == "refill")
+    for name, keep in bench.PRUNED.items():
+        assert f" E={keep} " in bench.workload_label(name)
+    assert bench.workload_label("bf16_prefill") == "bf16_prefill: T=8192 H=2048 E=512 k=10 I=640 shared=640 fmt=bf16"
