@@ -629,7 +629,8 @@ def bench_workload(args, dist: Dist, workload: str, with_e2e: bool = True, with_
                                                                  "(AWQ g32)",
                                        "nvfp4": "fp4 e2m1 x fp4 e2m1 (NVFP4)"}[wl.fmt],
         "data": "synthetic (seeded N(0,1) tokens, N(0,1/sqrt(fan_in)) weights)",
-        "config": {"workload": workload_label(workload), "tokens_per_step_per_gpu": T, "parallelism": f"dp{dist.world} (replicas, no collective)",
+        "config": {"workload": workload_label(workload), "tokens_per_step_per_gpu": T,
+                   "parallelism": f"dp{dist.world} (replicas, no collective)",
                    "launch": "eager C-ABI calls" if args.no_graph else "one CUDA graph per step (the C-ABI calls)",
                    "l2": (f"{n_units} layers with distinct weights in rotation ({layer_bytes / 2**30:.2f} GiB each); "
                           "between two uses of a layer the others stream >= 3x the 126 MB L2 of expert weights, "
